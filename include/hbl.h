@@ -1,0 +1,160 @@
+/*
+ * hbl.h -- C ABI of the B200 (sm_100a) H-BitLinear forward library.
+ *
+ * The layer is the H-BitLinear module of "BitNet v2: Native 4-bit
+ * Activations with Hadamard Transformation for 1-bit LLMs" (arXiv 2504.18415;
+ * section "H-BitLinear", the matrix-operation formula Y = Q(H(LN(X))) . Qw(W)).
+ * Per token row of length K it computes
+ *   1. LN: plain LayerNorm, no affine, eps_ln = 1e-5, biased variance;
+ *   2. H : the Sylvester-order Walsh-Hadamard transform of length K (a power of
+ *          two) scaled by 1/sqrt(K), computed as a fast Hadamard transform;
+ *   3. Q : per-token activation quantization, INT4 absmean
+ *          (beta = mean|t|, q = clip(rint(sqrt(7) t/(beta+eps)), -8, 7),
+ *          scale = beta/sqrt(7)) or INT8 absmax (gamma = max|t|,
+ *          q = clip(rint(127 t/(gamma+eps)), -128, 127), scale = gamma/127);
+ *   4. an exact integer GEMM with the ternary weight codes, int32 accumulation;
+ *   5. dequantisation y[m][n] = (float)acc[m][n] * (scale[m] * alpha).
+ * Weights are ternarised once by per-tensor absmean (alpha = mean|W|,
+ * w = clip(rint(W/(alpha+eps)), -1, 1)).  eps = 1e-5; rint rounds half to even.
+ *
+ * Conventions for every entry point:
+ *  - All memory is owned by the caller.  Pointers marked "device" must point
+ *    to device memory of the current CUDA device, 16-byte aligned.  The library
+ *    never allocates or frees memory, never synchronises the stream (except
+ *    hbl_last_device_error) and keeps no state between calls other than the
+ *    device error word read by hbl_last_device_error.
+ *  - Work is enqueued on `stream` (0 = legacy default stream) and is
+ *    asynchronous; outputs are valid once the stream reaches that point.
+ *  - Arguments are checked on the host before any launch.  A failed check
+ *    returns an error status and enqueues nothing.  Launch failures return
+ *    HBL_ERR_CUDA.  Nothing traps, asserts or exits.
+ *  - Supported sizes: K a power of two with 64 <= K <= 32768; M >= 1;
+ *    N >= 16 and a multiple of 16 (forward, ternary packing).
+ *  - Row-major layouts throughout.  x is [M][K]; W is [N][K] (out x in, the
+ *    layout of a PyTorch Linear weight); y is [M][N].
+ */
+#ifndef HBL_H_
+#define HBL_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  HBL_OK = 0,
+  HBL_ERR_INVALID_ARG = 1, /* null pointer, non-positive size, bad bits/dtype, misaligned */
+  HBL_ERR_UNSUPPORTED = 2, /* a size outside the supported set (e.g. K not a power of two) */
+  HBL_ERR_WORKSPACE = 3,   /* workspace pointer null or smaller than required */
+  HBL_ERR_CUDA = 4,        /* a CUDA runtime call or launch failed */
+  HBL_ERR_TIMEOUT = 5      /* a kernel gave up a bounded wait (see hbl_last_device_error) */
+} hbl_status;
+
+typedef enum { HBL_F32 = 0, HBL_BF16 = 1 } hbl_dtype;
+
+/* ---------------------------------------------------------------- sizes */
+
+/* Bytes of the packed ternary weight: N rows of K/4 bytes (2 bits per code:
+ * element 4j+i of a row sits at bits 2i..2i+1 of byte j; 00 = 0, 01 = +1,
+ * 11 = -1).  Returns 0 for invalid sizes. */
+size_t hbl_packed_ternary_bytes(int64_t K, int64_t N);
+
+/* Bytes of activation codes for M rows: bits = 4 -> M*K/2 (two's-complement
+ * nibbles, element 2j of a row in the low nibble of byte j, 2j+1 in the high
+ * nibble); bits = 8 -> M*K (int8).  Returns 0 for invalid arguments. */
+size_t hbl_codes_bytes(int64_t M, int64_t K, int bits);
+
+/* Workspace bytes needed by hbl_pack_ternary (partial sums of |W|). */
+size_t hbl_pack_ternary_workspace_bytes(int64_t K, int64_t N);
+
+/* Workspace bytes needed by hbl_forward: int8 activation codes [M][K],
+ * per-row scales [M] and the int8 weight codes [N][K] the tensor cores read.
+ * Returns 0 for invalid arguments. */
+size_t hbl_forward_workspace_bytes(int64_t M, int64_t K, int64_t N, int bits);
+
+/* ---------------------------------------------------------------- compute */
+
+/* Ternary weight quantization ("per-tensor absmean quantizes the weights to
+ * {-1, 0, 1}"; weight-quantization formula of section "H-BitLinear").
+ *   W         device, [N][K] of dtype wt (HBL_F32 or HBL_BF16)
+ *   packed    device, hbl_packed_ternary_bytes(K, N) bytes (output)
+ *   alpha_dev device, one float (output): alpha = mean|W| (accumulated in
+ *             double, rounded once to float)
+ *   workspace device, >= hbl_pack_ternary_workspace_bytes(K, N) bytes
+ * Codes: w = clip(rint(W * (1/(alpha+eps))), -1, 1), the reciprocal one float
+ * division, the product one float multiply. */
+hbl_status hbl_pack_ternary(const void* W, hbl_dtype wt, int64_t K, int64_t N, uint8_t* packed,
+                            float* alpha_dev, void* workspace, size_t workspace_bytes,
+                            cudaStream_t stream);
+
+/* LN -> H -> per-token quantization of M rows (the activation path of
+ * H-BitLinear: LayerNorm, online Hadamard transformation, then "per-token
+ * absmean (4-bit) / absmax (8-bit)" quantization).
+ *   x      device, [M][K] of dtype xt
+ *   bits   4 or 8
+ *   codes  device, hbl_codes_bytes(M, K, bits) bytes (output, layout above)
+ *   scales device, M floats (output): beta/sqrt(7) (bits 4) or gamma/127
+ *          (bits 8) per row
+ * Per row: beta (or gamma) from the float transform output t; the mean of |t|
+ * is accumulated in double and rounded once to float; r = c/(stat+eps) is one
+ * float division (c = sqrt(7) rounded to float, or 127); q = rint(t*r),
+ * clipped. */
+hbl_status hbl_fht_quant(const void* x, hbl_dtype xt, int64_t M, int64_t K, int bits,
+                         uint8_t* codes, float* scales, cudaStream_t stream);
+
+/* Whole H-BitLinear forward: y = dequant(Q(H(LN(x))) . w^T).
+ *   x          device, [M][K] of dtype xt
+ *   packed     device, packed ternary weight from hbl_pack_ternary ([N][K/4])
+ *   alpha_dev  device, the float alpha written by hbl_pack_ternary
+ *   bits       4 or 8
+ *   y          device, [M][N] of dtype yt (HBL_F32 or HBL_BF16, round to
+ *              nearest even): y = (float)acc * (scale[m] * alpha)
+ *   workspace  device, >= hbl_forward_workspace_bytes(M, K, N, bits) bytes,
+ *              256-byte aligned; its contents are scratch
+ * The integer GEMM runs on the tcgen05 tensor cores (kind::i8) with exact
+ * int32 accumulation. */
+hbl_status hbl_forward(const void* x, hbl_dtype xt, int64_t M, int64_t K, const uint8_t* packed,
+                       const float* alpha_dev, int64_t N, int bits, void* y, hbl_dtype yt,
+                       void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* ---------------------------------------------------------------- test hooks */
+
+/* Stages 1-2 alone: t = H LN(x) / sqrt(K) as float [M][K] (device output).
+ * The same kernel code as hbl_fht_quant up to the quantizer. */
+hbl_status hbl_debug_ln_fht(const void* x, hbl_dtype xt, int64_t M, int64_t K, float* t,
+                            cudaStream_t stream);
+
+/* Stage 3 alone on given float rows t [M][K] (device): the same quantizer as
+ * hbl_fht_quant.  K any multiple of 16 in [16, 65536]. */
+hbl_status hbl_quant_from_f32(const float* t, int64_t M, int64_t K, int bits, uint8_t* codes,
+                              float* scales, cudaStream_t stream);
+
+/* Integer GEMM alone: acc[m][n] = sum_k A[m][k] * B[n][k] (exact int32) on the
+ * tcgen05 tensor cores.  A device int8 [M][K], B device int8 [N][K],
+ * acc device int32 [M][N]; K a multiple of 16, N a multiple of 16. */
+hbl_status hbl_gemm_i8_i32(const int8_t* A, const int8_t* B, int64_t M, int64_t N, int64_t K,
+                           int32_t* acc, cudaStream_t stream);
+
+/* ---------------------------------------------------------------- errors */
+
+/* Synchronises `stream`, then reports and clears the device error word that
+ * kernels set when a bounded wait runs out: HBL_ERR_TIMEOUT if one did,
+ * HBL_ERR_CUDA if the synchronisation failed, else HBL_OK. */
+hbl_status hbl_last_device_error(cudaStream_t stream);
+
+/* Sets the device error word as a kernel would on a bounded-wait timeout
+ * (used by the tests of the error path; enqueued on `stream`). */
+hbl_status hbl_debug_raise_device_error(cudaStream_t stream);
+
+/* Static string for a status code. */
+const char* hbl_status_string(hbl_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HBL_H_ */
