@@ -1,1 +1,225 @@
-"""B200-native H-BitLinear forward (BitNet v2): CUDA kernels behind a C ABI."""
+"""B200-native H-BitLinear forward (BitNet v2): CUDA kernels behind a C ABI.
+
+The functions below carry the names of the C entry points in include/hbl.h and
+only marshal arguments: torch tensors supply device memory and the current
+CUDA stream, every step of the computation runs in libhbl.so.  Outputs that
+the caller does not pass are allocated here with torch (the library itself
+never allocates).  If libhbl.so is missing or fails to load, every call raises
+-- there is no CPU fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+import threading
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libhbl.so")
+HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "hbl.h")
+
+HBL_OK, HBL_ERR_INVALID_ARG, HBL_ERR_UNSUPPORTED, HBL_ERR_WORKSPACE, HBL_ERR_CUDA, HBL_ERR_TIMEOUT = range(6)
+HBL_F32, HBL_BF16 = 0, 1
+
+_lock = threading.Lock()
+_lib = None
+
+
+class HBLError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__("%s failed: %s" % (where, status_string(status)))
+
+
+def declared_symbols():
+    """Names of the functions declared in include/hbl.h."""
+    text = open(HEADER_PATH).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(hbl_[a-z0-9_]+)\s*\(", text)))
+
+
+def lib():
+    """The loaded libhbl.so (ctypes); raises if it is not built."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise ImportError("libhbl.so is not built (run python -m ternary_gemm_b200.build); "
+                                  "there is no fallback path")
+            L = ctypes.CDLL(LIB_PATH)
+            p, i64, i32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
+            L.hbl_packed_ternary_bytes.argtypes = [i64, i64]
+            L.hbl_packed_ternary_bytes.restype = sz
+            L.hbl_codes_bytes.argtypes = [i64, i64, i32]
+            L.hbl_codes_bytes.restype = sz
+            L.hbl_pack_ternary_workspace_bytes.argtypes = [i64, i64]
+            L.hbl_pack_ternary_workspace_bytes.restype = sz
+            L.hbl_forward_workspace_bytes.argtypes = [i64, i64, i64, i32]
+            L.hbl_forward_workspace_bytes.restype = sz
+            L.hbl_pack_ternary.argtypes = [p, i32, i64, i64, p, p, p, sz, p]
+            L.hbl_pack_ternary.restype = i32
+            L.hbl_fht_quant.argtypes = [p, i32, i64, i64, i32, p, p, p]
+            L.hbl_fht_quant.restype = i32
+            L.hbl_forward.argtypes = [p, i32, i64, i64, p, p, i64, i32, p, i32, p, sz, p]
+            L.hbl_forward.restype = i32
+            L.hbl_debug_ln_fht.argtypes = [p, i32, i64, i64, p, p]
+            L.hbl_debug_ln_fht.restype = i32
+            L.hbl_quant_from_f32.argtypes = [p, i64, i64, i32, p, p, p]
+            L.hbl_quant_from_f32.restype = i32
+            L.hbl_gemm_i8_i32.argtypes = [p, p, i64, i64, i64, p, p]
+            L.hbl_gemm_i8_i32.restype = i32
+            L.hbl_last_device_error.argtypes = [p]
+            L.hbl_last_device_error.restype = i32
+            L.hbl_debug_raise_device_error.argtypes = [p]
+            L.hbl_debug_raise_device_error.restype = i32
+            L.hbl_status_string.argtypes = [i32]
+            L.hbl_status_string.restype = ctypes.c_char_p
+            _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().hbl_status_string(int(status)).decode()
+
+
+def _check(status: int, where: str):
+    if status != HBL_OK:
+        raise HBLError(status, where)
+
+
+def _torch():
+    import torch
+    return torch
+
+
+def _stream(stream):
+    torch = _torch()
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dtype_code(t) -> int:
+    torch = _torch()
+    if t.dtype == torch.float32:
+        return HBL_F32
+    if t.dtype == torch.bfloat16:
+        return HBL_BF16
+    raise TypeError("expected float32 or bfloat16, got %s" % t.dtype)
+
+
+def _ptr(t) -> ctypes.c_void_p:
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError("tensors must be contiguous CUDA tensors")
+
+
+# ------------------------------------------------------------------ sizes
+
+def hbl_packed_ternary_bytes(K: int, N: int) -> int:
+    return int(lib().hbl_packed_ternary_bytes(K, N))
+
+
+def hbl_codes_bytes(M: int, K: int, bits: int) -> int:
+    return int(lib().hbl_codes_bytes(M, K, bits))
+
+
+def hbl_pack_ternary_workspace_bytes(K: int, N: int) -> int:
+    return int(lib().hbl_pack_ternary_workspace_bytes(K, N))
+
+
+def hbl_forward_workspace_bytes(M: int, K: int, N: int, bits: int) -> int:
+    return int(lib().hbl_forward_workspace_bytes(M, K, N, bits))
+
+
+# ------------------------------------------------------------------ compute
+
+def hbl_pack_ternary(W, packed=None, alpha=None, workspace=None, stream=None):
+    """W [N][K] (float32/bf16) -> (packed uint8 [N][K/4], alpha float32 [1])."""
+    torch = _torch()
+    _need_cuda(W)
+    N, K = W.shape
+    if packed is None:
+        packed = torch.empty((N, K // 4), dtype=torch.uint8, device=W.device)
+    if alpha is None:
+        alpha = torch.empty((1,), dtype=torch.float32, device=W.device)
+    if workspace is None:
+        workspace = torch.empty((max(1, hbl_pack_ternary_workspace_bytes(K, N)),), dtype=torch.uint8, device=W.device)
+    _check(lib().hbl_pack_ternary(_ptr(W), _dtype_code(W), K, N, _ptr(packed), _ptr(alpha), _ptr(workspace),
+                                  workspace.numel(), _stream(stream)), "hbl_pack_ternary")
+    return packed, alpha
+
+
+def hbl_fht_quant(x, bits: int, codes=None, scales=None, stream=None):
+    """x [M][K] -> (codes uint8 [M][K/2] (bits 4) or int8 [M][K] (bits 8), scales float32 [M])."""
+    torch = _torch()
+    _need_cuda(x)
+    M, K = x.shape
+    if codes is None:
+        codes = (torch.empty((M, K // 2), dtype=torch.uint8, device=x.device) if bits == 4
+                 else torch.empty((M, K), dtype=torch.int8, device=x.device))
+    if scales is None:
+        scales = torch.empty((M,), dtype=torch.float32, device=x.device)
+    _check(lib().hbl_fht_quant(_ptr(x), _dtype_code(x), M, K, bits, _ptr(codes), _ptr(scales), _stream(stream)),
+           "hbl_fht_quant")
+    return codes, scales
+
+
+def hbl_forward(x, packed, alpha, N: int, bits: int, y=None, y_dtype=None, workspace=None, stream=None):
+    """x [M][K], packed ternary [N][K/4], alpha [1] -> y [M][N] (dtype of x unless y_dtype)."""
+    torch = _torch()
+    _need_cuda(x, packed, alpha)
+    M, K = x.shape
+    if y is None:
+        y = torch.empty((M, N), dtype=y_dtype or x.dtype, device=x.device)
+    if workspace is None:
+        workspace = torch.empty((hbl_forward_workspace_bytes(M, K, N, bits),), dtype=torch.uint8, device=x.device)
+    _check(lib().hbl_forward(_ptr(x), _dtype_code(x), M, K, _ptr(packed), _ptr(alpha), N, bits, _ptr(y),
+                             _dtype_code(y), _ptr(workspace), workspace.numel(), _stream(stream)), "hbl_forward")
+    return y
+
+
+def hbl_debug_ln_fht(x, t=None, stream=None):
+    torch = _torch()
+    _need_cuda(x)
+    M, K = x.shape
+    if t is None:
+        t = torch.empty((M, K), dtype=torch.float32, device=x.device)
+    _check(lib().hbl_debug_ln_fht(_ptr(x), _dtype_code(x), M, K, _ptr(t), _stream(stream)), "hbl_debug_ln_fht")
+    return t
+
+
+def hbl_quant_from_f32(t, bits: int, codes=None, scales=None, stream=None):
+    torch = _torch()
+    _need_cuda(t)
+    M, K = t.shape
+    if codes is None:
+        codes = (torch.empty((M, K // 2), dtype=torch.uint8, device=t.device) if bits == 4
+                 else torch.empty((M, K), dtype=torch.int8, device=t.device))
+    if scales is None:
+        scales = torch.empty((M,), dtype=torch.float32, device=t.device)
+    _check(lib().hbl_quant_from_f32(_ptr(t), M, K, bits, _ptr(codes), _ptr(scales), _stream(stream)),
+           "hbl_quant_from_f32")
+    return codes, scales
+
+
+def hbl_gemm_i8_i32(A, B, acc=None, stream=None):
+    torch = _torch()
+    _need_cuda(A, B)
+    M, K = A.shape
+    N = B.shape[0]
+    if acc is None:
+        acc = torch.empty((M, N), dtype=torch.int32, device=A.device)
+    _check(lib().hbl_gemm_i8_i32(_ptr(A), _ptr(B), M, N, K, _ptr(acc), _stream(stream)), "hbl_gemm_i8_i32")
+    return acc
+
+
+def hbl_last_device_error(stream=None) -> int:
+    return int(lib().hbl_last_device_error(_stream(stream)))
+
+
+def hbl_debug_raise_device_error(stream=None):
+    _check(lib().hbl_debug_raise_device_error(_stream(stream)), "hbl_debug_raise_device_error")

@@ -1,0 +1,56 @@
+// Internal declarations shared by the translation units of libhbl.so.
+// Nothing here is part of the public ABI (include/hbl.h is).
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+
+#include <cuda_runtime.h>
+
+#include "../../include/hbl.h"
+
+namespace hbl {
+
+// K1 output modes of the fused LN -> Hadamard -> quantize kernel.
+enum K1Mode : int {
+  K1_T_F32 = 0,      // t = H LN(x)/sqrt(K) as float (no quantizer)
+  K1_Q4_PACKED = 1,  // INT4 absmean codes, two per byte
+  K1_Q4_I8 = 2,      // INT4 absmean codes widened to one int8 per element
+  K1_Q8_I8 = 3,      // INT8 absmax codes, one int8 per element
+};
+
+constexpr int kMinLogK = 6;   // K = 64
+constexpr int kMaxLogK = 15;  // K = 32768
+
+// Fused K1.  x: [M][K] (bf16 bits if in_bf16 else float).  out: float t,
+// packed nibbles or int8 codes as `mode` says; scales: [M] (ignored for
+// K1_T_F32).  Returns cudaSuccess or the launch error.
+cudaError_t launch_ln_fht_quant(const void* x, bool in_bf16, int64_t M, int log2k, K1Mode mode,
+                                void* out, float* scales, cudaStream_t stream);
+
+// The quantizer alone on float rows t [M][K] (K % 16 == 0).
+cudaError_t launch_quant_from_f32(const float* t, int64_t M, int64_t K, int bits, bool packed,
+                                  uint8_t* codes, float* scales, cudaStream_t stream);
+
+// Ternary weights: partial sums of |W| into ws (double[kTernaryPartials]),
+// then alpha and the 2-bit codes.
+constexpr int kTernaryPartials = 1184;  // 8 blocks per SM of a 148-SM B200
+cudaError_t launch_pack_ternary(const void* W, bool in_bf16, int64_t N, int64_t K, uint8_t* packed,
+                                float* alpha, double* partials, cudaStream_t stream);
+
+// 2-bit ternary codes [N][K/4] -> int8 codes [N][K] for the tensor cores.
+cudaError_t launch_widen_ternary(const uint8_t* packed, int64_t N, int64_t K, int8_t* out,
+                                 cudaStream_t stream);
+
+// tcgen05 int8 GEMM: acc[m][n] = sum_k A[m][k] B[n][k].  Epilogue: either the
+// raw int32 (y_mode 0) or y = (float)acc * (scales[m] * alpha[0]) as float
+// (y_mode 1) or bf16 (y_mode 2).
+cudaError_t launch_gemm_i8(const int8_t* A, const int8_t* B, int64_t M, int64_t N, int64_t K,
+                           int y_mode, void* y, const float* scales, const float* alpha,
+                           cudaStream_t stream);
+
+// Device error word (bounded-wait timeouts) -- lives in gemm_i8.cu.
+cudaError_t read_and_clear_device_error(cudaStream_t stream, int* value);
+cudaError_t raise_device_error(cudaStream_t stream);
+
+}  // namespace hbl

@@ -1,0 +1,432 @@
+// Exact int8 x int8 -> int32 GEMM on the sm_100a tensor cores (tcgen05,
+// kind::i8) with the H-BitLinear dequantisation fused into the epilogue
+// ("BitNet v2: Native 4-bit Activations with Hadamard Transformation for
+// 1-bit LLMs", section "H-BitLinear", matrix-operation formula: the quantised
+// activations times the ternary weights, rescaled by the per-token scale and
+// the weight scale alpha).
+//
+//   acc[m][n] = sum_k A[m][k] * B[n][k]     A: [M][K] int8, B: [N][K] int8
+//   y[m][n]   = (float)acc[m][n] * (scale[m] * alpha)     (float or bf16)
+//
+// Int4 activation codes and ternary weight codes are widened to int8 before
+// they reach this kernel (sm_100 has no int4 or ternary integer MMA); int8
+// products accumulate exactly in int32 (|acc| <= 127 * 32768 < 2^31).
+//
+// Design (one CTA per SM, persistent over 128 x 256 output tiles):
+//   warp 0      TMA producer: 128-byte-swizzled boxes of A (128 x 128 B) and
+//               B (256 x 128 B) into a kStages-deep shared-memory ring;
+//   warp 1      allocates 512 TMEM columns (two 128 x 256 int32
+//               accumulators) and one thread issues tcgen05.mma (M=128,
+//               N=256, K=32 per instruction, four per 128-byte k-block),
+//               committing each stage back to the producer and each finished
+//               accumulator to the epilogue;
+//   warps 2-5   epilogue: tcgen05.ld 32 columns at a time from the TMEM lane
+//               quarter each warp may access, scale, convert, store.
+// The accumulator double buffer lets the epilogue of tile i overlap the main
+// loop of tile i+1.  Every mbarrier wait is bounded: after ~2 s a thread sets
+// the CTA abort flag and the device error word, every role leaves its loop,
+// the MMA thread drains its outstanding MMAs (bounded) and TMEM is freed.
+#include <cstdint>
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+
+namespace hbl {
+
+__device__ int g_device_error = 0;
+
+namespace {
+
+constexpr int kBM = 128;
+constexpr int kBN = 256;
+constexpr int kBK = 128;  // bytes of K per stage (one 128-byte swizzle atom row)
+constexpr int kStages = 4;
+constexpr int kABytes = kBM * kBK;  // 16 KB
+constexpr int kBBytes = kBN * kBK;  // 32 KB
+constexpr int kStageBytes = kABytes + kBBytes;
+constexpr int kThreads = 192;
+constexpr uint32_t kTmemCols = 512;
+constexpr size_t kSmemBytes = 1024 + (size_t)kStages * kStageBytes + 256;
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
+
+// instruction descriptor, kind::i8: D s32, A s8, B s8, both K-major, M=128, N=256
+constexpr uint32_t kIdesc = (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kBN >> 3) << 17) |
+                            ((uint32_t)(kBM >> 4) << 24);
+
+struct Params {
+  int M, N, K;
+  int num_m, num_n, num_tiles, num_kb;
+  int y_mode;  // 0 int32, 1 float, 2 bf16
+  void* y;
+  const float* scales;
+  const float* alpha;
+};
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ uint64_t globaltimer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait for the phase with the given parity.  Returns false if the
+// CTA aborted or the limit ran out (then the abort flag and the device error
+// word are set).
+__device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 63u) == 0) {
+      if (*abort_flag) return false;
+      if (globaltimer() - t0 > kWaitLimitNs) {
+        *abort_flag = 1;
+        atomicExch(&g_device_error, 1);
+        return false;
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+          smem_u32(dst)),
+      "l"((uint64_t)map), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// UMMA shared-memory descriptor of a K-major tile written by TMA with
+// 128-byte swizzle: 8-row atoms of 1024 bytes (stride byte offset 1024), the
+// leading byte offset unused (1), version 1, layout type 2 (SWIZZLE_128B).
+__device__ __forceinline__ uint64_t sdesc(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);
+  d |= (uint64_t)1 << 16;
+  d |= (uint64_t)(1024 >> 4) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)2 << 61;
+  return d;
+}
+
+__device__ __forceinline__ void mma_i8(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(kIdesc), "r"(accumulate));
+}
+
+__device__ __forceinline__ void mma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ uint32_t bf16x2(float lo, float hi) {
+  uint32_t l = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(lo));
+  uint32_t h = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(hi));
+  return l | (h << 16);
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+gemm_i8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  uint8_t* sA = base;
+  uint8_t* sB = base + kStages * kABytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(base + kStages * kStageBytes);
+  uint64_t* empty = full + kStages;
+  uint64_t* tfull = empty + kStages;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 4);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  fence_before();
+  __syncthreads();
+  fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------ TMA producer
+    if (lane == 0) {
+      asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&tmA) : "memory");
+      asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&tmB) : "memory");
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x) {
+        const int m_blk = tile / p.num_n, n_blk = tile % p.num_n;
+        for (int kb = 0; kb < p.num_kb; ++kb) {
+          if (!wait_bounded(&empty[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
+          mbar_expect_tx(&full[stage], (uint32_t)kStageBytes);
+          tma_load_2d(sA + stage * kABytes, &tmA, kb * kBK, m_blk * kBM, &full[stage]);
+          tma_load_2d(sB + stage * kBBytes, &tmB, kb * kBK, n_blk * kBN, &full[stage]);
+          if (++stage == kStages) { stage = 0; phase ^= 1u; }
+        }
+      }
+      if (!ok) {
+        // give the copies already issued time to land before the CTA exits
+        const uint64_t t0 = globaltimer();
+        while (globaltimer() - t0 < 20000000ull) {
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x) {
+        if (!wait_bounded(&tempty[acc], acc_phase ^ 1u, abort_flag)) { ok = false; break; }
+        fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * kBN);
+        for (int kb = 0; kb < p.num_kb; ++kb) {
+          if (!wait_bounded(&full[stage], phase, abort_flag)) { ok = false; break; }
+          fence_after();
+          const uint64_t a0 = sdesc(smem_u32(sA + stage * kABytes));
+          const uint64_t b0 = sdesc(smem_u32(sB + stage * kBBytes));
+#pragma unroll
+          for (int k = 0; k < kBK / 32; ++k) {
+            // advance the start address by 32 bytes (2 x 16 B) per K=32 step
+            mma_i8(d_tmem, a0 + (uint64_t)(2 * k), b0 + (uint64_t)(2 * k), (kb | k) != 0 ? 1u : 0u);
+          }
+          mma_commit(&empty[stage]);
+          if (++stage == kStages) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        mma_commit(&tfull[acc]);
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
+      }
+      // all MMAs issued by this thread are complete once this commit arrives
+      mma_commit(drain);
+      const uint64_t t0 = globaltimer();
+      while (!mbar_try_wait(drain, 0) && globaltimer() - t0 < 200000000ull) {
+      }
+    }
+  } else {
+    // ------------------------------------------------ epilogue (warps 2..5)
+    const int quarter = warp & 3;  // TMEM lanes 32*quarter .. +31
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
+      int ok = 1;
+      if (lane == 0) ok = wait_bounded(&tfull[acc], acc_phase, abort_flag) ? 1 : 0;
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      fence_after();
+      const int m_blk = tile / p.num_n, n_blk = tile % p.num_n;
+      const int row = m_blk * kBM + quarter * 32 + lane;
+      const bool row_ok = row < p.M;
+      float sa = 0.0f;
+      if (p.y_mode != 0 && row_ok) sa = __fmul_rn(__ldg(p.scales + row), __ldg(p.alpha));
+      const uint32_t tbase = tmem_base + (uint32_t)(acc * kBN) + ((uint32_t)(quarter * 32) << 16);
+#pragma unroll 1
+      for (int c = 0; c < kBN; c += 32) {
+        uint32_t r[32];
+        tmem_ld32(tbase + (uint32_t)c, r);
+        const int col0 = n_blk * kBN + c;
+        if (!row_ok) continue;
+        if (p.y_mode == 0) {
+          int32_t* yrow = reinterpret_cast<int32_t*>(p.y) + (size_t)row * p.N;
+#pragma unroll
+          for (int j = 0; j < 32; j += 4)
+            if (col0 + j < p.N) *reinterpret_cast<uint4*>(yrow + col0 + j) = make_uint4(r[j], r[j + 1], r[j + 2], r[j + 3]);
+        } else if (p.y_mode == 1) {
+          float* yrow = reinterpret_cast<float*>(p.y) + (size_t)row * p.N;
+#pragma unroll
+          for (int j = 0; j < 32; j += 4) {
+            if (col0 + j < p.N) {
+              float4 v;
+              v.x = __fmul_rn(__int2float_rn((int)r[j]), sa);
+              v.y = __fmul_rn(__int2float_rn((int)r[j + 1]), sa);
+              v.z = __fmul_rn(__int2float_rn((int)r[j + 2]), sa);
+              v.w = __fmul_rn(__int2float_rn((int)r[j + 3]), sa);
+              *reinterpret_cast<float4*>(yrow + col0 + j) = v;
+            }
+          }
+        } else {
+          uint16_t* yrow = reinterpret_cast<uint16_t*>(p.y) + (size_t)row * p.N;
+#pragma unroll
+          for (int j = 0; j < 32; j += 8) {
+            if (col0 + j < p.N) {
+              uint4 v;
+              v.x = bf16x2(__fmul_rn(__int2float_rn((int)r[j]), sa), __fmul_rn(__int2float_rn((int)r[j + 1]), sa));
+              v.y = bf16x2(__fmul_rn(__int2float_rn((int)r[j + 2]), sa), __fmul_rn(__int2float_rn((int)r[j + 3]), sa));
+              v.z = bf16x2(__fmul_rn(__int2float_rn((int)r[j + 4]), sa), __fmul_rn(__int2float_rn((int)r[j + 5]), sa));
+              v.w = bf16x2(__fmul_rn(__int2float_rn((int)r[j + 6]), sa), __fmul_rn(__int2float_rn((int)r[j + 7]), sa));
+              *reinterpret_cast<uint4*>(yrow + col0 + j) = v;
+            }
+          }
+        }
+      }
+      fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[acc]);
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1u;
+    }
+  }
+
+  fence_before();
+  __syncthreads();
+  fence_after();
+  if (warp == 1) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kTmemCols)
+                 : "memory");
+  }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = []() -> PFN_cuTensorMapEncodeTiled_v12000 {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }();
+  return fn;
+}
+
+// 2-D K-major int8 tensor map: rows x K bytes, box kBK x box_rows, 128-byte swizzle.
+bool make_map(CUtensorMap* map, const void* ptr, int64_t rows, int64_t K, int box_rows) {
+  auto encode = get_encode();
+  if (!encode) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)K};
+  cuuint32_t box[2] = {(cuuint32_t)kBK, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+  return n;
+}
+
+}  // namespace
+
+cudaError_t launch_gemm_i8(const int8_t* A, const int8_t* B, int64_t M, int64_t N, int64_t K, int y_mode, void* y,
+                           const float* scales, const float* alpha, cudaStream_t stream) {
+  CUtensorMap ta, tb;
+  if (!make_map(&ta, A, M, K, kBM) || !make_map(&tb, B, N, K, kBN)) return cudaErrorInvalidValue;
+  Params p;
+  p.M = (int)M;
+  p.N = (int)N;
+  p.K = (int)K;
+  p.num_m = (int)((M + kBM - 1) / kBM);
+  p.num_n = (int)((N + kBN - 1) / kBN);
+  p.num_tiles = p.num_m * p.num_n;
+  p.num_kb = (int)((K + kBK - 1) / kBK);
+  p.y_mode = y_mode;
+  p.y = y;
+  p.scales = scales;
+  p.alpha = alpha;
+  cudaError_t e = cudaFuncSetAttribute(gemm_i8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+  if (e != cudaSuccess) return e;
+  const int grid = p.num_tiles < sm_count() ? p.num_tiles : sm_count();
+  gemm_i8_kernel<<<grid, kThreads, kSmemBytes, stream>>>(ta, tb, p);
+  return cudaGetLastError();
+}
+
+cudaError_t read_and_clear_device_error(cudaStream_t stream, int* value) {
+  cudaError_t e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) return e;
+  int v = 0, zero = 0;
+  e = cudaMemcpyFromSymbol(&v, g_device_error, sizeof(int));
+  if (e != cudaSuccess) return e;
+  e = cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int));
+  *value = v;
+  return e;
+}
+
+namespace {
+__global__ void raise_error_kernel() { atomicExch(&g_device_error, 1); }
+}  // namespace
+
+cudaError_t raise_device_error(cudaStream_t stream) {
+  raise_error_kernel<<<1, 1, 0, stream>>>();
+  return cudaGetLastError();
+}
+
+}  // namespace hbl

@@ -1,0 +1,199 @@
+// C ABI of libhbl.so (declarations and contracts in include/hbl.h): argument
+// checks, workspace carving and the launch sequence of each entry point.
+#include <cstdint>
+
+#include "common.cuh"
+
+namespace {
+
+using hbl::K1Mode;
+
+constexpr int64_t kMaxRows = int64_t(1) << 26;
+constexpr int64_t kMaxN = int64_t(1) << 20;
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+int log2_exact(int64_t K) {
+  if (K <= 0 || (K & (K - 1))) return -1;
+  int l = 0;
+  while ((int64_t(1) << l) < K) ++l;
+  return l;
+}
+
+size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+
+bool dtype_ok(hbl_dtype t) { return t == HBL_F32 || t == HBL_BF16; }
+
+hbl_status cuda_status(cudaError_t e) { return e == cudaSuccess ? HBL_OK : HBL_ERR_CUDA; }
+
+// K a power of two in [64, 32768] -> log2 K, else -1 / -2 (unsupported)
+hbl_status check_k(int64_t K, int* log2k) {
+  if (K <= 0) return HBL_ERR_INVALID_ARG;
+  int l = log2_exact(K);
+  if (l < hbl::kMinLogK || l > hbl::kMaxLogK) return HBL_ERR_UNSUPPORTED;
+  *log2k = l;
+  return HBL_OK;
+}
+
+hbl_status check_rows(int64_t M) {
+  if (M <= 0) return HBL_ERR_INVALID_ARG;
+  if (M > kMaxRows) return HBL_ERR_UNSUPPORTED;
+  return HBL_OK;
+}
+
+hbl_status check_n(int64_t N) {
+  if (N <= 0) return HBL_ERR_INVALID_ARG;
+  if (N % 16 != 0 || N > kMaxN) return HBL_ERR_UNSUPPORTED;
+  return HBL_OK;
+}
+
+struct ForwardLayout {
+  size_t a_off, s_off, b_off, total;
+};
+
+ForwardLayout forward_layout(int64_t M, int64_t K, int64_t N) {
+  ForwardLayout L;
+  L.a_off = 0;
+  L.s_off = align256((size_t)M * (size_t)K);
+  L.b_off = L.s_off + align256((size_t)M * 4);
+  L.total = L.b_off + align256((size_t)N * (size_t)K);
+  return L;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t hbl_packed_ternary_bytes(int64_t K, int64_t N) {
+  int l;
+  if (check_k(K, &l) != HBL_OK || check_n(N) != HBL_OK) return 0;
+  return (size_t)N * (size_t)(K / 4);
+}
+
+size_t hbl_codes_bytes(int64_t M, int64_t K, int bits) {
+  int l;
+  if (check_k(K, &l) != HBL_OK || check_rows(M) != HBL_OK || (bits != 4 && bits != 8)) return 0;
+  return bits == 4 ? (size_t)M * (size_t)(K / 2) : (size_t)M * (size_t)K;
+}
+
+size_t hbl_pack_ternary_workspace_bytes(int64_t K, int64_t N) {
+  int l;
+  if (check_k(K, &l) != HBL_OK || check_n(N) != HBL_OK) return 0;
+  return sizeof(double) * hbl::kTernaryPartials;
+}
+
+size_t hbl_forward_workspace_bytes(int64_t M, int64_t K, int64_t N, int bits) {
+  int l;
+  if (check_k(K, &l) != HBL_OK || check_rows(M) != HBL_OK || check_n(N) != HBL_OK || (bits != 4 && bits != 8))
+    return 0;
+  return forward_layout(M, K, N).total;
+}
+
+hbl_status hbl_pack_ternary(const void* W, hbl_dtype wt, int64_t K, int64_t N, uint8_t* packed, float* alpha_dev,
+                            void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  if (!W || !packed || !alpha_dev || !dtype_ok(wt)) return HBL_ERR_INVALID_ARG;
+  if (!aligned(W, 16) || !aligned(packed, 16) || !aligned(alpha_dev, 4)) return HBL_ERR_INVALID_ARG;
+  int l;
+  hbl_status s = check_k(K, &l);
+  if (s != HBL_OK) return s;
+  if ((s = check_n(N)) != HBL_OK) return s;
+  if (!workspace || !aligned(workspace, 16) || workspace_bytes < hbl_pack_ternary_workspace_bytes(K, N))
+    return HBL_ERR_WORKSPACE;
+  return cuda_status(hbl::launch_pack_ternary(W, wt == HBL_BF16, N, K, packed, alpha_dev,
+                                              reinterpret_cast<double*>(workspace), stream));
+}
+
+hbl_status hbl_fht_quant(const void* x, hbl_dtype xt, int64_t M, int64_t K, int bits, uint8_t* codes, float* scales,
+                         cudaStream_t stream) {
+  if (!x || !codes || !scales || !dtype_ok(xt) || (bits != 4 && bits != 8)) return HBL_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(codes, 16) || !aligned(scales, 4)) return HBL_ERR_INVALID_ARG;
+  int l;
+  hbl_status s = check_k(K, &l);
+  if (s != HBL_OK) return s;
+  if ((s = check_rows(M)) != HBL_OK) return s;
+  const K1Mode mode = bits == 4 ? hbl::K1_Q4_PACKED : hbl::K1_Q8_I8;
+  return cuda_status(hbl::launch_ln_fht_quant(x, xt == HBL_BF16, M, l, mode, codes, scales, stream));
+}
+
+hbl_status hbl_forward(const void* x, hbl_dtype xt, int64_t M, int64_t K, const uint8_t* packed,
+                       const float* alpha_dev, int64_t N, int bits, void* y, hbl_dtype yt, void* workspace,
+                       size_t workspace_bytes, cudaStream_t stream) {
+  if (!x || !packed || !alpha_dev || !y || !dtype_ok(xt) || !dtype_ok(yt) || (bits != 4 && bits != 8))
+    return HBL_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(packed, 16) || !aligned(alpha_dev, 4) || !aligned(y, 16))
+    return HBL_ERR_INVALID_ARG;
+  int l;
+  hbl_status s = check_k(K, &l);
+  if (s != HBL_OK) return s;
+  if ((s = check_rows(M)) != HBL_OK) return s;
+  if ((s = check_n(N)) != HBL_OK) return s;
+  const ForwardLayout L = forward_layout(M, K, N);
+  if (!workspace || !aligned(workspace, 256) || workspace_bytes < L.total) return HBL_ERR_WORKSPACE;
+  uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
+  int8_t* A = reinterpret_cast<int8_t*>(ws + L.a_off);
+  float* scales = reinterpret_cast<float*>(ws + L.s_off);
+  int8_t* B = reinterpret_cast<int8_t*>(ws + L.b_off);
+  const K1Mode mode = bits == 4 ? hbl::K1_Q4_I8 : hbl::K1_Q8_I8;
+  cudaError_t e = hbl::launch_ln_fht_quant(x, xt == HBL_BF16, M, l, mode, A, scales, stream);
+  if (e == cudaSuccess) e = hbl::launch_widen_ternary(packed, N, K, B, stream);
+  if (e == cudaSuccess) e = hbl::launch_gemm_i8(A, B, M, N, K, yt == HBL_BF16 ? 2 : 1, y, scales, alpha_dev, stream);
+  return cuda_status(e);
+}
+
+hbl_status hbl_debug_ln_fht(const void* x, hbl_dtype xt, int64_t M, int64_t K, float* t, cudaStream_t stream) {
+  if (!x || !t || !dtype_ok(xt)) return HBL_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(t, 16)) return HBL_ERR_INVALID_ARG;
+  int l;
+  hbl_status s = check_k(K, &l);
+  if (s != HBL_OK) return s;
+  if ((s = check_rows(M)) != HBL_OK) return s;
+  return cuda_status(hbl::launch_ln_fht_quant(x, xt == HBL_BF16, M, l, hbl::K1_T_F32, t, nullptr, stream));
+}
+
+hbl_status hbl_quant_from_f32(const float* t, int64_t M, int64_t K, int bits, uint8_t* codes, float* scales,
+                              cudaStream_t stream) {
+  if (!t || !codes || !scales || (bits != 4 && bits != 8)) return HBL_ERR_INVALID_ARG;
+  if (!aligned(t, 16) || !aligned(codes, 16) || !aligned(scales, 4)) return HBL_ERR_INVALID_ARG;
+  if (K <= 0) return HBL_ERR_INVALID_ARG;
+  if (K % 16 != 0 || K > 65536) return HBL_ERR_UNSUPPORTED;
+  hbl_status s = check_rows(M);
+  if (s != HBL_OK) return s;
+  return cuda_status(hbl::launch_quant_from_f32(t, M, K, bits, bits == 4, codes, scales, stream));
+}
+
+hbl_status hbl_gemm_i8_i32(const int8_t* A, const int8_t* B, int64_t M, int64_t N, int64_t K, int32_t* acc,
+                           cudaStream_t stream) {
+  if (!A || !B || !acc) return HBL_ERR_INVALID_ARG;
+  if (!aligned(A, 16) || !aligned(B, 16) || !aligned(acc, 16)) return HBL_ERR_INVALID_ARG;
+  if (K <= 0) return HBL_ERR_INVALID_ARG;
+  if (K % 16 != 0 || K > 65536) return HBL_ERR_UNSUPPORTED;
+  hbl_status s = check_rows(M);
+  if (s != HBL_OK) return s;
+  if ((s = check_n(N)) != HBL_OK) return s;
+  return cuda_status(hbl::launch_gemm_i8(A, B, M, N, K, 0, acc, nullptr, nullptr, stream));
+}
+
+hbl_status hbl_last_device_error(cudaStream_t stream) {
+  int v = 0;
+  cudaError_t e = hbl::read_and_clear_device_error(stream, &v);
+  if (e != cudaSuccess) return HBL_ERR_CUDA;
+  return v ? HBL_ERR_TIMEOUT : HBL_OK;
+}
+
+hbl_status hbl_debug_raise_device_error(cudaStream_t stream) {
+  return cuda_status(hbl::raise_device_error(stream));
+}
+
+const char* hbl_status_string(hbl_status status) {
+  switch (status) {
+    case HBL_OK: return "HBL_OK";
+    case HBL_ERR_INVALID_ARG: return "HBL_ERR_INVALID_ARG";
+    case HBL_ERR_UNSUPPORTED: return "HBL_ERR_UNSUPPORTED";
+    case HBL_ERR_WORKSPACE: return "HBL_ERR_WORKSPACE";
+    case HBL_ERR_CUDA: return "HBL_ERR_CUDA";
+    case HBL_ERR_TIMEOUT: return "HBL_ERR_TIMEOUT";
+  }
+  return "HBL_ERR_UNKNOWN";
+}
+
+}  // extern "C"

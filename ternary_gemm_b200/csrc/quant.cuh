@@ -1,0 +1,86 @@
+// Per-token activation quantizer shared by the fused LN+FHT+quant kernel and
+// the quantizer-only kernel, so both make bit-identical decisions.
+//
+// "BitNet v2: Native 4-bit Activations with Hadamard Transformation for 1-bit
+// LLMs", section "H-BitLinear", activation-quantization formula:
+//   4 bit, per-token absmean: beta = mean|t|,
+//          q = clip(rint(sqrt(7) t / (beta + eps)), -8, 7), scale = beta / sqrt(7)
+//   8 bit, per-token absmax : gamma = max|t|,
+//          q = clip(rint(127 t / (gamma + eps)), -128, 127), scale = gamma / 127
+// Arithmetic contract (float unless stated): the mean of |t| is accumulated in
+// double and rounded once to float; r = c / (stat + eps) is one IEEE division
+// per row; each code is rint of the float product t * r (round half to even).
+// The __f*_rn intrinsics keep the compiler from fusing these into FMAs, which
+// would round differently.
+#pragma once
+
+#include <cstdint>
+
+namespace hbl {
+namespace q {
+
+constexpr float kEps = 1e-5f;
+constexpr float kSqrt7 = 2.6457513110645906f;  // sqrt(7) rounded to float
+constexpr float kMagic = 12582912.0f;          // 1.5 * 2^23
+constexpr int kMagicBits = 0x4B400000;
+
+// |t| as a double, for the absmean accumulation.
+__device__ __forceinline__ double abs_f64(float t) { return (double)fabsf(t); }
+
+struct RowParams {
+  float r;      // multiplier applied to t before rounding
+  float scale;  // dequantisation factor of the row
+};
+
+// beta from the double sum of |t| over K elements.
+__device__ __forceinline__ RowParams params_int4(double abs_sum, int64_t K) {
+  float beta = (float)(abs_sum / (double)K);
+  RowParams p;
+  p.r = __fdiv_rn(kSqrt7, __fadd_rn(beta, kEps));
+  p.scale = __fdiv_rn(beta, kSqrt7);
+  return p;
+}
+
+// gamma = max |t| (exact, order free).
+__device__ __forceinline__ RowParams params_int8(float gamma) {
+  RowParams p;
+  p.r = __fdiv_rn(127.0f, __fadd_rn(gamma, kEps));
+  p.scale = __fdiv_rn(gamma, 127.0f);
+  return p;
+}
+
+// rint(fl(t * r)) for |t * r| < 2^22: adding 1.5 * 2^23 leaves a float whose
+// unit in the last place is 1, so the addition itself rounds to the nearest
+// integer, ties to even (1.5 * 2^23 is even), and the integer sits in the low
+// mantissa bits.  Exact for the whole range the callers use: |t r| <= K sqrt(7)
+// for absmean, < 128 for absmax.
+__device__ __forceinline__ int rint_code(float t, float r) {
+  float v = __fmul_rn(t, r);
+  float m = __fadd_rn(v, kMagic);
+  return __float_as_int(m) - kMagicBits;
+}
+
+// Eight codes -> eight 4-bit two's-complement fields, n[0] in the lowest
+// nibble; cvt.pack.sat saturates each input to [-8, 7] (the clip).
+__device__ __forceinline__ uint32_t pack_s4x8(const int (&n)[8]) {
+  uint32_t d;
+  asm("cvt.pack.sat.s4.s32.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(n[7]), "r"(n[6]), "r"(0u));
+  asm("cvt.pack.sat.s4.s32.b32 %0, %1, %2, %0;" : "+r"(d) : "r"(n[5]), "r"(n[4]));
+  asm("cvt.pack.sat.s4.s32.b32 %0, %1, %2, %0;" : "+r"(d) : "r"(n[3]), "r"(n[2]));
+  asm("cvt.pack.sat.s4.s32.b32 %0, %1, %2, %0;" : "+r"(d) : "r"(n[1]), "r"(n[0]));
+  return d;
+}
+
+// Four codes -> four int8 bytes, n[0] in the lowest byte, saturated to
+// [-128, 127].
+__device__ __forceinline__ uint32_t pack_s8x4(int n0, int n1, int n2, int n3) {
+  uint32_t d;
+  asm("cvt.pack.sat.s8.s32.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(n3), "r"(n2), "r"(0u));
+  asm("cvt.pack.sat.s8.s32.b32 %0, %1, %2, %0;" : "+r"(d) : "r"(n1), "r"(n0));
+  return d;
+}
+
+__device__ __forceinline__ int clip_int4(int n) { return max(-8, min(7, n)); }
+
+}  // namespace q
+}  // namespace hbl

@@ -1,0 +1,71 @@
+"""Shared helpers of the GPU parity tests: host <-> device marshalling and the
+comparison rules (tolerances written here, derived in the docstrings)."""
+import math
+
+import numpy as np
+
+
+def to_device(a):
+    """numpy float32 -> torch float32, numpy uint16 (bf16 bits) -> torch bfloat16, int8 -> int8."""
+    import torch
+    if a.dtype == np.uint16:
+        return torch.from_numpy(a.view(np.int16).copy()).view(torch.bfloat16).cuda()
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def to_host(t):
+    import torch
+    if t.dtype == torch.bfloat16:
+        return t.view(torch.int16).cpu().numpy().view(np.uint16)
+    return t.cpu().numpy()
+
+
+def unpack_nibbles(p, K):
+    """uint8 [M][K/2] -> int8 [M][K]; element 2j in the low nibble."""
+    p = np.asarray(p, dtype=np.uint8)
+    lo = (p & 0xF).astype(np.int8)
+    hi = (p >> 4).astype(np.int8)
+    lo = np.where(lo >= 8, lo - 16, lo)
+    hi = np.where(hi >= 8, hi - 16, hi)
+    out = np.empty((p.shape[0], K), np.int8)
+    out[:, 0::2] = lo
+    out[:, 1::2] = hi
+    return out
+
+
+def check_t(t_gpu, t64, rel=1e-5):
+    """Post-transform float values: per row ||dt||/||t|| <= rel and max|dt| <= rel * rms(t)."""
+    d = t_gpu.astype(np.float64) - t64
+    nrm = np.linalg.norm(t64, axis=1)
+    rms = nrm / math.sqrt(t64.shape[1])
+    nz = nrm > 0
+    assert np.all(np.linalg.norm(d, axis=1)[nz] <= rel * nrm[nz]), np.max(np.linalg.norm(d, axis=1)[nz] / nrm[nz])
+    assert np.all(np.abs(d).max(axis=1)[nz] <= rel * rms[nz]), np.max(np.abs(d).max(axis=1)[nz] / rms[nz])
+    assert np.all(np.abs(t_gpu[~nz]) == 0)
+
+
+def check_codes_near(q_gpu, q_orc, t_orc32, scale_orc, bits, min_agree=0.9999, half_tol=1e-4):
+    """End-to-end codes: >= 99.99% equal; every mismatch is off by one where the
+    oracle's t*r lies within `half_tol` of a rounding boundary (a half-integer)."""
+    c = math.sqrt(7.0) if bits == 4 else 127.0
+    q_gpu = q_gpu.astype(np.int32)
+    q_orc = q_orc.astype(np.int32)
+    mism = q_gpu != q_orc
+    agree = 1.0 - mism.mean()
+    assert agree >= min_agree, agree
+    if mism.any():
+        assert np.all(np.abs(q_gpu - q_orc)[mism] == 1)
+        rows = np.nonzero(mism)[0]
+        stat = scale_orc.astype(np.float64) * c          # beta or gamma
+        r = np.float32(c) / (stat.astype(np.float32) + np.float32(1e-5))
+        v = t_orc32[mism].astype(np.float64) * r[rows]
+        frac = np.abs(v - np.floor(v) - 0.5)
+        assert np.all(frac <= half_tol), frac.max()
+    return agree
+
+
+def rel_fro(a, b):
+    a = np.asarray(a, np.float64)
+    b = np.asarray(b, np.float64)
+    n = np.linalg.norm(b)
+    return np.linalg.norm(a - b) / (n if n > 0 else 1.0)

@@ -1,0 +1,129 @@
+"""The C ABI without a GPU: the library builds, loads, exports every symbol the
+header declares, answers size queries, and rejects bad arguments on the host
+before any launch (every call here fails validation, so nothing reaches CUDA).
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+import ternary_gemm_b200 as hbl
+from ternary_gemm_b200 import build as hbl_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    hbl_build.build()
+    return hbl.lib()
+
+
+def test_exports_every_declared_symbol(L):
+    names = hbl.declared_symbols()
+    assert len(names) >= 13
+    for n in names:
+        assert hasattr(L, n), n
+    # and nothing else is exported under the hbl_ prefix
+    out = os.popen("nm -D --defined-only %s" % hbl.LIB_PATH).read()
+    exported = set(re.findall(r"\bT (hbl_[a-z0-9_]+)\b", out))
+    assert exported == set(names)
+
+
+def test_size_queries(L):
+    assert hbl.hbl_packed_ternary_bytes(16384, 4096) == 4096 * 4096
+    assert hbl.hbl_codes_bytes(8192, 16384, 4) == 8192 * 8192
+    assert hbl.hbl_codes_bytes(8192, 16384, 8) == 8192 * 16384
+    assert hbl.hbl_pack_ternary_workspace_bytes(256, 256) > 0
+    ws = hbl.hbl_forward_workspace_bytes(8192, 16384, 4096, 4)
+    assert ws >= 8192 * 16384 + 8192 * 4 + 4096 * 16384
+    # invalid sizes give 0
+    assert hbl.hbl_packed_ternary_bytes(100, 256) == 0
+    assert hbl.hbl_codes_bytes(8, 256, 5) == 0
+    assert hbl.hbl_forward_workspace_bytes(8, 256, 24, 4) == 0
+    assert hbl.hbl_forward_workspace_bytes(0, 256, 256, 4) == 0
+
+
+FAKE = ctypes.c_void_p(0x10000)        # aligned, never dereferenced: validation fails first
+FAKE_ODD = ctypes.c_void_p(0x10001)
+NULL = ctypes.c_void_p(0)
+S0 = ctypes.c_void_p(0)
+
+
+@pytest.mark.parametrize("args,want", [
+    ((NULL, 1, 8, 256, 4, FAKE, FAKE, S0), hbl.HBL_ERR_INVALID_ARG),
+    ((FAKE, 1, 8, 256, 5, FAKE, FAKE, S0), hbl.HBL_ERR_INVALID_ARG),
+    ((FAKE, 7, 8, 256, 4, FAKE, FAKE, S0), hbl.HBL_ERR_INVALID_ARG),
+    ((FAKE_ODD, 1, 8, 256, 4, FAKE, FAKE, S0), hbl.HBL_ERR_INVALID_ARG),
+    ((FAKE, 1, 0, 256, 4, FAKE, FAKE, S0), hbl.HBL_ERR_INVALID_ARG),
+    ((FAKE, 1, 8, 100, 4, FAKE, FAKE, S0), hbl.HBL_ERR_UNSUPPORTED),
+    ((FAKE, 1, 8, 32, 4, FAKE, FAKE, S0), hbl.HBL_ERR_UNSUPPORTED),
+    ((FAKE, 1, 8, 65536, 8, FAKE, FAKE, S0), hbl.HBL_ERR_UNSUPPORTED),
+    ((FAKE, 1, 1 << 27, 256, 4, FAKE, FAKE, S0), hbl.HBL_ERR_UNSUPPORTED),
+])
+def test_fht_quant_validation(L, args, want):
+    assert L.hbl_fht_quant(*args) == want
+
+
+def test_forward_validation(L):
+    f = L.hbl_forward
+    assert f(FAKE, 1, 8, 256, FAKE, FAKE, 24, 4, FAKE, 1, FAKE, 1 << 30, S0) == hbl.HBL_ERR_UNSUPPORTED
+    assert f(FAKE, 1, 8, 256, FAKE, FAKE, 256, 3, FAKE, 1, FAKE, 1 << 30, S0) == hbl.HBL_ERR_INVALID_ARG
+    assert f(FAKE, 1, 8, 256, NULL, FAKE, 256, 4, FAKE, 1, FAKE, 1 << 30, S0) == hbl.HBL_ERR_INVALID_ARG
+    assert f(FAKE, 1, 8, 256, FAKE, FAKE, 256, 4, FAKE, 2, FAKE, 1 << 30, S0) == hbl.HBL_ERR_INVALID_ARG
+    need = hbl.hbl_forward_workspace_bytes(8, 256, 256, 4)
+    assert f(FAKE, 1, 8, 256, FAKE, FAKE, 256, 4, FAKE, 1, FAKE, need - 1, S0) == hbl.HBL_ERR_WORKSPACE
+    assert f(FAKE, 1, 8, 256, FAKE, FAKE, 256, 4, FAKE, 1, NULL, need, S0) == hbl.HBL_ERR_WORKSPACE
+    # the workspace must be 256-byte aligned
+    assert f(FAKE, 1, 8, 256, FAKE, FAKE, 256, 4, FAKE, 1, ctypes.c_void_p(0x10010), need, S0) == hbl.HBL_ERR_WORKSPACE
+
+
+def test_pack_ternary_validation(L):
+    f = L.hbl_pack_ternary
+    assert f(FAKE, 1, 256, 256, FAKE, FAKE, NULL, 1 << 20, S0) == hbl.HBL_ERR_WORKSPACE
+    assert f(FAKE, 1, 256, 256, FAKE, FAKE, FAKE, 8, S0) == hbl.HBL_ERR_WORKSPACE
+    assert f(FAKE, 1, 256, 40, FAKE, FAKE, FAKE, 1 << 20, S0) == hbl.HBL_ERR_UNSUPPORTED
+    assert f(NULL, 1, 256, 256, FAKE, FAKE, FAKE, 1 << 20, S0) == hbl.HBL_ERR_INVALID_ARG
+
+
+def test_hook_validation(L):
+    assert L.hbl_quant_from_f32(FAKE, 8, 24, 4, FAKE, FAKE, S0) == hbl.HBL_ERR_UNSUPPORTED
+    assert L.hbl_quant_from_f32(FAKE, 8, 32, 6, FAKE, FAKE, S0) == hbl.HBL_ERR_INVALID_ARG
+    assert L.hbl_gemm_i8_i32(FAKE, FAKE, 8, 256, 8, FAKE, S0) == hbl.HBL_ERR_UNSUPPORTED
+    assert L.hbl_gemm_i8_i32(FAKE, FAKE, 8, 20, 64, FAKE, S0) == hbl.HBL_ERR_UNSUPPORTED
+    assert L.hbl_debug_ln_fht(FAKE, 1, 8, 96, FAKE, S0) == hbl.HBL_ERR_UNSUPPORTED
+
+
+def test_status_strings(L):
+    assert hbl.status_string(hbl.HBL_OK) == "HBL_OK"
+    assert hbl.status_string(hbl.HBL_ERR_TIMEOUT) == "HBL_ERR_TIMEOUT"
+    assert hbl.status_string(99) == "HBL_ERR_UNKNOWN"
+
+
+def test_binding_fails_loudly_without_library(monkeypatch):
+    monkeypatch.setattr(hbl, "_lib", None)
+    monkeypatch.setattr(hbl, "LIB_PATH", "/nonexistent/libhbl.so")
+    with pytest.raises(ImportError):
+        hbl.lib()
+
+
+def test_oracle_and_cuda_path_are_independent():
+    """The oracle never imports the package and the CUDA sources never include the oracle."""
+    for f in os.listdir(os.path.join(ROOT, "oracle")):
+        text = open(os.path.join(ROOT, "oracle", f)).read() if f.endswith((".py", ".c")) else ""
+        if f.endswith(".c"):
+            for inc in re.findall(r'#include\s*[<"]([^>"]+)[>"]', text):
+                assert inc in ("fenv.h", "math.h", "stdint.h", "stdlib.h", "string.h"), (f, inc)
+        if f.endswith(".py"):
+            assert not re.search(r"^\s*(import|from)\s+ternary_gemm_b200", text, re.M), f
+    csrc = os.path.join(ROOT, "ternary_gemm_b200", "csrc")
+    for f in os.listdir(csrc):
+        text = open(os.path.join(csrc, f)).read()
+        for inc in re.findall(r'#include\s*"([^"]+)"', text):
+            assert "oracle" not in inc, (f, inc)
+    pkg = os.path.join(ROOT, "ternary_gemm_b200")
+    for f in os.listdir(pkg):
+        if f.endswith(".py"):
+            text = open(os.path.join(pkg, f)).read()
+            assert "import oracle" not in text and "from oracle" not in text, f

@@ -1,0 +1,152 @@
+"""GPU parity of the ternary packing, the tcgen05 int8 GEMM and the whole
+H-BitLinear forward against the CPU oracle (through the C ABI).
+
+Tolerances:
+  * ternary codes and alpha bit-exact;
+  * int32 GEMM accumulators bit-exact;
+  * y bit-exact against the oracle's GEMM + dequantisation of the library's
+    own codes (same integers, same float products, same bf16 rounding);
+  * y within 2e-3 relative Frobenius of the oracle's forward from x (bf16
+    outputs compared with the oracle's float y rounded to bf16).
+"""
+import numpy as np
+import pytest
+
+from helpers import rel_fro, to_device, to_host, unpack_nibbles
+from ternary_gemm_b200.inputs import WORKLOADS, make_w, make_x, sample_rows
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def H():
+    import torch
+    from ternary_gemm_b200 import build
+    assert torch.cuda.is_available()
+    build.build()
+    import ternary_gemm_b200 as hbl
+    return hbl
+
+
+# ----------------------------------------------------------------- ternary packing
+
+@pytest.mark.parametrize("name", ["tiny", "wo_1p3b", "wdown_3b"])
+def test_pack_ternary_bit_exact(H, orc, name):
+    W = make_w(WORKLOADS[name])
+    packed, alpha = H.hbl_pack_ternary(to_device(W))
+    w, a = orc.ternary(W)
+    assert to_host(alpha)[0] == a
+    assert np.array_equal(to_host(packed), orc.pack_ternary(w))
+
+
+def test_pack_ternary_edge_cases(H, orc):
+    W = np.zeros((16, 64), np.float32)
+    packed, alpha = H.hbl_pack_ternary(to_device(W))
+    assert to_host(alpha)[0] == 0 and np.all(to_host(packed) == 0)
+    rng = np.random.default_rng(0)
+    W = (rng.standard_normal((32, 128)) * 0.02).astype(np.float32)
+    W[3, 7] = 1e6                                   # one weight dominates alpha
+    packed, alpha = H.hbl_pack_ternary(to_device(W))
+    w, a = orc.ternary(W)
+    assert to_host(alpha)[0] == a and np.array_equal(to_host(packed), orc.pack_ternary(w))
+
+
+# ----------------------------------------------------------------- int8 GEMM
+
+@pytest.mark.parametrize("M,N,K", [(1, 16, 16), (8, 256, 256), (128, 256, 128), (300, 272, 2048),
+                                   (257, 512, 4096), (64, 48, 208), (1000, 4096, 64), (129, 1040, 1024)])
+def test_gemm_exact(H, orc, M, N, K):
+    rng = np.random.default_rng(M * 7 + N * 3 + K)
+    A = rng.integers(-128, 128, (M, K)).astype(np.int8)
+    B = rng.integers(-128, 128, (N, K)).astype(np.int8)
+    acc = to_host(H.hbl_gemm_i8_i32(to_device(A), to_device(B)))
+    assert np.array_equal(acc, orc.gemm_i32(A, B))
+
+
+@pytest.mark.slow
+def test_gemm_exact_7b_shape_sampled(H, orc):
+    M, N, K = 8192, 4096, 16384
+    rng = np.random.default_rng(5)
+    A = rng.integers(-8, 8, (M, K)).astype(np.int8)
+    B = rng.integers(-1, 2, (N, K)).astype(np.int8)
+    acc = to_host(H.hbl_gemm_i8_i32(to_device(A), to_device(B)))
+    rows = sample_rows(M, 24)
+    assert np.array_equal(acc[rows], orc.gemm_i32(A[rows], B))
+
+
+# ----------------------------------------------------------------- forward
+
+def _forward_check(H, orc, x, W, bits, rows=None, y_dtype=None):
+    import torch
+    M, K = x.shape
+    N = W.shape[0]
+    xd = to_device(x)
+    packed, alpha = H.hbl_pack_ternary(to_device(W))
+    y = H.hbl_forward(xd, packed, alpha, N, bits, y_dtype=y_dtype)
+    torch.cuda.synchronize()
+    rows = np.arange(M) if rows is None else rows
+    y_h = to_host(y)[rows]
+    bf16_out = y.dtype == torch.bfloat16
+    w, a = orc.ternary(W)
+    assert to_host(alpha)[0] == a
+    # exact: the oracle's GEMM + dequant of the library's own codes
+    codes, scales = H.hbl_fht_quant(to_device(x[rows]), bits)
+    q = unpack_nibbles(to_host(codes), K) if bits == 4 else to_host(codes)
+    y_exact = orc.dequant(orc.gemm_i32(q, w), to_host(scales), a)
+    if bf16_out:
+        assert np.array_equal(y_h, orc.round_to_bf16(y_exact))
+    else:
+        assert np.array_equal(y_h, y_exact)
+    # end to end from x
+    y_orc, _, _ = orc.forward_rows(x, w, a, bits, rows=rows)
+    if bf16_out:
+        err = rel_fro(orc.bf16_bits_to_float(y_h), orc.bf16_bits_to_float(orc.round_to_bf16(y_orc)))
+    else:
+        err = rel_fro(y_h, y_orc)
+    assert err <= 2e-3, err
+    return err
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+def test_forward_tiny(H, orc, bits):
+    wl = WORKLOADS["tiny"]
+    _forward_check(H, orc, make_x(wl), make_w(wl), bits)
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+@pytest.mark.parametrize("M,K,N", [(300, 2048, 272), (1, 4096, 4096), (16, 1024, 256), (130, 64, 16)])
+def test_forward_ragged(H, orc, bits, M, K, N):
+    wl = WORKLOADS["sweep"].with_shape(M, K, N)
+    _forward_check(H, orc, make_x(wl), make_w(wl), bits)
+
+
+def test_forward_float_output_from_bf16(H, orc):
+    import torch
+    wl = WORKLOADS["sweep"].with_shape(64, 1024, 512)
+    _forward_check(H, orc, make_x(wl), make_w(wl), 4, y_dtype=torch.float32)
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name,bits", [("wo_1p3b", 4), ("wo_1p3b", 8), ("wdown_3b", 4), ("wdown_7b", 4),
+                                       ("wdown_7b", 8)])
+def test_forward_full_size_sampled_rows(H, orc, name, bits):
+    wl = WORKLOADS[name]
+    _forward_check(H, orc, make_x(wl), make_w(wl), bits, rows=sample_rows(wl.M, 32))
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("M", [1, 16, 128, 1024, 16384])
+def test_forward_decode_to_batch_sweep(H, orc, M):
+    wl = WORKLOADS["sweep"].with_shape(M, 4096, 4096)
+    _forward_check(H, orc, make_x(wl), make_w(wl), 4, rows=sample_rows(M, 16))
+
+
+# ----------------------------------------------------------------- error path
+
+def test_device_error_word(H):
+    import torch
+    assert H.hbl_last_device_error() == H.HBL_OK
+    H.hbl_debug_raise_device_error()
+    assert H.hbl_last_device_error() == H.HBL_ERR_TIMEOUT
+    assert H.hbl_last_device_error() == H.HBL_OK
+    torch.cuda.synchronize()
