@@ -1,0 +1,439 @@
+#!/usr/bin/env python
+"""Benchmark of the H-BitLinear forward (BitNet v2) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step is one whole forward -- LayerNorm, Hadamard transform, INT4 absmean
+quantization, ternary int8 GEMM on the tensor cores, dequantisation -- over
+one batch of the 7B-like Wdown workload (M=8192 tokens, K=16384, N=4096, bf16
+in and out).  Ternarising the weight happens once before timing (weights are
+static at inference).  The input (268 MB of bf16) is larger than the 126 MB
+L2, so no step finds the previous step's activations in cache.
+
+Rank 0 prints one JSON line.  `value` is tokens/s of the whole job (every rank
+runs its own replica of the workload: the path shards over tokens with no
+collective, so scaling is weak), from CUDA events on the launching stream,
+max over ranks.  Extra keys: the roofline of the dominant kernel (the GEMM,
+timed per launch with CUDA events on its stream through the stage entry
+points), the LN+FHT+quant kernel's HBM figure, an end-to-end figure through
+host memory, the oracle on host cores, and SM clocks sampled during timing.
+
+`--impl reference` times the CPU oracle (the pages publish no code to run) on
+bounded samples of the same workload, on rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "H-BitLinear fwd tokens/s + INT8-MMA TOPS (7B Wdown); FHT+quant HBM GB/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+INT8_OVER_BF16 = 2.0  # nominal dense ratio on B200: 4.5 POPS int8 vs 2.25 PFLOP/s bf16
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="wdown_7b")
+    ap.add_argument("--bits", type=int, default=4, choices=[4, 8])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--sweep", choices=["k1", "fwd"], default=None,
+                    help="instead of the step line: the LN+FHT+INT4 kernel alone at M=65536 for each K, "
+                         "or the whole forward at K=N=4096 for each M (one JSON line per point)")
+    a = ap.parse_args(argv)
+    a.warmup = max(3, a.warmup)
+    return a
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ------------------------------------------------------------------ ranks
+
+class Ranks:
+    """torch.distributed plumbing: barrier and max-over-ranks, nothing on the data path."""
+
+    def __init__(self, backend: str):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.pg = None
+        if self.world > 1:
+            import datetime
+            import torch.distributed as dist
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=180))
+            self.pg = dist
+
+    def barrier(self):
+        if self.pg is not None:
+            self.pg.barrier()
+
+    def max(self, v: float, device=None) -> float:
+        if self.pg is None:
+            return v
+        import torch
+        t = torch.tensor([float(v)], dtype=torch.float64, device=device)
+        self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.pg is not None:
+            self.pg.destroy_process_group()
+
+
+def aggregate_value(tokens_per_rank: int, world: int, max_seconds_per_step: float) -> float:
+    """Whole-job throughput: all ranks' tokens over the slowest rank's step time."""
+    return tokens_per_rank * world / max_seconds_per_step
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """nvidia-smi samples (200 ms) of SM clock and throttle reasons while timing."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.lines = []
+        self.t = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", self.gpu_id, "--query-gpu=" + self.FIELDS,
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.t.join(timeout=2)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        load = [s for s in sm if mx and s > 0.3 * max(mx)] or sm
+        return {"sm_mhz": statistics.median(load) if load else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ CPU baseline (oracle)
+
+def oracle_rows_per_second(wl, bits: int, seconds: float, max_rows: int = 512):
+    """Time the oracle's forward on consecutive seeded rows until `seconds` pass."""
+    import numpy as np
+    import oracle
+    from ternary_gemm_b200.inputs import make_w, make_x_rows
+    oracle.build()
+    w, a = oracle.ternary(make_w(wl))
+    rows = np.arange(min(max_rows, wl.M), dtype=np.int64)
+    x = make_x_rows(wl, rows)
+    done, t0 = 0, time.perf_counter()
+    while done < rows.size:
+        oracle.forward_rows(x[done:done + 1], w, a, bits)
+        done += 1
+        if time.perf_counter() - t0 >= seconds:
+            break
+    dt = time.perf_counter() - t0
+    return done / dt, done, dt
+
+
+def run_reference(args):
+    """The reference arm: the CPU oracle on bounded samples, rank 0 only."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import numpy as np
+    import oracle
+    from ternary_gemm_b200.inputs import WORKLOADS, make_w, make_x_rows
+    wl = WORKLOADS[args.workload]
+    oracle.build()
+    w, a = oracle.ternary(make_w(wl))
+    per_step = 1
+    x = make_x_rows(wl, np.arange((args.warmup + args.steps) * per_step, dtype=np.int64) % wl.M)
+    for s in range(args.warmup):
+        oracle.forward_rows(x[s:s + 1], w, a, args.bits)
+    t0 = time.perf_counter()
+    for s in range(args.warmup, args.warmup + args.steps):
+        oracle.forward_rows(x[s:s + 1], w, a, args.bits)
+    dt = time.perf_counter() - t0
+    value = args.steps * per_step / dt
+    sample = ("%d rows of %s (M=%d K=%d N=%d, INT%d), one row per step: LN+FHT+quant+GEMM+dequant in the "
+              "single-threaded C oracle" % (args.steps, wl.name, wl.M, wl.K, wl.N, args.bits))
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": int(os.environ.get("WORLD_SIZE", "1")),
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3 / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
+            "impl": "reference",
+            "config": {"workload": wl.name, "M": wl.M, "K": wl.K, "N": wl.N, "bits": args.bits,
+                       "x_dtype": wl.dtype, "parallelism": "replicas"},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ ours
+
+def _to_device(a):
+    import numpy as np
+    import torch
+    if a.dtype == np.uint16:
+        return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).cuda()
+    return torch.from_numpy(a).cuda()
+
+
+def bench_ours(args):
+    import numpy as np
+    import torch
+    from ternary_gemm_b200 import build as hbl_build
+    hbl_build.build()
+    import ternary_gemm_b200 as hbl
+    from ternary_gemm_b200.inputs import WORKLOADS, make_w, make_x
+
+    ranks = Ranks("nccl")
+    torch.cuda.set_device(ranks.local)
+    dev = torch.device("cuda", ranks.local)
+    wl = WORKLOADS[args.workload]
+    M, K, N, bits = wl.M, wl.K, wl.N, args.bits
+    peaks, peak_kind = load_peaks()
+
+    # CPU baseline first, before any GPU work in this process (rank 0, N = 1 only)
+    cpu = None
+    if ranks.rank == 0 and ranks.world == 1 and not args.no_cpu_baseline:
+        v, n, dt = oracle_rows_per_second(wl, bits, args.cpu_seconds)
+        cpu = {"value": v, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+               "sample": "%d rows of %s (K=%d, N=%d, INT%d) through LN+FHT+quant+GEMM+dequant, single-threaded C "
+                         "oracle, %.1f s" % (n, wl.name, K, N, bits, dt)}
+
+    x = _to_device(make_x(wl))
+    W = _to_device(make_w(wl))
+    stream = torch.cuda.current_stream()
+    packed, alpha = hbl.hbl_pack_ternary(W)
+    del W
+    y = torch.empty((M, N), dtype=x.dtype, device=dev)
+    ws = torch.empty((hbl.hbl_forward_workspace_bytes(M, K, N, bits),), dtype=torch.uint8, device=dev)
+
+    def step():
+        hbl.hbl_forward(x, packed, alpha, N, bits, y=y, workspace=ws)
+
+    gpu_uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    clocks = ClockSampler(gpu_uuid)
+    clocks.start()
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+
+    # -------- headline: K whole forwards
+    ranks.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    e1.synchronize()
+    ranks.barrier()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.steps
+    ms_max = ranks.max(ms, dev)
+    value = aggregate_value(M, ranks.world, ms_max / 1e3)
+
+    # -------- per-kernel times through the stage entry points (same kernels as hbl_forward)
+    A = torch.empty((M, K), dtype=torch.int8, device=dev)
+    sc = torch.empty((M,), dtype=torch.float32, device=dev)
+    Wi = torch.empty((N, K), dtype=torch.int8, device=dev)
+    nst = max(20, min(args.steps, 200))
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(nst)]
+    for _ in range(3):
+        hbl.hbl_fht_quant_i8(x, bits, codes=A, scales=sc)
+        hbl.hbl_widen_ternary(packed, K, w=Wi)
+        hbl.hbl_gemm_dequant(A, Wi, sc, alpha, y=y)
+    torch.cuda.synchronize()
+    for i in range(nst):
+        evs[i][0].record(stream)
+        hbl.hbl_fht_quant_i8(x, bits, codes=A, scales=sc)
+        evs[i][1].record(stream)
+        hbl.hbl_widen_ternary(packed, K, w=Wi)
+        evs[i][2].record(stream)
+        hbl.hbl_gemm_dequant(A, Wi, sc, alpha, y=y)
+        evs[i][3].record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    t_k1 = statistics.mean(e[0].elapsed_time(e[1]) for e in evs) / 1e3
+    t_wd = statistics.mean(e[1].elapsed_time(e[2]) for e in evs) / 1e3
+    t_gm = statistics.mean(e[2].elapsed_time(e[3]) for e in evs) / 1e3
+    t_gm = ranks.max(t_gm, dev)
+    t_k1 = ranks.max(t_k1, dev)
+
+    ops = 2.0 * M * N * K
+    int8_peak = peaks["bf16_tflops"] * INT8_OVER_BF16
+    achieved_tops = ops / t_gm / 1e12
+    k1_bytes = M * K * (2 if wl.dtype == "bf16" else 4) + M * K + 4 * M
+    k1_gbs = k1_bytes / t_k1 / 1e9
+    roofline = {"bound": "tensor", "kernel": "gemm_i8_kernel (tcgen05 kind::i8 + dequant epilogue)",
+                "achieved": achieved_tops, "peak": int8_peak, "unit": "TFLOP/s", "frac": achieved_tops / int8_peak,
+                "traffic": None,
+                "peak_source": "%s bf16 burst %.1f TFLOP/s x %.0f (nominal int8/bf16 dense ratio)"
+                               % (peak_kind, peaks["bf16_tflops"], INT8_OVER_BF16),
+                "algorithmic_ops_per_launch": ops, "launch_ms": t_gm * 1e3,
+                "frac_of_nominal_4500": achieved_tops / 4500.0}
+    k1 = {"bound": "hbm", "kernel": "ln_fht_quant_kernel (INT%d, int8 codes out)" % bits, "achieved": k1_gbs,
+          "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": k1_gbs / peaks["hbm_gbs"],
+          "algorithmic_bytes_per_launch": k1_bytes, "launch_ms": t_k1 * 1e3}
+
+    # -------- end to end through host memory (pinned), the public call
+    e2e = None
+    if not args.no_e2e:
+        xh = torch.empty(x.shape, dtype=x.dtype, pin_memory=True)
+        xh.copy_(x)
+        yh = torch.empty(y.shape, dtype=y.dtype, pin_memory=True)
+        xd = torch.empty_like(x)
+        for _ in range(2):
+            xd.copy_(xh, non_blocking=True)
+            hbl.hbl_forward(xd, packed, alpha, N, bits, y=y, workspace=ws)
+            yh.copy_(y, non_blocking=True)
+        torch.cuda.synchronize()
+        ranks.barrier()
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for _ in range(args.e2e_steps):
+            xd.copy_(xh, non_blocking=True)
+            hbl.hbl_forward(xd, packed, alpha, N, bits, y=y, workspace=ws)
+            yh.copy_(y, non_blocking=True)
+        f1.record(stream)
+        f1.synchronize()
+        ranks.barrier()
+        e2e_ms = ranks.max(f0.elapsed_time(f1) / args.e2e_steps, dev)
+        e2e = {"value": aggregate_value(M, ranks.world, e2e_ms / 1e3), "unit": "tokens/s",
+               "h2d_bytes_per_step": x.numel() * x.element_size(),
+               "d2h_bytes_per_step": y.numel() * y.element_size(), "ms_per_step": e2e_ms}
+
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ranks.world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "int8", "data": "synthetic",
+            "config": {"workload": wl.name, "M": M, "K": K, "N": N, "bits": bits, "x_dtype": wl.dtype,
+                       "y_dtype": wl.dtype, "l2": "inputs larger than L2 (x is %d MB per step)"
+                       % (x.numel() * x.element_size() // 2 ** 20), "parallelism": "replicas"},
+            "roofline": roofline, "k1": k1, "int8_tops": achieved_tops,
+            "stages_ms": {"ln_fht_quant": t_k1 * 1e3, "widen_ternary": t_wd * 1e3, "gemm_dequant": t_gm * 1e3},
+            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 3 * args.steps, "clocks": clk}
+    if ranks.rank == 0:
+        print(json.dumps(line), flush=True)
+    ranks.barrier()
+    ranks.close()
+    return 0
+
+
+def bench_sweep(args):
+    """Size sweeps (one JSON line per point, rank 0 / one GPU)."""
+    import numpy as np
+    import torch
+    from ternary_gemm_b200 import build as hbl_build
+    hbl_build.build()
+    import ternary_gemm_b200 as hbl
+    from ternary_gemm_b200.inputs import SWEEP_FWD_MS, SWEEP_K1_KS, WORKLOADS, make_w, make_x
+    peaks, peak_kind = load_peaks()
+    base = WORKLOADS["sweep"]
+    reps = max(3, min(args.steps, 50))
+    stream = torch.cuda.current_stream()
+
+    def timed(fn, n):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(n):
+            fn()
+        b.record(stream)
+        b.synchronize()
+        return a.elapsed_time(b) / n / 1e3
+
+    if args.sweep == "k1":
+        M = 65536
+        for K in SWEEP_K1_KS:
+            distinct = 4096                      # 4096 seeded rows, repeated to M on the device
+            x = _to_device(make_x(base.with_shape(distinct, K, 256))).repeat(M // distinct, 1)
+            codes = torch.empty((M, K // 2), dtype=torch.uint8, device="cuda")
+            sc = torch.empty((M,), dtype=torch.float32, device="cuda")
+            t = timed(lambda: hbl.hbl_fht_quant(x, 4, codes=codes, scales=sc), reps)
+            nbytes = M * K * 2 + M * K // 2 + 4 * M
+            gbs = nbytes / t / 1e9
+            print(json.dumps({"sweep": "k1_ln_fht_int4", "M": M, "K": K, "ms": t * 1e3, "GB/s": gbs,
+                              "frac_hbm": gbs / peaks["hbm_gbs"], "peak_kind": peak_kind,
+                              "bytes_per_launch": nbytes, "input": "4096 seeded rows repeated to 65536"}),
+                  flush=True)
+            del x, codes, sc
+            torch.cuda.empty_cache()
+    else:
+        K = N = 4096
+        W = _to_device(make_w(base.with_shape(1, K, N)))
+        packed, alpha = hbl.hbl_pack_ternary(W)
+        for M in SWEEP_FWD_MS:
+            x = _to_device(make_x(base.with_shape(M, K, N)))
+            y = torch.empty((M, N), dtype=x.dtype, device="cuda")
+            ws = torch.empty((hbl.hbl_forward_workspace_bytes(M, K, N, 4),), dtype=torch.uint8, device="cuda")
+            t = timed(lambda: hbl.hbl_forward(x, packed, alpha, N, 4, y=y, workspace=ws), reps)
+            print(json.dumps({"sweep": "fwd_int4", "M": M, "K": K, "N": N, "us": t * 1e6, "tokens/s": M / t,
+                              "int8_tops": 2.0 * M * N * K / t / 1e12}), flush=True)
+    return 0
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.sweep:
+        return bench_sweep(args)
+    if args.impl == "reference":
+        return run_reference(args)
+    return bench_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

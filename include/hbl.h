@@ -121,6 +121,29 @@ hbl_status hbl_forward(const void* x, hbl_dtype xt, int64_t M, int64_t K, const 
                        const float* alpha_dev, int64_t N, int bits, void* y, hbl_dtype yt,
                        void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
+/* ---------------------------------------------------------------- forward stages
+ * hbl_forward is exactly these three calls on slices of its workspace; they
+ * are public so that callers can keep the widened weight resident, overlap
+ * stages, or time each kernel on their own stream. */
+
+/* Activation path with one int8 per code (the layout the tensor cores read):
+ * the same LN -> H -> quantizer as hbl_fht_quant, codes device int8 [M][K]
+ * (INT4 codes in [-8, 7], INT8 codes in [-128, 127]), scales device [M]. */
+hbl_status hbl_fht_quant_i8(const void* x, hbl_dtype xt, int64_t M, int64_t K, int bits, int8_t* codes,
+                            float* scales, cudaStream_t stream);
+
+/* Packed 2-bit ternary codes [N][K/4] -> int8 codes [N][K] (device). */
+hbl_status hbl_widen_ternary(const uint8_t* packed, int64_t K, int64_t N, int8_t* w, cudaStream_t stream);
+
+/* The integer GEMM with the dequantisation fused into its epilogue:
+ * y[m][n] = (float)(sum_k A[m][k] w[n][k]) * (scales[m] * alpha_dev[0]),
+ * stored as yt.  A device int8 [M][K], w device int8 [N][K], scales device
+ * float [M], alpha_dev device float, y device [M][N].  K a multiple of 16 up
+ * to 65536, N a multiple of 16. */
+hbl_status hbl_gemm_dequant(const int8_t* A, const int8_t* w, int64_t M, int64_t N, int64_t K,
+                            const float* scales, const float* alpha_dev, void* y, hbl_dtype yt,
+                            cudaStream_t stream);
+
 /* ---------------------------------------------------------------- test hooks */
 
 /* Stages 1-2 alone: t = H LN(x) / sqrt(K) as float [M][K] (device output).

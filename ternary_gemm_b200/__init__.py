@@ -62,6 +62,12 @@ def lib():
             L.hbl_fht_quant.restype = i32
             L.hbl_forward.argtypes = [p, i32, i64, i64, p, p, i64, i32, p, i32, p, sz, p]
             L.hbl_forward.restype = i32
+            L.hbl_fht_quant_i8.argtypes = [p, i32, i64, i64, i32, p, p, p]
+            L.hbl_fht_quant_i8.restype = i32
+            L.hbl_widen_ternary.argtypes = [p, i64, i64, p, p]
+            L.hbl_widen_ternary.restype = i32
+            L.hbl_gemm_dequant.argtypes = [p, p, i64, i64, i64, p, p, p, i32, p]
+            L.hbl_gemm_dequant.restype = i32
             L.hbl_debug_ln_fht.argtypes = [p, i32, i64, i64, p, p]
             L.hbl_debug_ln_fht.restype = i32
             L.hbl_quant_from_f32.argtypes = [p, i64, i64, i32, p, p, p]
@@ -179,6 +185,44 @@ def hbl_forward(x, packed, alpha, N: int, bits: int, y=None, y_dtype=None, works
         workspace = torch.empty((hbl_forward_workspace_bytes(M, K, N, bits),), dtype=torch.uint8, device=x.device)
     _check(lib().hbl_forward(_ptr(x), _dtype_code(x), M, K, _ptr(packed), _ptr(alpha), N, bits, _ptr(y),
                              _dtype_code(y), _ptr(workspace), workspace.numel(), _stream(stream)), "hbl_forward")
+    return y
+
+
+def hbl_fht_quant_i8(x, bits: int, codes=None, scales=None, stream=None):
+    """x [M][K] -> (int8 codes [M][K], one per byte, scales float32 [M])."""
+    torch = _torch()
+    _need_cuda(x)
+    M, K = x.shape
+    if codes is None:
+        codes = torch.empty((M, K), dtype=torch.int8, device=x.device)
+    if scales is None:
+        scales = torch.empty((M,), dtype=torch.float32, device=x.device)
+    _check(lib().hbl_fht_quant_i8(_ptr(x), _dtype_code(x), M, K, bits, _ptr(codes), _ptr(scales),
+                                  _stream(stream)), "hbl_fht_quant_i8")
+    return codes, scales
+
+
+def hbl_widen_ternary(packed, K: int, w=None, stream=None):
+    """Packed ternary [N][K/4] -> int8 codes [N][K]."""
+    torch = _torch()
+    _need_cuda(packed)
+    N = packed.shape[0]
+    if w is None:
+        w = torch.empty((N, K), dtype=torch.int8, device=packed.device)
+    _check(lib().hbl_widen_ternary(_ptr(packed), K, N, _ptr(w), _stream(stream)), "hbl_widen_ternary")
+    return w
+
+
+def hbl_gemm_dequant(A, w, scales, alpha, y=None, y_dtype=None, stream=None):
+    """int8 A [M][K], int8 w [N][K] -> y = (A w^T) * (scales[m] * alpha) [M][N]."""
+    torch = _torch()
+    _need_cuda(A, w, scales, alpha)
+    M, K = A.shape
+    N = w.shape[0]
+    if y is None:
+        y = torch.empty((M, N), dtype=y_dtype or torch.bfloat16, device=A.device)
+    _check(lib().hbl_gemm_dequant(_ptr(A), _ptr(w), M, N, K, _ptr(scales), _ptr(alpha), _ptr(y), _dtype_code(y),
+                                  _stream(stream)), "hbl_gemm_dequant")
     return y
 
 

@@ -6,21 +6,26 @@
 //
 // One row of K = 2^k elements is spread over T = K/64 threads holding 64
 // floats each in registers; R rows share a CTA so that a CTA has >= 128
-// threads.  The Sylvester transform is the product of one 2-point butterfly
-// per index bit, and those factors commute, so the k butterfly stages may run
-// in any order.  Three passes cover all bits with two trips through shared
-// memory:
+// threads, and registers are capped at 128 so that 2-4 CTAs share an SM (one
+// loads while another computes).  The Sylvester transform is the product of
+// one 2-point butterfly per index bit and those factors commute, so the k
+// stages may run in any order.  Three passes cover all bits with two trips
+// through shared memory:
 //   pass 1: coalesced 16-byte loads give each thread index bits {0,1,2} (within
 //           a 16-byte vector) and the top three bits {k-3,k-2,k-1} (eight
 //           vectors T*8 elements apart); those 6 stages run in registers.
-//   pass 2: (k >= 10) each thread reads the 2^(k-9) elements spanning bits
-//           {6..k-4} from shared memory and runs those stages.
+//   pass 2: (k >= 10) each thread reads 2^(k-9) vectors of 2^(15-k) contiguous
+//           floats spanning bits {6..k-4} and runs those stages.
 //   pass 3: each thread reads 64 contiguous elements (bits 0..5) and runs the
-//           stages of bits {3,4,5} not done yet; the row is then complete and
-//           contiguous per thread, ready for the quantizer and 16-byte stores.
-// Shared memory uses an XOR swizzle of index bits 5..8 into bits 2..4 that
-// keeps the vector writes of pass 1, the scalar accesses of pass 2 and the
-// vector reads of pass 3 free of bank conflicts.
+//           stages of bits {3,4,5} not done yet; the row is complete and each
+//           thread's slice is contiguous, ready for the quantizer and 16-byte
+//           stores.
+// Shared memory uses an XOR swizzle of index bits 5..8 into bits 2..4; it is
+// linear over GF(2), so an address splits into a per-thread part (eight
+// precomputed bases) and a compile-time offset, and it keeps the accesses of
+// all three passes free of bank conflicts.  Butterflies, scaling and the
+// quantizer's products run as paired f32x2 instructions (one issue slot for
+// two IEEE float operations).
 //
 // LayerNorm is folded around the transform: a row offset mu~ (the mean of the
 // row's first 8 values, identical in every thread) is subtracted first so
@@ -43,28 +48,105 @@ struct Shape {
   static constexpr int T = K / E;                       // threads per row
   static constexpr int R = T >= 128 ? 1 : 128 / T;      // rows per CTA
   static constexpr int THREADS = T * R;
+  static constexpr int MINB = THREADS >= 512 ? 1 : (THREADS >= 256 ? 2 : 4);  // -> <= 128 registers
   static constexpr int PAD = T < 32 ? 16 : 0;           // floats of padding per row
   static constexpr int STRIDE = K + PAD;                // floats per row in smem
   static constexpr int WPR = T > 32 ? T / 32 : 1;       // warps per row
   static constexpr size_t SMEM = (size_t)R * STRIDE * 4 + (size_t)R * WPR * 8;
+  static constexpr int NPB = LOGK >= 10 ? LOGK - 9 : 0;  // pass-2 processed bits {6 .. 5+NPB}
+  static constexpr int PB = 6 - NPB;                      // pass-2 vector bits {0 .. PB-1}
 };
 
-__device__ __forceinline__ int swz(int i) {
-  int f = ((((i >> 5) ^ (i >> 6)) & 1) << 2) | (((i >> 7) & 1) << 3) | (((i >> 8) & 1) << 4);
-  return i ^ f;
+// The swizzle: index bits 5..8 XORed into bits 2..4 (linear over GF(2)).
+__host__ __device__ constexpr int swz(int i) {
+  return i ^ (((((i >> 5) ^ (i >> 6)) & 1) << 2) | (((i >> 7) & 1) << 3) | (((i >> 8) & 1) << 4));
+}
+
+// Shared-memory addresses of index (tb | C) for a per-thread tb and a
+// compile-time C with disjoint bits: swz(tb | C) = swz(tb) ^ swz(C); the XOR
+// part of swz(C) falls in bits 2..4 and selects one of eight bases, the rest
+// is an immediate offset.
+struct SwzBase {
+  int b[8];
+  __device__ __forceinline__ SwzBase(int row_off, int tb) {
+    const int s = swz(tb);
+#pragma unroll
+    for (int v = 0; v < 8; ++v) b[v] = row_off + (s ^ (v << 2));
+  }
+  template <int C>
+  __device__ __forceinline__ int at() const {
+    constexpr int sc = swz(C);
+    return b[(sc >> 2) & 7] + (sc & ~0x1C);
+  }
+};
+
+// ---------------------------------------------------------------- paired float ops
+
+__device__ __forceinline__ void bfly2(float& a0, float& a1, float& b0, float& b1) {
+  asm("{\n\t.reg .b64 A, B, S, D;\n\t"
+      "mov.b64 A, {%0, %1};\n\tmov.b64 B, {%2, %3};\n\t"
+      "add.rn.f32x2 S, A, B;\n\tsub.rn.f32x2 D, A, B;\n\t"
+      "mov.b64 {%0, %1}, S;\n\tmov.b64 {%2, %3}, D;\n\t}"
+      : "+f"(a0), "+f"(a1), "+f"(b0), "+f"(b1));
+}
+
+__device__ __forceinline__ void sub2(float& a0, float& a1, float c) {
+  asm("{\n\t.reg .b64 A, C;\n\t"
+      "mov.b64 A, {%0, %1};\n\tmov.b64 C, {%2, %2};\n\t"
+      "sub.rn.f32x2 A, A, C;\n\tmov.b64 {%0, %1}, A;\n\t}"
+      : "+f"(a0), "+f"(a1) : "f"(c));
+}
+
+__device__ __forceinline__ void mul2(float& a0, float& a1, float c) {
+  asm("{\n\t.reg .b64 A, C;\n\t"
+      "mov.b64 A, {%0, %1};\n\tmov.b64 C, {%2, %2};\n\t"
+      "mul.rn.f32x2 A, A, C;\n\tmov.b64 {%0, %1}, A;\n\t}"
+      : "+f"(a0), "+f"(a1) : "f"(c));
+}
+
+// (s0, s1) += (a0*a0, a1*a1)
+__device__ __forceinline__ void sq_acc2(float& s0, float& s1, float a0, float a1) {
+  asm("{\n\t.reg .b64 A, S;\n\t"
+      "mov.b64 A, {%2, %3};\n\tmov.b64 S, {%0, %1};\n\t"
+      "fma.rn.f32x2 S, A, A, S;\n\tmov.b64 {%0, %1}, S;\n\t}"
+      : "+f"(s0), "+f"(s1) : "f"(a0), "f"(a1));
+}
+
+// bits of fl(fl(t * r) + 1.5*2^23) for a pair (see q::rint_code)
+__device__ __forceinline__ void magic2(float t0, float t1, float r, uint32_t& m0, uint32_t& m1) {
+  asm("{\n\t.reg .b64 A, R, M;\n\t"
+      "mov.b64 A, {%2, %3};\n\tmov.b64 R, {%4, %4};\n\tmov.b64 M, {%5, %5};\n\t"
+      "mul.rn.f32x2 A, A, R;\n\tadd.rn.f32x2 A, A, M;\n\t"
+      "mov.b64 {%0, %1}, A;\n\t}"
+      : "=r"(m0), "=r"(m1) : "f"(t0), "f"(t1), "f"(r), "f"(q::kMagic));
 }
 
 // Butterfly over register-index bit B: (e[r], e[r + 2^B]) -> (sum, difference).
 template <int B, int N>
 __device__ __forceinline__ void stage(float (&e)[N]) {
+  if constexpr (B == 0) {
 #pragma unroll
-  for (int r = 0; r < N; ++r) {
-    if (!(r & (1 << B))) {
-      float a = e[r], c = e[r | (1 << B)];
+    for (int r = 0; r < N; r += 2) {
+      float a = e[r], c = e[r + 1];
       e[r] = a + c;
-      e[r | (1 << B)] = a - c;
+      e[r + 1] = a - c;
     }
+  } else {
+#pragma unroll
+    for (int r = 0; r < N; r += 2)
+      if (!(r & (1 << B))) bfly2(e[r], e[r + 1], e[r | (1 << B)], e[(r | (1 << B)) + 1]);
   }
+}
+
+template <int N>
+__device__ __forceinline__ void stage_range(float (&e)[N], int lo, int hi) {
+  // register bits lo..hi-1 (lo, hi compile-time after inlining)
+  if (lo <= 0 && 0 < hi) stage<0>(e);
+  if (lo <= 1 && 1 < hi) stage<1>(e);
+  if (lo <= 2 && 2 < hi) stage<2>(e);
+  if (lo <= 3 && 3 < hi) stage<3>(e);
+  if (lo <= 4 && 4 < hi) stage<4>(e);
+  if (lo <= 5 && 5 < hi) stage<5>(e);
 }
 
 // Row-wide all-reduce over the T threads of a row (deterministic order: every
@@ -109,7 +191,6 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4& u, float* o) {
   o[7] = __uint_as_float(u.w & 0xffff0000u);
 }
 
-// 8 consecutive input values starting at element `i` of the row.
 template <bool BF16>
 __device__ __forceinline__ void load8(const void* xrow, int i, float* o) {
   if constexpr (BF16) {
@@ -123,14 +204,79 @@ __device__ __forceinline__ void load8(const void* xrow, int i, float* o) {
   }
 }
 
-// Index bit j of the "other" bits of pass 2: {0,1,2,3,4,5,k-3,k-2,k-1}.
+// Thread bit j of pass 2 -> index bit: {PB .. 5} then {k-3, k-2, k-1}.
 template <int LOGK>
-__host__ __device__ constexpr int other_bit(int j) {
-  return j < 6 ? j : LOGK - 9 + j;
+__host__ __device__ constexpr int p2_bit(int j) {
+  return j < 6 - Shape<LOGK>::PB ? Shape<LOGK>::PB + j : LOGK - 3 + (j - (6 - Shape<LOGK>::PB));
+}
+
+// 4 floats (or fewer, for vectors narrower than 16 bytes) at a smem address.
+template <int W>
+__device__ __forceinline__ void lds(const float* s, int a, float* o) {
+  if constexpr (W == 4) {
+    float4 v = *reinterpret_cast<const float4*>(s + a);
+    o[0] = v.x; o[1] = v.y; o[2] = v.z; o[3] = v.w;
+  } else if constexpr (W == 2) {
+    float2 v = *reinterpret_cast<const float2*>(s + a);
+    o[0] = v.x; o[1] = v.y;
+  } else {
+    o[0] = s[a];
+  }
+}
+
+template <int W>
+__device__ __forceinline__ void sts(float* s, int a, const float* o) {
+  if constexpr (W == 4) {
+    *reinterpret_cast<float4*>(s + a) = make_float4(o[0], o[1], o[2], o[3]);
+  } else if constexpr (W == 2) {
+    *reinterpret_cast<float2*>(s + a) = make_float2(o[0], o[1]);
+  } else {
+    s[a] = o[0];
+  }
+}
+
+template <int LOGK, int R0, int NREG>
+struct Pass2 {
+  // registers r = p * 2^PB + v  <->  index tb | (p << 6) | v; chunks of W floats
+  static constexpr int PB = Shape<LOGK>::PB;
+  static constexpr int W = PB >= 2 ? 4 : (PB == 1 ? 2 : 1);
+  template <int R>
+  __device__ __forceinline__ static void load(float (&e)[64], const float* smem, const SwzBase& sb) {
+    if constexpr (R < 64) {
+      constexpr int p = R >> PB, v = R & ((1 << PB) - 1);
+      lds<W>(smem, sb.at<(p << 6) | v>(), &e[R]);
+      load<R + W>(e, smem, sb);
+    }
+  }
+  template <int R>
+  __device__ __forceinline__ static void store(const float (&e)[64], float* smem, const SwzBase& sb) {
+    if constexpr (R < 64) {
+      constexpr int p = R >> PB, v = R & ((1 << PB) - 1);
+      sts<W>(smem, sb.at<(p << 6) | v>(), &e[R]);
+      store<R + W>(e, smem, sb);
+    }
+  }
+};
+
+template <int J>
+__device__ __forceinline__ void load_pass3(float (&e)[64], const float* smem, const SwzBase& sb) {
+  if constexpr (J < 16) {
+    lds<4>(smem, sb.at<4 * J>(), &e[4 * J]);
+    load_pass3<J + 1>(e, smem, sb);
+  }
+}
+
+template <int JJ, int T>
+__device__ __forceinline__ void store_pass1(const float (&e)[64], float* smem, const SwzBase& sb) {
+  if constexpr (JJ < 8) {
+    sts<4>(smem, sb.at<JJ * T * 8>(), &e[JJ * 8]);
+    sts<4>(smem, sb.at<JJ * T * 8 + 4>(), &e[JJ * 8 + 4]);
+    store_pass1<JJ + 1, T>(e, smem, sb);
+  }
 }
 
 template <int LOGK, bool BF16, int MODE>
-__global__ void __launch_bounds__(Shape<LOGK>::THREADS, 1)
+__global__ void __launch_bounds__(Shape<LOGK>::THREADS, Shape<LOGK>::MINB)
 ln_fht_quant_kernel(const void* __restrict__ x, int64_t M, float sK, void* __restrict__ out,
                     float* __restrict__ scales) {
   using S = Shape<LOGK>;
@@ -146,7 +292,7 @@ ln_fht_quant_kernel(const void* __restrict__ x, int64_t M, float sK, void* __res
   const bool active = row < M;
   const size_t esz = BF16 ? 2 : 4;
   const void* xrow = reinterpret_cast<const unsigned char*>(x) + (size_t)(active ? row : 0) * K * esz;
-  float* srow = smem + rl * S::STRIDE;
+  const int row_off = rl * S::STRIDE;
 
   float e[64];
 
@@ -163,70 +309,46 @@ ln_fht_quant_kernel(const void* __restrict__ x, int64_t M, float sK, void* __res
     for (int r = 0; r < 64; ++r) e[r] = 0.0f;
   }
 #pragma unroll
-  for (int r = 0; r < 64; ++r) e[r] = e[r] - mu;
-  stage<0>(e); stage<1>(e); stage<2>(e); stage<3>(e); stage<4>(e); stage<5>(e);
-#pragma unroll
-  for (int jj = 0; jj < 8; ++jj) {
-    int i0 = (jj * T + t) * 8;
-    *reinterpret_cast<float4*>(srow + swz(i0)) = make_float4(e[jj * 8 + 0], e[jj * 8 + 1], e[jj * 8 + 2], e[jj * 8 + 3]);
-    *reinterpret_cast<float4*>(srow + swz(i0 + 4)) = make_float4(e[jj * 8 + 4], e[jj * 8 + 5], e[jj * 8 + 6], e[jj * 8 + 7]);
+  for (int r = 0; r < 64; r += 2) sub2(e[r], e[r + 1], mu);
+  stage_range(e, 0, 6);
+  {
+    SwzBase sb(row_off, t * 8);
+    store_pass1<0, T>(e, smem, sb);
   }
   __syncthreads();
 
-  // ---- pass 2: stages of bits {6 .. k-4}
+  // ---- pass 2: stages of bits {6 .. k-4} on vectors of 2^PB floats
   if constexpr (LOGK >= 10) {
-    constexpr int NPB = LOGK - 9;
-    constexpr int NP = 1 << NPB;
-    constexpr int G = 64 / NP;
     int tb = 0;
 #pragma unroll
-    for (int j = 0; j < LOGK - 6; ++j) tb |= ((t >> j) & 1) << other_bit<LOGK>(j);
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-      int gb = 0;
-#pragma unroll
-      for (int j = 0; j < 15 - LOGK; ++j) gb |= ((g >> j) & 1) << other_bit<LOGK>(LOGK - 6 + j);
-#pragma unroll
-      for (int p = 0; p < NP; ++p) e[g * NP + p] = srow[swz(tb | gb | (p << 6))];
-    }
-    if constexpr (NPB > 0) stage<0>(e);
-    if constexpr (NPB > 1) stage<1>(e);
-    if constexpr (NPB > 2) stage<2>(e);
-    if constexpr (NPB > 3) stage<3>(e);
-    if constexpr (NPB > 4) stage<4>(e);
-    if constexpr (NPB > 5) stage<5>(e);
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-      int gb = 0;
-#pragma unroll
-      for (int j = 0; j < 15 - LOGK; ++j) gb |= ((g >> j) & 1) << other_bit<LOGK>(LOGK - 6 + j);
-#pragma unroll
-      for (int p = 0; p < NP; ++p) srow[swz(tb | gb | (p << 6))] = e[g * NP + p];
-    }
+    for (int j = 0; j < LOGK - 6; ++j) tb |= ((t >> j) & 1) << p2_bit<LOGK>(j);
+    SwzBase sb(row_off, tb);
+    Pass2<LOGK, 0, 64>::template load<0>(e, smem, sb);
+    stage_range(e, S::PB, 6);
+    Pass2<LOGK, 0, 64>::template store<0>(e, smem, sb);
     __syncthreads();
   }
 
   // ---- pass 3: 64 contiguous elements per thread, stages of bits {3,4,5} left
   const int base = t * 64;
-#pragma unroll
-  for (int j = 0; j < 16; ++j) {
-    float4 v = *reinterpret_cast<const float4*>(srow + swz(base + 4 * j));
-    e[4 * j + 0] = v.x; e[4 * j + 1] = v.y; e[4 * j + 2] = v.z; e[4 * j + 3] = v.w;
+  {
+    SwzBase sb(row_off, base);
+    load_pass3<0>(e, smem, sb);
   }
-  if constexpr (3 < LOGK - 3) stage<3>(e);
-  if constexpr (4 < LOGK - 3) stage<4>(e);
-  if constexpr (5 < LOGK - 3) stage<5>(e);
+  stage_range(e, 3, LOGK - 3 < 6 ? LOGK - 3 : 6);
 
   // ---- LayerNorm statistics from the transform: K^2 var = sum_{i>=1} Y_i^2
-  float ss = 0.0f;
+  float s0 = 0.0f, s1 = 0.0f;
+  const float e0 = e[0];
+  if (t == 0) e[0] = 0.0f;
 #pragma unroll
-  for (int r = 1; r < 64; ++r) ss = fmaf(e[r], e[r], ss);
-  if (t != 0) ss = fmaf(e[0], e[0], ss);
-  ss = RowReduce<T, S::WPR>::run(ss, AddF(), reinterpret_cast<float*>(red), rl, t);
+  for (int r = 0; r < 64; r += 2) sq_acc2(s0, s1, e[r], e[r + 1]);
+  if (t == 0) e[0] = e0;
+  float ss = RowReduce<T, S::WPR>::run(s0 + s1, AddF(), reinterpret_cast<float*>(red), rl, t);
   const float var = ss * (1.0f / ((float)K * (float)K));
   const float cmul = __fmul_rn(__fdiv_rn(1.0f, sqrtf(__fadd_rn(var, 1e-5f))), sK);
 #pragma unroll
-  for (int r = 0; r < 64; ++r) e[r] = __fmul_rn(e[r], cmul);
+  for (int r = 0; r < 64; r += 2) mul2(e[r], e[r + 1], cmul);
   if (t == 0) e[0] = 0.0f;
 
   if constexpr (MODE == K1_T_F32) {
@@ -256,29 +378,29 @@ ln_fht_quant_kernel(const void* __restrict__ x, int64_t M, float sK, void* __res
     }
     if (!active) return;
     if (t == 0) scales[row] = p.scale;
+    uint32_t m[64];
+#pragma unroll
+    for (int r = 0; r < 64; r += 2) magic2(e[r], e[r + 1], p.r, m[r], m[r + 1]);
     if constexpr (MODE == K1_Q4_PACKED) {
       uint32_t w[8];
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
         int n[8];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) n[u] = q::rint_code(e[8 * j + u], p.r);
+        for (int u = 0; u < 8; ++u) n[u] = (int)m[8 * j + u] - q::kMagicBits;
         w[j] = q::pack_s4x8(n);
       }
       uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(out) + (size_t)row * (K / 2) + base / 2);
       dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
       dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
     } else {
+      if constexpr (MODE == K1_Q4_I8) {
+#pragma unroll
+        for (int r = 0; r < 64; ++r) m[r] = q::clip_magic_int4(m[r]);
+      }
       uint32_t w[16];
 #pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        int n0 = q::rint_code(e[4 * j + 0], p.r), n1 = q::rint_code(e[4 * j + 1], p.r);
-        int n2 = q::rint_code(e[4 * j + 2], p.r), n3 = q::rint_code(e[4 * j + 3], p.r);
-        if constexpr (MODE == K1_Q4_I8) {
-          n0 = q::clip_int4(n0); n1 = q::clip_int4(n1); n2 = q::clip_int4(n2); n3 = q::clip_int4(n3);
-        }
-        w[j] = q::pack_s8x4(n0, n1, n2, n3);
-      }
+      for (int j = 0; j < 16; ++j) w[j] = q::gather_low_bytes(m[4 * j], m[4 * j + 1], m[4 * j + 2], m[4 * j + 3]);
       uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(out) + (size_t)row * K + base);
 #pragma unroll
       for (int j = 0; j < 4; ++j) dst[j] = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
@@ -290,8 +412,7 @@ template <int LOGK, bool BF16, int MODE>
 cudaError_t launch_one(const void* x, int64_t M, void* out, float* scales, cudaStream_t stream) {
   using S = Shape<LOGK>;
   auto kern = ln_fht_quant_kernel<LOGK, BF16, MODE>;
-  static cudaError_t attr = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 (int)S::SMEM);
+  cudaError_t attr = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)S::SMEM);
   if (attr != cudaSuccess) return attr;
   const int64_t grid = (M + S::R - 1) / S::R;
   const float sK = (float)(1.0 / sqrt((double)S::K));

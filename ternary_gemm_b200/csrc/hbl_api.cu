@@ -140,6 +140,41 @@ hbl_status hbl_forward(const void* x, hbl_dtype xt, int64_t M, int64_t K, const 
   return cuda_status(e);
 }
 
+hbl_status hbl_fht_quant_i8(const void* x, hbl_dtype xt, int64_t M, int64_t K, int bits, int8_t* codes,
+                            float* scales, cudaStream_t stream) {
+  if (!x || !codes || !scales || !dtype_ok(xt) || (bits != 4 && bits != 8)) return HBL_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(codes, 16) || !aligned(scales, 4)) return HBL_ERR_INVALID_ARG;
+  int l;
+  hbl_status s = check_k(K, &l);
+  if (s != HBL_OK) return s;
+  if ((s = check_rows(M)) != HBL_OK) return s;
+  const K1Mode mode = bits == 4 ? hbl::K1_Q4_I8 : hbl::K1_Q8_I8;
+  return cuda_status(hbl::launch_ln_fht_quant(x, xt == HBL_BF16, M, l, mode, codes, scales, stream));
+}
+
+hbl_status hbl_widen_ternary(const uint8_t* packed, int64_t K, int64_t N, int8_t* w, cudaStream_t stream) {
+  if (!packed || !w) return HBL_ERR_INVALID_ARG;
+  if (!aligned(packed, 16) || !aligned(w, 16)) return HBL_ERR_INVALID_ARG;
+  int l;
+  hbl_status s = check_k(K, &l);
+  if (s != HBL_OK) return s;
+  if ((s = check_n(N)) != HBL_OK) return s;
+  return cuda_status(hbl::launch_widen_ternary(packed, N, K, w, stream));
+}
+
+hbl_status hbl_gemm_dequant(const int8_t* A, const int8_t* w, int64_t M, int64_t N, int64_t K, const float* scales,
+                            const float* alpha_dev, void* y, hbl_dtype yt, cudaStream_t stream) {
+  if (!A || !w || !scales || !alpha_dev || !y || !dtype_ok(yt)) return HBL_ERR_INVALID_ARG;
+  if (!aligned(A, 16) || !aligned(w, 16) || !aligned(scales, 4) || !aligned(alpha_dev, 4) || !aligned(y, 16))
+    return HBL_ERR_INVALID_ARG;
+  if (K <= 0) return HBL_ERR_INVALID_ARG;
+  if (K % 16 != 0 || K > 65536) return HBL_ERR_UNSUPPORTED;
+  hbl_status s = check_rows(M);
+  if (s != HBL_OK) return s;
+  if ((s = check_n(N)) != HBL_OK) return s;
+  return cuda_status(hbl::launch_gemm_i8(A, w, M, N, K, yt == HBL_BF16 ? 2 : 1, y, scales, alpha_dev, stream));
+}
+
 hbl_status hbl_debug_ln_fht(const void* x, hbl_dtype xt, int64_t M, int64_t K, float* t, cudaStream_t stream) {
   if (!x || !t || !dtype_ok(xt)) return HBL_ERR_INVALID_ARG;
   if (!aligned(x, 16) || !aligned(t, 16)) return HBL_ERR_INVALID_ARG;

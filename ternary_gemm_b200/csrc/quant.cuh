@@ -24,8 +24,18 @@ constexpr float kSqrt7 = 2.6457513110645906f;  // sqrt(7) rounded to float
 constexpr float kMagic = 12582912.0f;          // 1.5 * 2^23
 constexpr int kMagicBits = 0x4B400000;
 
-// |t| as a double, for the absmean accumulation.
-__device__ __forceinline__ double abs_f64(float t) { return (double)fabsf(t); }
+// |t| as a double, for the absmean accumulation, built with integer
+// operations instead of a float->double conversion (which runs on the
+// quarter-rate conversion pipe): for a normal float the double has the same
+// sign, exponent + 896 and the mantissa shifted by 29, so the value is exact.
+// Zero maps to zero.  |t| below 2^-126 (subnormal) maps into [2^-127, 2^-126),
+// i.e. it is counted with an absolute error below 2^-126 -- invisible at float
+// resolution for any row whose sum of |t| exceeds 2^-100.
+__device__ __forceinline__ double abs_f64(float t) {
+  const uint32_t b = __float_as_uint(t) & 0x7fffffffu;
+  const uint32_t hi = b ? (b >> 3) + 0x38000000u : 0u;
+  return __hiloint2double((int)hi, (int)(b << 29));
+}
 
 struct RowParams {
   float r;      // multiplier applied to t before rounding
@@ -81,6 +91,19 @@ __device__ __forceinline__ uint32_t pack_s8x4(int n0, int n1, int n2, int n3) {
 }
 
 __device__ __forceinline__ int clip_int4(int n) { return max(-8, min(7, n)); }
+
+// The bits of fl(fl(t r) + 1.5*2^23) are kMagicBits + rint(t r), so clipping
+// the bits clips the code, and the low byte is the code as an int8.
+__device__ __forceinline__ uint32_t clip_magic_int4(uint32_t m) {
+  return (uint32_t)max(kMagicBits - 8, min(kMagicBits + 7, (int)m));
+}
+
+// Low bytes of four words -> one word, a in the lowest byte.
+__device__ __forceinline__ uint32_t gather_low_bytes(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  const uint32_t ab = __byte_perm(a, b, 0x0040);
+  const uint32_t cd = __byte_perm(c, d, 0x0040);
+  return __byte_perm(ab, cd, 0x5410);
+}
 
 }  // namespace q
 }  // namespace hbl

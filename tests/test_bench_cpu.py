@@ -1,0 +1,94 @@
+"""Host logic of bench.py on CPU: max-over-ranks timing and whole-job
+aggregation across two gloo ranks, the reference arm's rank gating, and the
+clock-sample parser."""
+import json
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+import bench  # noqa: E402
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    p = s.getsockname()[1]
+    s.close()
+    return p
+
+
+def _rank_main(rank, world, port, out_dir):
+    os.environ.update({"RANK": str(rank), "WORLD_SIZE": str(world), "LOCAL_RANK": str(rank),
+                       "MASTER_ADDR": "127.0.0.1", "MASTER_PORT": str(port)})
+    r = bench.Ranks("gloo")
+    r.barrier()
+    ms = 10.0 + 5.0 * rank                      # rank 1 is the slower one
+    m = r.max(ms)
+    value = bench.aggregate_value(8192, r.world, m / 1e3)
+    with open(os.path.join(out_dir, "rank%d.json" % rank), "w") as f:
+        json.dump({"max": m, "value": value, "world": r.world}, f)
+    r.barrier()
+    r.close()
+
+
+def test_two_rank_max_and_aggregate(tmp_path):
+    import torch.multiprocessing as mp
+    port = _free_port()
+    mp.start_processes(_rank_main, args=(2, port, str(tmp_path)), nprocs=2, join=True, start_method="spawn")
+    res = [json.load(open(tmp_path / ("rank%d.json" % r))) for r in range(2)]
+    for d in res:
+        assert d["world"] == 2
+        assert d["max"] == 15.0                  # every rank sees the slowest rank's time
+        assert d["value"] == pytest.approx(2 * 8192 / 0.015)
+
+
+def test_aggregate_single():
+    assert bench.aggregate_value(8192, 1, 0.5e-3) == pytest.approx(16384000.0)
+
+
+def test_reference_arm_nonzero_rank_exits_without_work(tmp_path):
+    env = dict(os.environ, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1")
+    p = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1",
+                        "--warmup", "3"], env=env, capture_output=True, text=True, timeout=120)
+    assert p.returncode == 0 and p.stdout.strip() == ""
+
+
+def test_reference_arm_line(tmp_path):
+    env = dict(os.environ, RANK="0", WORLD_SIZE="1", LOCAL_RANK="0")
+    p = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "2",
+                        "--warmup", "3", "--workload", "wo_1p3b"], env=env, capture_output=True, text=True,
+                       timeout=300)
+    assert p.returncode == 0, p.stderr
+    line = json.loads(p.stdout.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["value"] > 0 and line["unit"] == "tokens/s"
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"
+    assert line["cpu_baseline"]["value"] == line["value"]
+
+
+def test_clock_parser():
+    c = bench.ClockSampler("GPU-x")
+
+    class P:
+        def terminate(self):
+            pass
+
+        def wait(self, timeout=None):
+            return 0
+
+    class T:
+        def join(self, timeout=None):
+            pass
+
+    c.proc, c.t = P(), T()
+    c.lines = ["0, 1965, 1965, 700.5, 0x0, Not Active, Not Active, Not Active, Not Active",
+               "0, 1800, 1965, 990.0, 0x4, Not Active, Not Active, Not Active, Active",
+               "0, 1900, 1965, 950.0, 0x0, Not Active, Not Active, Not Active, Not Active",
+               "garbage"]
+    r = c.stop()
+    assert r["sm_mhz"] == 1900 and r["sm_max_mhz"] == 1965 and r["reasons"] == ["sw_power_cap"]
+    assert r["samples"] == 3
