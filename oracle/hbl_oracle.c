@@ -33,7 +33,8 @@
  * their integer decisions in single precision, as the GPU does: the mean of
  * |t| is accumulated in double and rounded once to float, the reciprocal
  * sqrt(7)/(beta+eps) is one IEEE float division per row, and each code is
- * rint of one float product.
+ * rint of the exact product of the float t and the float reciprocal (one
+ * rounding, half to even).
  */
 #include <fenv.h>
 #include <math.h>
@@ -180,8 +181,9 @@ int orc_quant(const float* t, int64_t M, int64_t K, int bits, int8_t* codes, flo
     volatile float den = stat + ORC_EPS_Q;  /* one float add */
     volatile float rcp = c / den;           /* one float division per row */
     for (int64_t i = 0; i < K; ++i) {
-      volatile float v = r[i] * rcp;        /* one float product per element */
-      double q = orc_rint((double)v);
+      /* rint of the exact product t * r: a product of two floats is exact in
+       * double, so this is one rounding to the nearest integer */
+      double q = orc_rint((double)r[i] * (double)rcp);
       if (q < lo) q = lo;
       if (q > hi) q = hi;
       codes[m * K + i] = (int8_t)q;
@@ -196,8 +198,9 @@ int orc_quant(const float* t, int64_t M, int64_t K, int bits, int8_t* codes, flo
 
 /* Per-tensor absmean ternarization of W [N][K] (row-major, out x in):
  * alpha = mean|W| (double sum, rounded once to float),
- * w = clip(rint(W / (alpha + eps)), -1, 1) computed as W * (1/(alpha+eps)) in
- * float.  ("per-tensor absmean quantizes the weights to {-1, 0, 1}") */
+ * w = clip(rint(W / (alpha + eps)), -1, 1) computed as rint of the exact
+ * product W * r with the float reciprocal r = 1/(alpha+eps).
+ * ("per-tensor absmean quantizes the weights to {-1, 0, 1}") */
 void orc_ternary(const void* W, int dtype, int64_t N, int64_t K, int8_t* w, float* alpha) {
   fesetround(FE_TONEAREST);
   double s = 0.0;
@@ -207,8 +210,7 @@ void orc_ternary(const void* W, int dtype, int64_t N, int64_t K, int8_t* w, floa
   volatile float den = a + ORC_EPS_Q;
   volatile float rcp = 1.0f / den;
   for (int64_t i = 0; i < n; ++i) {
-    volatile float v = (float)orc_load(W, dtype, i) * rcp;
-    double q = orc_rint((double)v);
+    double q = orc_rint(orc_load(W, dtype, i) * (double)rcp);   /* exact product, one rounding */
     if (q < -1.0) q = -1.0;
     if (q > 1.0) q = 1.0;
     w[i] = (int8_t)q;

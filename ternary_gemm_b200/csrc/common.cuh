@@ -49,7 +49,9 @@ cudaError_t launch_gemm_i8(const int8_t* A, const int8_t* B, int64_t M, int64_t 
                            int y_mode, void* y, const float* scales, const float* alpha,
                            cudaStream_t stream);
 
-// Device error word (bounded-wait timeouts) -- lives in gemm_i8.cu.
+// Device error word (bounded-wait timeouts) -- lives in gemm_i8.cu; kernels in
+// other translation units receive its device address.
+int* device_error_word();
 cudaError_t read_and_clear_device_error(cudaStream_t stream, int* value);
 cudaError_t raise_device_error(cudaStream_t stream);
 

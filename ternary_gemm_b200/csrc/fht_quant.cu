@@ -6,8 +6,9 @@
 //
 // One row of K = 2^k elements is spread over T = K/64 threads holding 64
 // floats each in registers; R rows share a CTA so that a CTA has >= 128
-// threads, and registers are capped at 128 so that 2-4 CTAs share an SM (one
-// loads while another computes).  The Sylvester transform is the product of
+// threads, and the register budget is set so that 3-5 CTAs share an SM: the
+// butterflies (FMA pipe), the integer work of the quantizer (ALU pipe) and
+// the exchanges (shared memory) of different rows then overlap.  The Sylvester transform is the product of
 // one 2-point butterfly per index bit and those factors commute, so the k
 // stages may run in any order.  Three passes cover all bits with two trips
 // through shared memory:
@@ -28,8 +29,9 @@
 // two IEEE float operations).
 //
 // LayerNorm is folded around the transform: a row offset mu~ (the mean of the
-// row's first 8 values, identical in every thread) is subtracted first so
-// that large means do not cost precision, then Y = H (x - mu~).  Because row 0
+// row's first 8 values, identical in every thread) is subtracted first when it
+// exceeds their spread, so that large means do not cost precision; then
+// Y = H (x - mu~) (mu~ = 0 otherwise).  Because row 0
 // of H is all ones, Y_0 = K (mu - mu~) and sum_{i>=1} Y_i^2 = K^2 var, so
 //   t_i = Y_i / sqrt(K (var + eps_ln))  for i >= 1,   t_0 = 0,
 // which is exactly H LN(x) / sqrt(K) with the biased variance and no affine.
@@ -48,11 +50,15 @@ struct Shape {
   static constexpr int T = K / E;                       // threads per row
   static constexpr int R = T >= 128 ? 1 : 128 / T;      // rows per CTA
   static constexpr int THREADS = T * R;
-  static constexpr int MINB = THREADS >= 512 ? 1 : (THREADS >= 256 ? 2 : 4);  // -> <= 128 registers
+  // CTAs per SM the register budget is tuned for: 512 threads -> 128 regs,
+  // 256 -> 80 regs (3 CTAs), 128 -> 96 regs (5 CTAs)
+  static constexpr int MINB = THREADS >= 512 ? 1 : (THREADS >= 256 ? 3 : 5);
   static constexpr int PAD = T < 32 ? 16 : 0;           // floats of padding per row
   static constexpr int STRIDE = K + PAD;                // floats per row in smem
   static constexpr int WPR = T > 32 ? T / 32 : 1;       // warps per row
-  static constexpr size_t SMEM = (size_t)R * STRIDE * 4 + (size_t)R * WPR * 8;
+  static constexpr size_t XCH = (size_t)R * STRIDE * 4;   // exchange buffer (floats)
+  static constexpr size_t RED = (size_t)R * WPR * 8;       // one row-reduction scratch
+  static constexpr size_t SMEM = XCH + 2 * RED;            // two reductions, separate slots
   static constexpr int NPB = LOGK >= 10 ? LOGK - 9 : 0;  // pass-2 processed bits {6 .. 5+NPB}
   static constexpr int PB = 6 - NPB;                      // pass-2 vector bits {0 .. PB-1}
 };
@@ -112,11 +118,11 @@ __device__ __forceinline__ void sq_acc2(float& s0, float& s1, float a0, float a1
       : "+f"(s0), "+f"(s1) : "f"(a0), "f"(a1));
 }
 
-// bits of fl(fl(t * r) + 1.5*2^23) for a pair (see q::rint_code)
+// bits of fl(t * r + 1.5*2^23) for a pair, one rounding each (see q::rint_code)
 __device__ __forceinline__ void magic2(float t0, float t1, float r, uint32_t& m0, uint32_t& m1) {
   asm("{\n\t.reg .b64 A, R, M;\n\t"
       "mov.b64 A, {%2, %3};\n\tmov.b64 R, {%4, %4};\n\tmov.b64 M, {%5, %5};\n\t"
-      "mul.rn.f32x2 A, A, R;\n\tadd.rn.f32x2 A, A, M;\n\t"
+      "fma.rn.f32x2 A, A, R, M;\n\t"
       "mov.b64 {%0, %1}, A;\n\t}"
       : "=r"(m0), "=r"(m1) : "f"(t0), "f"(t1), "f"(r), "f"(q::kMagic));
 }
@@ -150,7 +156,8 @@ __device__ __forceinline__ void stage_range(float (&e)[N], int lo, int hi) {
 }
 
 // Row-wide all-reduce over the T threads of a row (deterministic order: every
-// thread of the row ends with the identical value).
+// thread of the row ends with the identical value).  `red` must not be reused
+// by the CTA afterwards (each reduction has its own slot).
 template <int T, int WPR>
 struct RowReduce {
   template <typename V, typename Op>
@@ -164,7 +171,6 @@ struct RowReduce {
       v = red[rl * WPR];
 #pragma unroll
       for (int w = 1; w < WPR; ++w) v = op(v, red[rl * WPR + w]);
-      __syncthreads();
     }
     return v;
   }
@@ -275,6 +281,7 @@ __device__ __forceinline__ void store_pass1(const float (&e)[64], float* smem, c
   }
 }
 
+// One CTA handles one group of R rows.
 template <int LOGK, bool BF16, int MODE>
 __global__ void __launch_bounds__(Shape<LOGK>::THREADS, Shape<LOGK>::MINB)
 ln_fht_quant_kernel(const void* __restrict__ x, int64_t M, float sK, void* __restrict__ out,
@@ -283,7 +290,8 @@ ln_fht_quant_kernel(const void* __restrict__ x, int64_t M, float sK, void* __res
   constexpr int K = S::K, T = S::T, R = S::R;
   extern __shared__ __align__(16) unsigned char smem_raw[];
   float* smem = reinterpret_cast<float*>(smem_raw);
-  void* red = smem_raw + (size_t)R * S::STRIDE * 4;
+  void* red1 = smem_raw + S::XCH;
+  void* red2 = smem_raw + S::XCH + S::RED;
 
   const int tid = threadIdx.x;
   const int rl = tid / T;
@@ -296,20 +304,31 @@ ln_fht_quant_kernel(const void* __restrict__ x, int64_t M, float sK, void* __res
 
   float e[64];
 
-  // ---- pass 1: load, remove the row offset, stages of bits {0,1,2,k-3,k-2,k-1}
-  float mu = 0.0f;
+  // ---- pass 1: load, remove a large row offset, stages of bits {0,1,2,k-3,k-2,k-1}
+  float f8[8] = {0, 0, 0, 0, 0, 0, 0, 0};
   if (active) {
-    float f[8];
-    load8<BF16>(xrow, 0, f);
-    mu = (((f[0] + f[1]) + (f[2] + f[3])) + ((f[4] + f[5]) + (f[6] + f[7]))) * 0.125f;
+    load8<BF16>(xrow, 0, f8);
 #pragma unroll
     for (int jj = 0; jj < 8; ++jj) load8<BF16>(xrow, (jj * T + t) * 8, &e[jj * 8]);
   } else {
 #pragma unroll
     for (int r = 0; r < 64; ++r) e[r] = 0.0f;
   }
+  {
+    // mu~ = mean of the row's first 8 values; subtracted only when it exceeds
+    // their spread, i.e. when the row mean could cost float precision
+    const float mu = (((f8[0] + f8[1]) + (f8[2] + f8[3])) + ((f8[4] + f8[5]) + (f8[6] + f8[7]))) * 0.125f;
+    float lo = f8[0], hi = f8[0];
 #pragma unroll
-  for (int r = 0; r < 64; r += 2) sub2(e[r], e[r + 1], mu);
+    for (int u = 1; u < 8; ++u) {
+      lo = fminf(lo, f8[u]);
+      hi = fmaxf(hi, f8[u]);
+    }
+    if (fabsf(mu) > hi - lo) {
+#pragma unroll
+      for (int r = 0; r < 64; r += 2) sub2(e[r], e[r + 1], mu);
+    }
+  }
   stage_range(e, 0, 6);
   {
     SwzBase sb(row_off, t * 8);
@@ -344,7 +363,7 @@ ln_fht_quant_kernel(const void* __restrict__ x, int64_t M, float sK, void* __res
 #pragma unroll
   for (int r = 0; r < 64; r += 2) sq_acc2(s0, s1, e[r], e[r + 1]);
   if (t == 0) e[0] = e0;
-  float ss = RowReduce<T, S::WPR>::run(s0 + s1, AddF(), reinterpret_cast<float*>(red), rl, t);
+  const float ss = RowReduce<T, S::WPR>::run(s0 + s1, AddF(), reinterpret_cast<float*>(red1), rl, t);
   const float var = ss * (1.0f / ((float)K * (float)K));
   const float cmul = __fmul_rn(__fdiv_rn(1.0f, sqrtf(__fadd_rn(var, 1e-5f))), sK);
 #pragma unroll
@@ -357,15 +376,14 @@ ln_fht_quant_kernel(const void* __restrict__ x, int64_t M, float sK, void* __res
 #pragma unroll
       for (int j = 0; j < 16; ++j) dst[j] = make_float4(e[4 * j], e[4 * j + 1], e[4 * j + 2], e[4 * j + 3]);
     }
-    return;
   } else {
     q::RowParams p;
     if constexpr (MODE == K1_Q8_I8) {
-      float g = 0.0f;
+      float gm = 0.0f;
 #pragma unroll
-      for (int r = 0; r < 64; ++r) g = fmaxf(g, fabsf(e[r]));
-      g = RowReduce<T, S::WPR>::run(g, MaxF(), reinterpret_cast<float*>(red), rl, t);
-      p = q::params_int8(g);
+      for (int r = 0; r < 64; ++r) gm = fmaxf(gm, fabsf(e[r]));
+      gm = RowReduce<T, S::WPR>::run(gm, MaxF(), reinterpret_cast<float*>(red2), rl, t);
+      p = q::params_int8(gm);
     } else {
       double a0 = 0.0, a1 = 0.0;
 #pragma unroll
@@ -373,37 +391,39 @@ ln_fht_quant_kernel(const void* __restrict__ x, int64_t M, float sK, void* __res
         a0 += q::abs_f64(e[r]);
         a1 += q::abs_f64(e[r + 1]);
       }
-      double a = RowReduce<T, S::WPR>::run(a0 + a1, AddD(), reinterpret_cast<double*>(red), rl, t);
+      const double a = RowReduce<T, S::WPR>::run(a0 + a1, AddD(), reinterpret_cast<double*>(red2), rl, t);
       p = q::params_int4(a, K);
     }
-    if (!active) return;
-    if (t == 0) scales[row] = p.scale;
-    uint32_t m[64];
+    if (active) {
+      if (t == 0) scales[row] = p.scale;
+      uint32_t m[64];
 #pragma unroll
-    for (int r = 0; r < 64; r += 2) magic2(e[r], e[r + 1], p.r, m[r], m[r + 1]);
-    if constexpr (MODE == K1_Q4_PACKED) {
-      uint32_t w[8];
+      for (int r = 0; r < 64; r += 2) magic2(e[r], e[r + 1], p.r, m[r], m[r + 1]);
+      if constexpr (MODE == K1_Q4_PACKED) {
+        uint32_t w[8];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        int n[8];
+        for (int j = 0; j < 8; ++j) {
+          int n[8];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) n[u] = (int)m[8 * j + u] - q::kMagicBits;
-        w[j] = q::pack_s4x8(n);
+          for (int u = 0; u < 8; ++u) n[u] = (int)m[8 * j + u] - q::kMagicBits;
+          w[j] = q::pack_s4x8(n);
+        }
+        uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(out) + (size_t)row * (K / 2) + base / 2);
+        dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+        dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+      } else {
+        if constexpr (MODE == K1_Q4_I8) {
+#pragma unroll
+          for (int r = 0; r < 64; ++r) m[r] = q::clip_magic_int4(m[r]);
+        }
+        uint32_t w[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+          w[j] = q::gather_low_bytes(m[4 * j], m[4 * j + 1], m[4 * j + 2], m[4 * j + 3]);
+        uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(out) + (size_t)row * K + base);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) dst[j] = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
       }
-      uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(out) + (size_t)row * (K / 2) + base / 2);
-      dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
-      dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
-    } else {
-      if constexpr (MODE == K1_Q4_I8) {
-#pragma unroll
-        for (int r = 0; r < 64; ++r) m[r] = q::clip_magic_int4(m[r]);
-      }
-      uint32_t w[16];
-#pragma unroll
-      for (int j = 0; j < 16; ++j) w[j] = q::gather_low_bytes(m[4 * j], m[4 * j + 1], m[4 * j + 2], m[4 * j + 3]);
-      uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(out) + (size_t)row * K + base);
-#pragma unroll
-      for (int j = 0; j < 4; ++j) dst[j] = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
     }
   }
 }
@@ -412,8 +432,8 @@ template <int LOGK, bool BF16, int MODE>
 cudaError_t launch_one(const void* x, int64_t M, void* out, float* scales, cudaStream_t stream) {
   using S = Shape<LOGK>;
   auto kern = ln_fht_quant_kernel<LOGK, BF16, MODE>;
-  cudaError_t attr = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)S::SMEM);
-  if (attr != cudaSuccess) return attr;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)S::SMEM);
+  if (e != cudaSuccess) return e;
   const int64_t grid = (M + S::R - 1) / S::R;
   const float sK = (float)(1.0 / sqrt((double)S::K));
   kern<<<(unsigned)grid, S::THREADS, S::SMEM, stream>>>(x, M, sK, out, scales);

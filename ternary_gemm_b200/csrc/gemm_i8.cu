@@ -12,7 +12,10 @@
 // they reach this kernel (sm_100 has no int4 or ternary integer MMA); int8
 // products accumulate exactly in int32 (|acc| <= 127 * 32768 < 2^31).
 //
-// Design (one CTA per SM, persistent over 128 x 256 output tiles):
+// Two variants share the helpers below: the 2-SM kernel (M >= 256, described
+// above gemm_i8_2sm_kernel) and this 1-SM kernel for short M.
+//
+// 1-SM design (one CTA per SM, persistent over 128 x 256 output tiles):
 //   warp 0      TMA producer: 128-byte-swizzled boxes of A (128 x 128 B) and
 //               B (256 x 128 B) into a kStages-deep shared-memory ring;
 //   warp 1      allocates 512 TMEM columns (two 128 x 256 int32
@@ -351,6 +354,274 @@ gemm_i8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   }
 }
 
+// ---------------------------------------------------------------- 2-SM variant
+// A cluster of two CTAs (one per SM of a TPC) computes a 256 x 256 tile with
+// tcgen05.mma.cta_group::2 (M = 256): each CTA holds 128 rows of A and 128 of
+// the 256 B rows in its own shared memory, so each SM streams half the B
+// bytes of the 1-SM kernel per MMA, and a 6-stage ring of 32 KB stages fits.
+// Both CTAs' TMA loads complete on the leader CTA's full barrier (the leader
+// alone expects the 64 KB of a stage); only the leader issues MMAs; its
+// commits arrive on the same-offset barriers of both CTAs (commit multicast,
+// no multicast loads).  Each CTA's epilogue reads its own TMEM (its 128 rows)
+// and arrives on the leader's accumulator-empty barrier.
+constexpr int k2Stages = 6;
+constexpr int k2ABytes = 128 * kBK;  // 16 KB: this CTA's 128 rows of A
+constexpr int k2BBytes = 128 * kBK;  // 16 KB: this CTA's 128 of the 256 B rows
+constexpr int k2StageBytes = k2ABytes + k2BBytes;
+constexpr size_t k2SmemBytes = 1024 + (size_t)k2Stages * k2StageBytes + 256;
+// kind::i8, D s32, A/B s8 K-major, M = 256, N = 256
+constexpr uint32_t kIdesc2 = (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(256 >> 3) << 17) |
+                             ((uint32_t)(256 >> 4) << 24);
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+// Address of the same shared variable in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
+__device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* map, int x, int y, uint32_t leader_bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
+      "[%4];" ::"r"(smem_u32(dst)),
+      "l"((uint64_t)map), "r"(x), "r"(y), "r"(leader_bar)
+      : "memory");
+}
+
+__device__ __forceinline__ void mma_i8_pair(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::i8 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(kIdesc2), "r"(accumulate));
+}
+
+// arrive on the barrier at this offset in both CTAs of the pair once the
+// leader's outstanding MMAs complete
+__device__ __forceinline__ void mma_commit_pair(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+          smem_u32(bar)),
+      "h"((uint16_t)0x3)
+      : "memory");
+}
+
+__device__ __forceinline__ void mma_commit_local2(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void epilogue_tile(const Params& p, uint32_t tbase, int row, int n0) {
+  const bool row_ok = row < p.M;
+  float sa = 0.0f;
+  if (p.y_mode != 0 && row_ok) sa = __fmul_rn(__ldg(p.scales + row), __ldg(p.alpha));
+#pragma unroll 1
+  for (int c = 0; c < 256; c += 32) {
+    uint32_t r[32];
+    tmem_ld32(tbase + (uint32_t)c, r);
+    const int col0 = n0 + c;
+    if (!row_ok) continue;
+    if (p.y_mode == 0) {
+      int32_t* yrow = reinterpret_cast<int32_t*>(p.y) + (size_t)row * p.N;
+#pragma unroll
+      for (int j = 0; j < 32; j += 4)
+        if (col0 + j < p.N) *reinterpret_cast<uint4*>(yrow + col0 + j) = make_uint4(r[j], r[j + 1], r[j + 2], r[j + 3]);
+    } else if (p.y_mode == 1) {
+      float* yrow = reinterpret_cast<float*>(p.y) + (size_t)row * p.N;
+#pragma unroll
+      for (int j = 0; j < 32; j += 4) {
+        if (col0 + j < p.N) {
+          float4 v;
+          v.x = __fmul_rn(__int2float_rn((int)r[j]), sa);
+          v.y = __fmul_rn(__int2float_rn((int)r[j + 1]), sa);
+          v.z = __fmul_rn(__int2float_rn((int)r[j + 2]), sa);
+          v.w = __fmul_rn(__int2float_rn((int)r[j + 3]), sa);
+          *reinterpret_cast<float4*>(yrow + col0 + j) = v;
+        }
+      }
+    } else {
+      uint16_t* yrow = reinterpret_cast<uint16_t*>(p.y) + (size_t)row * p.N;
+#pragma unroll
+      for (int j = 0; j < 32; j += 8) {
+        if (col0 + j < p.N) {
+          uint4 v;
+          v.x = bf16x2(__fmul_rn(__int2float_rn((int)r[j]), sa), __fmul_rn(__int2float_rn((int)r[j + 1]), sa));
+          v.y = bf16x2(__fmul_rn(__int2float_rn((int)r[j + 2]), sa), __fmul_rn(__int2float_rn((int)r[j + 3]), sa));
+          v.z = bf16x2(__fmul_rn(__int2float_rn((int)r[j + 4]), sa), __fmul_rn(__int2float_rn((int)r[j + 5]), sa));
+          v.w = bf16x2(__fmul_rn(__int2float_rn((int)r[j + 6]), sa), __fmul_rn(__int2float_rn((int)r[j + 7]), sa));
+          *reinterpret_cast<uint4*>(yrow + col0 + j) = v;
+        }
+      }
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+gemm_i8_2sm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  uint8_t* sA = base;
+  uint8_t* sB = base + k2Stages * k2ABytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(base + k2Stages * k2StageBytes);
+  uint64_t* empty = full + k2Stages;
+  uint64_t* tfull = empty + k2Stages;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint64_t* exitb = drain + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(exitb + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int cid = blockIdx.x >> 1;
+  const int ncl = gridDim.x >> 1;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < k2Stages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 8);
+    }
+    mbar_init(drain, 1);
+    mbar_init(exitb, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+  }
+  fence_before();
+  cluster_sync_all();
+  fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&tmA) : "memory");
+      asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&tmB) : "memory");
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int tile = cid; tile < p.num_tiles && ok; tile += ncl) {
+        const int m_blk = tile / p.num_n, n_blk = tile % p.num_n;
+        for (int kb = 0; kb < p.num_kb; ++kb) {
+          if (!wait_bounded(&empty[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
+          const uint32_t fbar = mapa_shared(smem_u32(&full[stage]), 0);
+          if (leader) mbar_expect_tx(&full[stage], (uint32_t)(2 * k2StageBytes));
+          tma_load_2d_pair(sA + stage * k2ABytes, &tmA, kb * kBK, m_blk * 256 + (int)rank * 128, fbar);
+          tma_load_2d_pair(sB + stage * k2BBytes, &tmB, kb * kBK, n_blk * 256 + (int)rank * 128, fbar);
+          if (++stage == k2Stages) { stage = 0; phase ^= 1u; }
+        }
+      }
+      if (!ok) {
+        const uint64_t t0 = globaltimer();
+        while (globaltimer() - t0 < 20000000ull) {
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && leader) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int tile = cid; tile < p.num_tiles && ok; tile += ncl) {
+        if (!wait_bounded(&tempty[acc], acc_phase ^ 1u, abort_flag)) { ok = false; break; }
+        fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * 256);
+        for (int kb = 0; kb < p.num_kb; ++kb) {
+          if (!wait_bounded(&full[stage], phase, abort_flag)) { ok = false; break; }
+          fence_after();
+          const uint64_t a0 = sdesc(smem_u32(sA + stage * k2ABytes));
+          const uint64_t b0 = sdesc(smem_u32(sB + stage * k2BBytes));
+#pragma unroll
+          for (int k = 0; k < kBK / 32; ++k)
+            mma_i8_pair(d_tmem, a0 + (uint64_t)(2 * k), b0 + (uint64_t)(2 * k), (kb | k) != 0 ? 1u : 0u);
+          mma_commit_pair(&empty[stage]);
+          if (++stage == k2Stages) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        mma_commit_pair(&tfull[acc]);
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
+      }
+      mma_commit_local2(drain);
+      const uint64_t t0 = globaltimer();
+      while (!mbar_try_wait(drain, 0) && globaltimer() - t0 < 200000000ull) {
+      }
+    }
+  } else {
+    const int quarter = warp & 3;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int tile = cid; tile < p.num_tiles; tile += ncl) {
+      int ok = 1;
+      if (lane == 0) ok = wait_bounded(&tfull[acc], acc_phase, abort_flag) ? 1 : 0;
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      fence_after();
+      const int m_blk = tile / p.num_n, n_blk = tile % p.num_n;
+      const int row = m_blk * 256 + (int)rank * 128 + quarter * 32 + lane;
+      epilogue_tile(p, tmem_base + (uint32_t)(acc * 256) + ((uint32_t)(quarter * 32) << 16), row, n_blk * 256);
+      fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        if (leader)
+          mbar_arrive(&tempty[acc]);
+        else
+          mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[acc]), 0));
+      }
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1u;
+    }
+  }
+
+  // neither CTA may free its shared memory or TMEM while the pair still uses
+  // them: a bounded handshake through each other's exit barrier
+  fence_before();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    mbar_arrive_cluster(mapa_shared(smem_u32(exitb), rank ^ 1u));
+    const uint64_t t0 = globaltimer();
+    while (!mbar_try_wait(exitb, 0)) {
+      if (globaltimer() - t0 > kWaitLimitNs) {
+        atomicExch(&g_device_error, 1);
+        break;
+      }
+    }
+  }
+  __syncthreads();
+  fence_after();
+  if (warp == 1) {
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kTmemCols)
+                 : "memory");
+  }
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = []() -> PFN_cuTensorMapEncodeTiled_v12000 {
     void* ptr = nullptr;
@@ -402,11 +673,51 @@ cudaError_t launch_gemm_i8(const int8_t* A, const int8_t* B, int64_t M, int64_t 
   p.y = y;
   p.scales = scales;
   p.alpha = alpha;
+  if (M >= 256) {
+    // 2-SM tiles of 256 x 256
+    CUtensorMap tb2;
+    if (!make_map(&tb2, B, N, K, 128)) return cudaErrorInvalidValue;
+    p.num_m = (int)((M + 255) / 256);
+    p.num_n = (int)((N + 255) / 256);
+    p.num_tiles = p.num_m * p.num_n;
+    cudaError_t e = cudaFuncSetAttribute(gemm_i8_2sm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)k2SmemBytes);
+    if (e != cudaSuccess) return e;
+    const int pairs = sm_count() / 2;
+    const int nclusters = p.num_tiles < pairs ? p.num_tiles : pairs;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(2 * nclusters), 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = k2SmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, gemm_i8_2sm_kernel, ta, tb2, p);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+  }
   cudaError_t e = cudaFuncSetAttribute(gemm_i8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
   if (e != cudaSuccess) return e;
   const int grid = p.num_tiles < sm_count() ? p.num_tiles : sm_count();
   gemm_i8_kernel<<<grid, kThreads, kSmemBytes, stream>>>(ta, tb, p);
   return cudaGetLastError();
+}
+
+int* device_error_word() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  static int* cache[64] = {nullptr};
+  if (!cache[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return nullptr;
+    cache[dev] = reinterpret_cast<int*>(p);
+  }
+  return cache[dev];
 }
 
 cudaError_t read_and_clear_device_error(cudaStream_t stream, int* value) {

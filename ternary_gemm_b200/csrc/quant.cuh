@@ -9,9 +9,8 @@
 //          q = clip(rint(127 t / (gamma + eps)), -128, 127), scale = gamma / 127
 // Arithmetic contract (float unless stated): the mean of |t| is accumulated in
 // double and rounded once to float; r = c / (stat + eps) is one IEEE division
-// per row; each code is rint of the float product t * r (round half to even).
-// The __f*_rn intrinsics keep the compiler from fusing these into FMAs, which
-// would round differently.
+// per row; each code is rint of the exact product t * r (round half to even,
+// a single rounding).  The __f*_rn intrinsics pin every rounding.
 #pragma once
 
 #include <cstdint>
@@ -59,15 +58,14 @@ __device__ __forceinline__ RowParams params_int8(float gamma) {
   return p;
 }
 
-// rint(fl(t * r)) for |t * r| < 2^22: adding 1.5 * 2^23 leaves a float whose
-// unit in the last place is 1, so the addition itself rounds to the nearest
+// rint(t * r) of the exact product, for |t * r| < 2^22: t * r + 1.5 * 2^23
+// lies in [2^23, 2^24) where a float's unit in the last place is 1, so the one
+// rounding of the fused multiply-add is the rounding of t * r to the nearest
 // integer, ties to even (1.5 * 2^23 is even), and the integer sits in the low
-// mantissa bits.  Exact for the whole range the callers use: |t r| <= K sqrt(7)
-// for absmean, < 128 for absmax.
+// mantissa bits.  Exact over the whole range the callers use: |t r| <= K sqrt(7)
+// for absmean, < 127.5 for absmax.
 __device__ __forceinline__ int rint_code(float t, float r) {
-  float v = __fmul_rn(t, r);
-  float m = __fadd_rn(v, kMagic);
-  return __float_as_int(m) - kMagicBits;
+  return __float_as_int(__fmaf_rn(t, r, kMagic)) - kMagicBits;
 }
 
 // Eight codes -> eight 4-bit two's-complement fields, n[0] in the lowest
@@ -92,7 +90,7 @@ __device__ __forceinline__ uint32_t pack_s8x4(int n0, int n1, int n2, int n3) {
 
 __device__ __forceinline__ int clip_int4(int n) { return max(-8, min(7, n)); }
 
-// The bits of fl(fl(t r) + 1.5*2^23) are kMagicBits + rint(t r), so clipping
+// The bits of fl(t r + 1.5*2^23) are kMagicBits + rint(t r), so clipping
 // the bits clips the code, and the low byte is the code as an int8.
 __device__ __forceinline__ uint32_t clip_magic_int4(uint32_t m) {
   return (uint32_t)max(kMagicBits - 8, min(kMagicBits + 7, (int)m));

@@ -3,7 +3,7 @@
 // weight-quantization formula: per-tensor absmean to {-1, 0, 1}):
 //   alpha = mean |W|,  w = clip(rint(W / (alpha + eps)), -1, 1).
 // alpha is accumulated in double and rounded once to float; the codes use one
-// float reciprocal 1/(alpha+eps) and one float product per weight.
+// float reciprocal r = 1/(alpha+eps) and rint of the exact product W r.
 //
 // Kernel 1 writes kTernaryPartials double partial sums (fixed grid, fixed
 // per-thread order, fixed tree).  Kernel 2 has every CTA reduce the same
@@ -57,11 +57,12 @@ abs_partials_kernel(const void* __restrict__ W, int64_t nchunks, double* __restr
 }
 
 __device__ __forceinline__ uint32_t ternary_field(float w, float r) {
-  // clip before rounding keeps the product inside the exact range of
-  // rint_code; clip(rint(v), -1, 1) == clip(rint(clip(v, -2, 2)), -1, 1).
-  float v = fminf(fmaxf(__fmul_rn(w, r), -2.0f), 2.0f);
-  int n = __float_as_int(__fadd_rn(v, q::kMagic)) - q::kMagicBits;
-  n = max(-1, min(1, n));
+  // rint of the exact product w * r, clipped to [-1, 1].  Where |w r| >= 2 the
+  // code is the sign; below, the fused multiply-add rounds exactly (see
+  // q::rint_code) and only |w r| < 2^22 reaches it.
+  int n = __float_as_int(__fmaf_rn(w, r, q::kMagic)) - q::kMagicBits;
+  const float p = __fmul_rn(w, r);
+  n = fabsf(p) >= 2.0f ? (p > 0.0f ? 1 : -1) : max(-1, min(1, n));
   return (uint32_t)n & 3u;  // 0 -> 00, 1 -> 01, -1 -> 11
 }
 
