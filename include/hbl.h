@@ -144,6 +144,29 @@ hbl_status hbl_gemm_dequant(const int8_t* A, const int8_t* w, int64_t M, int64_t
                             const float* scales, const float* alpha_dev, void* y, hbl_dtype yt,
                             cudaStream_t stream);
 
+/* ---------------------------------------------------------------- no caller workspace
+ * The paper has no counterpart to this entry point; it exists for callers
+ * that cannot allocate device memory when they run a layer (a fixed memory
+ * budget reserved up front, allocator-free runtimes or plugins handed only a
+ * layer's tensors, hosts where cudaMalloc may block or fail late).
+ *
+ * hbl_forward_noalloc computes exactly what hbl_forward computes, with the
+ * same arguments minus the workspace: it uses a fixed 32 MiB area of device
+ * memory that belongs to the library (a file-scope __device__ array that every
+ * GPU loading the library holds until the process exits).  Shapes whose
+ * hbl_forward_workspace_bytes(M, K, N, bits) exceeds 32 MiB are rejected with
+ * HBL_ERR_WORKSPACE before anything is launched; other argument errors are
+ * those of hbl_forward.  It calls no allocator.
+ *  - The first call on a device (with that device current) looks up the
+ *    area's device address once (cudaGetSymbolAddress, a query); make that
+ *    first call before any stream capture.
+ *  - All calls share the area, which keeps the last call's contents; nothing
+ *    in it needs to start at zero.  Calls whose kernels overlap on the GPU
+ *    (other streams, unordered host threads) race on it: serialise them. */
+hbl_status hbl_forward_noalloc(const void* x, hbl_dtype xt, int64_t M, int64_t K, const uint8_t* packed,
+                               const float* alpha_dev, int64_t N, int bits, void* y, hbl_dtype yt,
+                               cudaStream_t stream);
+
 /* ---------------------------------------------------------------- test hooks */
 
 /* Stages 1-2 alone: t = H LN(x) / sqrt(K) as float [M][K] (device output).

@@ -62,6 +62,8 @@ def lib():
             L.hbl_fht_quant.restype = i32
             L.hbl_forward.argtypes = [p, i32, i64, i64, p, p, i64, i32, p, i32, p, sz, p]
             L.hbl_forward.restype = i32
+            L.hbl_forward_noalloc.argtypes = [p, i32, i64, i64, p, p, i64, i32, p, i32, p]
+            L.hbl_forward_noalloc.restype = i32
             L.hbl_fht_quant_i8.argtypes = [p, i32, i64, i64, i32, p, p, p]
             L.hbl_fht_quant_i8.restype = i32
             L.hbl_widen_ternary.argtypes = [p, i64, i64, p, p]
@@ -185,6 +187,19 @@ def hbl_forward(x, packed, alpha, N: int, bits: int, y=None, y_dtype=None, works
         workspace = torch.empty((hbl_forward_workspace_bytes(M, K, N, bits),), dtype=torch.uint8, device=x.device)
     _check(lib().hbl_forward(_ptr(x), _dtype_code(x), M, K, _ptr(packed), _ptr(alpha), N, bits, _ptr(y),
                              _dtype_code(y), _ptr(workspace), workspace.numel(), _stream(stream)), "hbl_forward")
+    return y
+
+
+def hbl_forward_noalloc(x, packed, alpha, N: int, bits: int, y=None, y_dtype=None, stream=None):
+    """hbl_forward without a workspace, for callers that cannot allocate device memory: the library's
+    fixed 32 MiB area is used instead (shapes needing more are rejected; concurrent calls race on it)."""
+    torch = _torch()
+    _need_cuda(x, packed, alpha)
+    M, K = x.shape
+    if y is None:
+        y = torch.empty((M, N), dtype=y_dtype or x.dtype, device=x.device)
+    _check(lib().hbl_forward_noalloc(_ptr(x), _dtype_code(x), M, K, _ptr(packed), _ptr(alpha), N, bits, _ptr(y),
+                                     _dtype_code(y), _stream(stream)), "hbl_forward_noalloc")
     return y
 
 
