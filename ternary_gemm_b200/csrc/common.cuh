@@ -7,7 +7,7 @@
 
 #include <cuda_runtime.h>
 
-#include "../../include/hbl.h"
+#include "hbl.h"
 
 namespace hbl {
 
