@@ -49,8 +49,13 @@ def _L():
     global _lib
     with _lock:
         if _lib is None:
-            build()
-            lib = ctypes.CDLL(_LIB_PATH)
+            # HBL_ORACLE_LIB points the wrapper at another build of hbl_oracle.c
+            # (the mutation tests load copies with planted mistakes)
+            path = os.environ.get("HBL_ORACLE_LIB")
+            if not path:
+                build()
+                path = _LIB_PATH
+            lib = ctypes.CDLL(path)
             p, i64, i32, f32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_float
             lib.orc_ln_fht.argtypes = [p, i32, i64, i64, p, p]
             lib.orc_ln_fht.restype = i32

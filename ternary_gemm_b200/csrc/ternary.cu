@@ -104,24 +104,35 @@ pack_kernel(const void* __restrict__ W, int64_t nwords, int64_t count, const dou
   }
 }
 
-// 16 codes (one word) -> 16 int8 bytes: field f -> (f & 1) - (f & 2).
+// Eight 2-bit fields (the low 16 bits of w) -> eight nibbles, field i in
+// nibble i: three shift-or-mask steps.
+__device__ __forceinline__ uint32_t spread_fields(uint32_t w) {
+  uint32_t y = w & 0xffffu;
+  y = (y | (y << 8)) & 0x00ff00ffu;
+  y = (y | (y << 4)) & 0x0f0f0f0fu;
+  y = (y | (y << 2)) & 0x33333333u;
+  return y;
+}
+
+// 2-bit code -> int8 byte by a byte-permute lookup: the table's bytes are
+// 00 -> 0x00, 01 -> 0x01, 10 -> 0x00 (unused pattern), 11 -> 0xFF (-1).
+__device__ __forceinline__ uint4 widen16(uint32_t w) {
+  constexpr uint32_t kLut = 0xff000100u;
+  const uint32_t lo = spread_fields(w), hi = spread_fields(w >> 16);
+  return make_uint4(__byte_perm(kLut, 0u, lo & 0xffffu), __byte_perm(kLut, 0u, lo >> 16),
+                    __byte_perm(kLut, 0u, hi & 0xffffu), __byte_perm(kLut, 0u, hi >> 16));
+}
+
+// 64 codes (four words) per thread -> 64 int8 bytes.
 __global__ void __launch_bounds__(kThreads)
-widen_kernel(const uint32_t* __restrict__ packed, int64_t nwords, uint4* __restrict__ out) {
-  for (int64_t wi = (int64_t)blockIdx.x * kThreads + threadIdx.x; wi < nwords; wi += (int64_t)gridDim.x * kThreads) {
-    uint32_t w = __ldg(packed + wi);
-    uint32_t o[4];
-#pragma unroll
-    for (int b = 0; b < 4; ++b) {
-      uint32_t word = 0;
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        uint32_t f = (w >> (2 * (4 * b + j))) & 3u;
-        int v = (int)(f & 1u) - (int)(f & 2u);
-        word |= ((uint32_t)v & 0xffu) << (8 * j);
-      }
-      o[b] = word;
-    }
-    out[wi] = make_uint4(o[0], o[1], o[2], o[3]);
+widen_kernel(const uint4* __restrict__ packed, int64_t nquads, uint4* __restrict__ out) {
+  for (int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x; i < nquads; i += (int64_t)gridDim.x * kThreads) {
+    const uint4 w = __ldg(packed + i);
+    uint4* o = out + 4 * i;
+    o[0] = widen16(w.x);
+    o[1] = widen16(w.y);
+    o[2] = widen16(w.z);
+    o[3] = widen16(w.w);
   }
 }
 
@@ -153,8 +164,8 @@ cudaError_t launch_pack_ternary(const void* W, bool in_bf16, int64_t N, int64_t 
 }
 
 cudaError_t launch_widen_ternary(const uint8_t* packed, int64_t N, int64_t K, int8_t* out, cudaStream_t stream) {
-  const int64_t nwords = N * K / 16;
-  widen_kernel<<<grid_for(nwords), kThreads, 0, stream>>>(reinterpret_cast<const uint32_t*>(packed), nwords,
+  const int64_t nquads = N * K / 64;  // N K is a multiple of 1024 (K >= 64, N % 16 == 0)
+  widen_kernel<<<grid_for(nquads), kThreads, 0, stream>>>(reinterpret_cast<const uint4*>(packed), nquads,
                                                           reinterpret_cast<uint4*>(out));
   return cudaGetLastError();
 }

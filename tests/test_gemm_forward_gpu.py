@@ -51,6 +51,14 @@ def test_pack_ternary_edge_cases(H, orc):
     assert to_host(alpha)[0] == a and np.array_equal(to_host(packed), orc.pack_ternary(w))
 
 
+@pytest.mark.parametrize("N,K", [(16, 64), (272, 2048), (4096, 16384)])
+def test_widen_ternary_bit_exact(H, orc, N, K):
+    w = np.random.default_rng(N + K).integers(-1, 2, (N, K)).astype(np.int8)
+    packed = orc.pack_ternary(w)
+    wi = to_host(H.hbl_widen_ternary(to_device(packed), K))
+    assert np.array_equal(wi, w)
+
+
 # ----------------------------------------------------------------- int8 GEMM
 
 @pytest.mark.parametrize("M,N,K", [(1, 16, 16), (8, 256, 256), (128, 256, 128), (300, 272, 2048),

@@ -1,0 +1,64 @@
+"""The pins catch plausible mistakes: each mutant below is a copy of the oracle
+with one planted slip, compiled on the CPU; the pin suite must fail on every
+one of them (and pass on the unmodified oracle, which test_oracle_pins checks).
+"""
+import concurrent.futures as cf
+import os
+import subprocess
+import sys
+import tempfile
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+SRC = os.path.join(ROOT, "oracle", "hbl_oracle.c")
+
+# (name, text in hbl_oracle.c, replacement)
+MUTANTS = [
+    ("drop 1/sqrt(K)", "double sc = 1.0 / sqrt((double)K);", "double sc = 1.0;"),
+    ("butterfly difference sign", "v[j + h] = a - b;", "v[j + h] = b - a;"),
+    ("skip the last butterfly stage", "for (int64_t h = 1; h < n; h *= 2)", "for (int64_t h = 1; h < n / 2; h *= 2)"),
+    ("unbiased variance", "v /= (double)K;", "v /= (double)(K - 1);"),
+    ("missing LayerNorm eps", "1.0 / sqrt(v + ORC_EPS_LN)", "1.0 / sqrt(v)"),
+    ("LayerNorm without mean subtraction", "u[i] = (x[i] - mu) * inv;", "u[i] = x[i] * inv;"),
+    ("round half away from zero", "static double orc_rint(double v) { return rint(v); }",
+     "static double orc_rint(double v) { return round(v); }"),
+    ("INT4 clip to 8", "const double hi = (bits == 4) ? 7.0 : 127.0;", "const double hi = (bits == 4) ? 8.0 : 127.0;"),
+    ("missing quantizer eps", "volatile float den = stat + ORC_EPS_Q;", "volatile float den = stat;"),
+    ("absmean over K-1", "stat = (float)(s / (double)K);", "stat = (float)(s / (double)(K - 1));"),
+    ("scale inverted", "volatile float sc = stat / c;", "volatile float sc = c / stat;"),
+    ("alpha without abs", "for (int64_t i = 0; i < n; ++i) s += fabs(orc_load(W, dtype, i));",
+     "for (int64_t i = 0; i < n; ++i) s += orc_load(W, dtype, i);"),
+    ("ternary clip to 2", "if (q > 1.0) q = 1.0;", "if (q > 2.0) q = 2.0;"),
+    ("transposed GEMM operand", "s += (int64_t)A[m * K + k] * (int64_t)B[n * K + k];",
+     "s += (int64_t)A[m * K + k] * (int64_t)B[k * N + n];"),
+    ("dequant without alpha", "volatile float sa = scales[m] * alpha;", "volatile float sa = scales[m];"),
+    ("nibbles swapped", "out[m * (K / 2) + j] = (uint8_t)(lo | (hi << 4));",
+     "out[m * (K / 2) + j] = (uint8_t)(hi | (lo << 4));"),
+    ("ternary -1 encoded as 10", "unsigned f = (v == 0) ? 0u : (v == 1 ? 1u : 3u);",
+     "unsigned f = (v == 0) ? 0u : (v == 1 ? 1u : 2u);"),
+]
+
+
+def _run_mutant(m):
+    name, old, new = m
+    src = open(SRC).read()
+    assert src.count(old) == 1, name
+    with tempfile.TemporaryDirectory() as d:
+        c = os.path.join(d, "mut.c")
+        so = os.path.join(d, "mut.so")
+        open(c, "w").write(src.replace(old, new))
+        subprocess.run(["gcc", "-O2", "-ffp-contract=off", "-std=c11", "-fPIC", "-shared", "-o", so, c, "-lm"],
+                       check=True)
+        env = dict(os.environ, HBL_ORACLE_LIB=so)
+        p = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
+                            os.path.join(ROOT, "tests", "test_oracle_pins.py")],
+                           env=env, capture_output=True, text=True, timeout=600)
+        return name, p.returncode, p.stdout[-400:]
+
+
+def test_every_planted_mistake_fails_a_pin():
+    with cf.ThreadPoolExecutor(max_workers=min(8, os.cpu_count() or 1)) as ex:
+        results = list(ex.map(_run_mutant, MUTANTS))
+    survivors = [(n, out) for n, rc, out in results if rc == 0]
+    assert not survivors, "mutants not caught by any pin: %s" % [n for n, _ in survivors]
