@@ -52,7 +52,7 @@ def parse_args(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
-    ap.add_argument("--sweep", choices=["k1", "fwd"], default=None,
+    ap.add_argument("--sweep", choices=["k1", "fwd", "k1_noh"], default=None,
                     help="instead of the step line: the LN+FHT+INT4 kernel alone at M=65536 for each K, "
                          "or the whole forward at K=N=4096 for each M (one JSON line per point)")
     a = ap.parse_args(argv)
@@ -594,17 +594,21 @@ def bench_sweep(args):
         b.synchronize()
         return a.elapsed_time(b) / n / 1e3
 
-    if args.sweep == "k1":
+    if args.sweep in ("k1", "k1_noh"):
         M = 65536
         for K in SWEEP_K1_KS:
             distinct = 4096                      # 4096 seeded rows, repeated to M on the device
             x = _to_device(make_x(base.with_shape(distinct, K, 256))).repeat(M // distinct, 1)
             codes = torch.empty((M, K // 2), dtype=torch.uint8, device="cuda")
             sc = torch.empty((M,), dtype=torch.float32, device="cuda")
-            t = timed(lambda: hbl.hbl_fht_quant(x, 4, codes=codes, scales=sc), reps)
+            if args.sweep == "k1":
+                t = timed(lambda: hbl.hbl_fht_quant(x, 4, codes=codes, scales=sc), reps)
+            else:   # the same LayerNorm + INT4 path without the Hadamard transform
+                t = timed(lambda: hbl.hbl_norm_quant(x, 4, hbl.HBL_NORM_LAYER, codes=codes, scales=sc), reps)
             nbytes = M * K * 2 + M * K // 2 + 4 * M
             gbs = nbytes / t / 1e9
-            print(json.dumps({"sweep": "k1_ln_fht_int4", "M": M, "K": K, "ms": t * 1e3, "GB/s": gbs,
+            name = "k1_ln_fht_int4" if args.sweep == "k1" else "ln_int4_no_transform"
+            print(json.dumps({"sweep": name, "M": M, "K": K, "ms": t * 1e3, "GB/s": gbs,
                               "frac_hbm": gbs / peaks["hbm_gbs"], "peak_kind": peak_kind,
                               "bytes_per_launch": nbytes, "input": "4096 seeded rows repeated to 65536"}),
                   flush=True)

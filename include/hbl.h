@@ -121,6 +121,51 @@ hbl_status hbl_forward(const void* x, hbl_dtype xt, int64_t M, int64_t K, const 
                        const float* alpha_dev, int64_t N, int bits, void* y, hbl_dtype yt,
                        void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
+/* ---------------------------------------------------------------- the transform alone; rotated weights
+ * The Hadamard ablation of the pages compares rotating only the activations
+ * (H-BitLinear) with rotating weights and activations.  Rotating each weight
+ * row by the same orthogonal H/sqrt(K) leaves the product unchanged before
+ * quantization, (H x).(H w) = x.w, so the rotated weight runs through
+ * hbl_forward unchanged. */
+
+/* t = H_K x / sqrt(K) per row (Sylvester order), float out [M][K] (device);
+ * K a power of two in [64, 32768]. */
+hbl_status hbl_fht(const void* x, hbl_dtype xt, int64_t M, int64_t K, float* t, cudaStream_t stream);
+
+/* Workspace bytes of hbl_pack_ternary_rotated: the float rotated weight
+ * [N][K] plus the partial sums of hbl_pack_ternary. */
+size_t hbl_pack_ternary_rotated_workspace_bytes(int64_t K, int64_t N);
+
+/* Ternary quantization of the rotated weight W' = W H_K / sqrt(K) (each row
+ * of W [N][K] transformed along K in float), then exactly hbl_pack_ternary on
+ * W': alpha = mean|W'|, w = clip(rint(W' / (alpha + eps)), -1, 1), packed.
+ * Same arguments and layouts as hbl_pack_ternary; workspace device, >=
+ * hbl_pack_ternary_rotated_workspace_bytes(K, N) bytes, 256-byte aligned. */
+hbl_status hbl_pack_ternary_rotated(const void* W, hbl_dtype wt, int64_t K, int64_t N, uint8_t* packed,
+                                    float* alpha_dev, void* workspace, size_t workspace_bytes,
+                                    cudaStream_t stream);
+
+/* ---------------------------------------------------------------- BitLinear without the transform
+ * The activation path of the BitLinear layers that have no Hadamard
+ * transform ("all linear layers except the input/output embeddings" are
+ * fine-tuned to 4-bit activations, H-BitLinear only replaces Wo and Wdown;
+ * BitNet b1.58 keeps 8-bit absmax activations): normalisation, then the same
+ * per-token quantizer as hbl_fht_quant. */
+typedef enum { HBL_NORM_LAYER = 0, HBL_NORM_RMS = 1 } hbl_norm;
+
+/* t = LN(x) (HBL_NORM_LAYER: mean subtraction, biased variance) or
+ * RMSNorm(x) (HBL_NORM_RMS: x / sqrt(mean x^2 + eps)), eps 1e-5, no affine;
+ * then INT4 absmean (bits 4, codes packed two per byte) or INT8 absmax
+ * (bits 8) exactly as hbl_fht_quant.  K a power of two in [256, 32768];
+ * codes and scales as in hbl_fht_quant. */
+hbl_status hbl_norm_quant(const void* x, hbl_dtype xt, int64_t M, int64_t K, hbl_norm norm, int bits,
+                          uint8_t* codes, float* scales, cudaStream_t stream);
+
+/* The normalisation alone: t as float [M][K] (device), the same kernel code as
+ * hbl_norm_quant up to its quantizer (test hook). */
+hbl_status hbl_debug_norm(const void* x, hbl_dtype xt, int64_t M, int64_t K, hbl_norm norm, float* t,
+                          cudaStream_t stream);
+
 /* ---------------------------------------------------------------- forward stages
  * hbl_forward is exactly these three calls on slices of its workspace; they
  * are public so that callers can keep the widened weight resident, overlap

@@ -67,6 +67,12 @@ def _L():
             lib.orc_hadamard_entry.restype = i32
             lib.orc_layernorm_row.argtypes = [p, i64, p]
             lib.orc_layernorm_row.restype = None
+            lib.orc_fht_rows.argtypes = [p, i32, i64, i64, p, p]
+            lib.orc_fht_rows.restype = i32
+            lib.orc_rmsnorm_row.argtypes = [p, i64, p]
+            lib.orc_rmsnorm_row.restype = None
+            lib.orc_norm_rows.argtypes = [p, i32, i64, i64, i32, p, p]
+            lib.orc_norm_rows.restype = i32
             lib.orc_quant.argtypes = [p, i64, i64, i32, p, p]
             lib.orc_quant.restype = i32
             lib.orc_ternary.argtypes = [p, i32, i64, i64, p, p]
@@ -144,6 +150,46 @@ def ln_fht(x: np.ndarray):
     rc = _L().orc_ln_fht(_ptr(x), dt, M, K, _ptr(t64), _ptr(t32))
     if rc != 0:
         raise ValueError("orc_ln_fht failed (%d): K must be a power of two" % rc)
+    return t64, t32
+
+
+def fht_rows(x: np.ndarray):
+    """t = H_K x / sqrt(K) per row, no normalisation.  Returns (t64 double, t32 float)."""
+    x, dt = _as_input(x)
+    M, K = x.shape
+    t64 = np.empty((M, K), np.float64)
+    t32 = np.empty((M, K), np.float32)
+    if _L().orc_fht_rows(_ptr(x), dt, M, K, _ptr(t64), _ptr(t32)) != 0:
+        raise ValueError("orc_fht_rows failed: K must be a power of two")
+    return t64, t32
+
+
+def ternary_rotated(W: np.ndarray):
+    """Ternarisation of the rotated weight W H/sqrt(K) (rows rotated in double, rounded to float)."""
+    _, w32 = fht_rows(W)
+    return ternary(w32)
+
+
+def rmsnorm_row(x: np.ndarray) -> np.ndarray:
+    """RMSNorm of one row in double, no affine, eps 1e-5."""
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    u = np.empty_like(x)
+    _L().orc_rmsnorm_row(_ptr(x), x.size, _ptr(u))
+    return u
+
+
+LAYER_NORM, RMS_NORM = 0, 1
+
+
+def norm_rows(x: np.ndarray, norm: int = LAYER_NORM):
+    """t = LN(x) or RMSNorm(x) per row: the activation path of a BitLinear layer
+    without the Hadamard transform.  Returns (t64 double, t32 float)."""
+    x, dt = _as_input(x)
+    M, K = x.shape
+    t64 = np.empty((M, K), np.float64)
+    t32 = np.empty((M, K), np.float32)
+    if _L().orc_norm_rows(_ptr(x), dt, M, K, int(norm), _ptr(t64), _ptr(t32)) != 0:
+        raise ValueError("orc_norm_rows failed")
     return t64, t32
 
 

@@ -153,6 +153,58 @@ int orc_ln_fht(const void* x, int dtype, int64_t M, int64_t K, double* t64, floa
   return 0;
 }
 
+/* RMSNorm of one row in double: u = x / sqrt(mean x^2 + eps_ln), no affine.
+ * (The model around H-BitLinear uses RMSNorm; the BitLinear layers without
+ * the Hadamard transform are normalised this way or with LayerNorm.) */
+void orc_rmsnorm_row(const double* x, int64_t K, double* u) {
+  double s = 0.0;
+  for (int64_t i = 0; i < K; ++i) s += x[i] * x[i];
+  double inv = 1.0 / sqrt(s / (double)K + ORC_EPS_LN);
+  for (int64_t i = 0; i < K; ++i) u[i] = x[i] * inv;
+}
+
+/* The activation path of a BitLinear layer without the Hadamard transform:
+ * t = LN(x) (norm = 0) or RMSNorm(x) (norm = 1) per row, any K >= 1.
+ * Outputs the double result and its rounding to float (either may be NULL). */
+int orc_norm_rows(const void* x, int dtype, int64_t M, int64_t K, int norm, double* t64, float* t32) {
+  if (K < 1 || (norm != 0 && norm != 1)) return -1;
+  double* row = (double*)malloc(sizeof(double) * (size_t)K);
+  double* u = (double*)malloc(sizeof(double) * (size_t)K);
+  if (!row || !u) { free(row); free(u); return -2; }
+  for (int64_t m = 0; m < M; ++m) {
+    for (int64_t i = 0; i < K; ++i) row[i] = orc_load(x, dtype, m * K + i);
+    if (norm == 0) orc_layernorm_row(row, K, u);
+    else orc_rmsnorm_row(row, K, u);
+    for (int64_t i = 0; i < K; ++i) {
+      if (t64) t64[m * K + i] = u[i];
+      if (t32) t32[m * K + i] = (float)u[i];
+    }
+  }
+  free(row);
+  free(u);
+  return 0;
+}
+
+/* t = H_K x / sqrt(K) per row in double (no normalisation): the rotation the
+ * Hadamard ablation also applies to the weights.  K a power of two. */
+int orc_fht_rows(const void* x, int dtype, int64_t M, int64_t K, double* t64, float* t32) {
+  if (K < 1 || (K & (K - 1))) return -1;
+  double* row = (double*)malloc(sizeof(double) * (size_t)K);
+  if (!row) return -2;
+  double inv_sqrt_k = 1.0 / sqrt((double)K);
+  for (int64_t m = 0; m < M; ++m) {
+    for (int64_t i = 0; i < K; ++i) row[i] = orc_load(x, dtype, m * K + i);
+    orc_fht_unnormalized(row, K);
+    for (int64_t i = 0; i < K; ++i) {
+      double t = row[i] * inv_sqrt_k;
+      if (t64) t64[m * K + i] = t;
+      if (t32) t32[m * K + i] = (float)t;
+    }
+  }
+  free(row);
+  return 0;
+}
+
 /* --------------------------------------------------- activation quantizers */
 
 /* Per-token activation quantization of M rows of length K (any K >= 1).

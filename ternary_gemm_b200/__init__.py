@@ -20,6 +20,7 @@ HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "hbl.h")
 
 HBL_OK, HBL_ERR_INVALID_ARG, HBL_ERR_UNSUPPORTED, HBL_ERR_WORKSPACE, HBL_ERR_CUDA, HBL_ERR_TIMEOUT = range(6)
 HBL_F32, HBL_BF16 = 0, 1
+HBL_NORM_LAYER, HBL_NORM_RMS = 0, 1
 
 _lock = threading.Lock()
 _lib = None
@@ -62,6 +63,16 @@ def lib():
             L.hbl_fht_quant.restype = i32
             L.hbl_forward.argtypes = [p, i32, i64, i64, p, p, i64, i32, p, i32, p, sz, p]
             L.hbl_forward.restype = i32
+            L.hbl_fht.argtypes = [p, i32, i64, i64, p, p]
+            L.hbl_fht.restype = i32
+            L.hbl_pack_ternary_rotated_workspace_bytes.argtypes = [i64, i64]
+            L.hbl_pack_ternary_rotated_workspace_bytes.restype = sz
+            L.hbl_pack_ternary_rotated.argtypes = [p, i32, i64, i64, p, p, p, sz, p]
+            L.hbl_pack_ternary_rotated.restype = i32
+            L.hbl_norm_quant.argtypes = [p, i32, i64, i64, i32, i32, p, p, p]
+            L.hbl_norm_quant.restype = i32
+            L.hbl_debug_norm.argtypes = [p, i32, i64, i64, i32, p, p]
+            L.hbl_debug_norm.restype = i32
             L.hbl_forward_noalloc.argtypes = [p, i32, i64, i64, p, p, i64, i32, p, i32, p]
             L.hbl_forward_noalloc.restype = i32
             L.hbl_fht_quant_i8.argtypes = [p, i32, i64, i64, i32, p, p, p]
@@ -188,6 +199,65 @@ def hbl_forward(x, packed, alpha, N: int, bits: int, y=None, y_dtype=None, works
     _check(lib().hbl_forward(_ptr(x), _dtype_code(x), M, K, _ptr(packed), _ptr(alpha), N, bits, _ptr(y),
                              _dtype_code(y), _ptr(workspace), workspace.numel(), _stream(stream)), "hbl_forward")
     return y
+
+
+def hbl_fht(x, t=None, stream=None):
+    """t = H_K x / sqrt(K) per row (the transform alone), float32 [M][K]."""
+    torch = _torch()
+    _need_cuda(x)
+    M, K = x.shape
+    if t is None:
+        t = torch.empty((M, K), dtype=torch.float32, device=x.device)
+    _check(lib().hbl_fht(_ptr(x), _dtype_code(x), M, K, _ptr(t), _stream(stream)), "hbl_fht")
+    return t
+
+
+def hbl_pack_ternary_rotated_workspace_bytes(K: int, N: int) -> int:
+    return int(lib().hbl_pack_ternary_rotated_workspace_bytes(K, N))
+
+
+def hbl_pack_ternary_rotated(W, packed=None, alpha=None, workspace=None, stream=None):
+    """Ternarise W H_K/sqrt(K) (weights rotated like the activations): (packed, alpha)."""
+    torch = _torch()
+    _need_cuda(W)
+    N, K = W.shape
+    if packed is None:
+        packed = torch.empty((N, K // 4), dtype=torch.uint8, device=W.device)
+    if alpha is None:
+        alpha = torch.empty((1,), dtype=torch.float32, device=W.device)
+    if workspace is None:
+        workspace = torch.empty((hbl_pack_ternary_rotated_workspace_bytes(K, N),), dtype=torch.uint8,
+                                device=W.device)
+    _check(lib().hbl_pack_ternary_rotated(_ptr(W), _dtype_code(W), K, N, _ptr(packed), _ptr(alpha),
+                                          _ptr(workspace), workspace.numel(), _stream(stream)),
+           "hbl_pack_ternary_rotated")
+    return packed, alpha
+
+
+def hbl_norm_quant(x, bits: int, norm: int = HBL_NORM_LAYER, codes=None, scales=None, stream=None):
+    """BitLinear activation path without the transform: LN or RMSNorm, then INT4/INT8 codes."""
+    torch = _torch()
+    _need_cuda(x)
+    M, K = x.shape
+    if codes is None:
+        codes = (torch.empty((M, K // 2), dtype=torch.uint8, device=x.device) if bits == 4
+                 else torch.empty((M, K), dtype=torch.int8, device=x.device))
+    if scales is None:
+        scales = torch.empty((M,), dtype=torch.float32, device=x.device)
+    _check(lib().hbl_norm_quant(_ptr(x), _dtype_code(x), M, K, int(norm), bits, _ptr(codes), _ptr(scales),
+                                _stream(stream)), "hbl_norm_quant")
+    return codes, scales
+
+
+def hbl_debug_norm(x, norm: int = HBL_NORM_LAYER, t=None, stream=None):
+    torch = _torch()
+    _need_cuda(x)
+    M, K = x.shape
+    if t is None:
+        t = torch.empty((M, K), dtype=torch.float32, device=x.device)
+    _check(lib().hbl_debug_norm(_ptr(x), _dtype_code(x), M, K, int(norm), _ptr(t), _stream(stream)),
+           "hbl_debug_norm")
+    return t
 
 
 def hbl_forward_noalloc(x, packed, alpha, N: int, bits: int, y=None, y_dtype=None, stream=None):

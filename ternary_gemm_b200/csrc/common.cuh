@@ -17,6 +17,7 @@ enum K1Mode : int {
   K1_Q4_PACKED = 1,  // INT4 absmean codes, two per byte
   K1_Q4_I8 = 2,      // INT4 absmean codes widened to one int8 per element
   K1_Q8_I8 = 3,      // INT8 absmax codes, one int8 per element
+  K1_FHT_F32 = 4,    // the plain scaled transform H x / sqrt(K) as float (no LN, no quantizer)
 };
 
 constexpr int kMinLogK = 6;   // K = 64
@@ -27,6 +28,11 @@ constexpr int kMaxLogK = 15;  // K = 32768
 // K1_T_F32).  Returns cudaSuccess or the launch error.
 cudaError_t launch_ln_fht_quant(const void* x, bool in_bf16, int64_t M, int log2k, K1Mode mode,
                                 void* out, float* scales, cudaStream_t stream);
+
+// LayerNorm (rms = false) or RMSNorm (rms = true) then the quantizer, without
+// the Hadamard transform; K a power of two in [256, 32768].
+cudaError_t launch_norm_quant(const void* x, bool in_bf16, int64_t M, int64_t K, bool rms, K1Mode mode,
+                              void* out, float* scales, cudaStream_t stream);
 
 // The quantizer alone on float rows t [M][K] (K % 16 == 0).
 cudaError_t launch_quant_from_f32(const float* t, int64_t M, int64_t K, int bits, bool packed,

@@ -39,9 +39,12 @@
 
 #include "common.cuh"
 #include "quant.cuh"
+#include "rowkit.cuh"
 
 namespace hbl {
 namespace {
+
+using namespace rowkit;
 
 template <int LOGK>
 struct Shape {
@@ -61,6 +64,7 @@ struct Shape {
   static constexpr size_t SMEM = XCH + 2 * RED;            // two reductions, separate slots
   static constexpr int NPB = LOGK >= 10 ? LOGK - 9 : 0;  // pass-2 processed bits {6 .. 5+NPB}
   static constexpr int PB = 6 - NPB;                      // pass-2 vector bits {0 .. PB-1}
+  static_assert(NPB >= 0 && NPB <= 6 && PB >= 0 && PB <= 6, "pass-2 split");
 };
 
 // The swizzle: index bits 5..8 XORed into bits 2..4 (linear over GF(2)).
@@ -85,47 +89,6 @@ struct SwzBase {
     return b[(sc >> 2) & 7] + (sc & ~0x1C);
   }
 };
-
-// ---------------------------------------------------------------- paired float ops
-
-__device__ __forceinline__ void bfly2(float& a0, float& a1, float& b0, float& b1) {
-  asm("{\n\t.reg .b64 A, B, S, D;\n\t"
-      "mov.b64 A, {%0, %1};\n\tmov.b64 B, {%2, %3};\n\t"
-      "add.rn.f32x2 S, A, B;\n\tsub.rn.f32x2 D, A, B;\n\t"
-      "mov.b64 {%0, %1}, S;\n\tmov.b64 {%2, %3}, D;\n\t}"
-      : "+f"(a0), "+f"(a1), "+f"(b0), "+f"(b1));
-}
-
-__device__ __forceinline__ void sub2(float& a0, float& a1, float c) {
-  asm("{\n\t.reg .b64 A, C;\n\t"
-      "mov.b64 A, {%0, %1};\n\tmov.b64 C, {%2, %2};\n\t"
-      "sub.rn.f32x2 A, A, C;\n\tmov.b64 {%0, %1}, A;\n\t}"
-      : "+f"(a0), "+f"(a1) : "f"(c));
-}
-
-__device__ __forceinline__ void mul2(float& a0, float& a1, float c) {
-  asm("{\n\t.reg .b64 A, C;\n\t"
-      "mov.b64 A, {%0, %1};\n\tmov.b64 C, {%2, %2};\n\t"
-      "mul.rn.f32x2 A, A, C;\n\tmov.b64 {%0, %1}, A;\n\t}"
-      : "+f"(a0), "+f"(a1) : "f"(c));
-}
-
-// (s0, s1) += (a0*a0, a1*a1)
-__device__ __forceinline__ void sq_acc2(float& s0, float& s1, float a0, float a1) {
-  asm("{\n\t.reg .b64 A, S;\n\t"
-      "mov.b64 A, {%2, %3};\n\tmov.b64 S, {%0, %1};\n\t"
-      "fma.rn.f32x2 S, A, A, S;\n\tmov.b64 {%0, %1}, S;\n\t}"
-      : "+f"(s0), "+f"(s1) : "f"(a0), "f"(a1));
-}
-
-// bits of fl(t * r + 1.5*2^23) for a pair, one rounding each (see q::rint_code)
-__device__ __forceinline__ void magic2(float t0, float t1, float r, uint32_t& m0, uint32_t& m1) {
-  asm("{\n\t.reg .b64 A, R, M;\n\t"
-      "mov.b64 A, {%2, %3};\n\tmov.b64 R, {%4, %4};\n\tmov.b64 M, {%5, %5};\n\t"
-      "fma.rn.f32x2 A, A, R, M;\n\t"
-      "mov.b64 {%0, %1}, A;\n\t}"
-      : "=r"(m0), "=r"(m1) : "f"(t0), "f"(t1), "f"(r), "f"(q::kMagic));
-}
 
 // Butterfly over register-index bit B: (e[r], e[r + 2^B]) -> (sum, difference).
 template <int B, int N>
@@ -153,61 +116,6 @@ __device__ __forceinline__ void stage_range(float (&e)[N], int lo, int hi) {
   if (lo <= 3 && 3 < hi) stage<3>(e);
   if (lo <= 4 && 4 < hi) stage<4>(e);
   if (lo <= 5 && 5 < hi) stage<5>(e);
-}
-
-// Row-wide all-reduce over the T threads of a row (deterministic order: every
-// thread of the row ends with the identical value).  `red` must not be reused
-// by the CTA afterwards (each reduction has its own slot).
-template <int T, int WPR>
-struct RowReduce {
-  template <typename V, typename Op>
-  __device__ __forceinline__ static V run(V v, Op op, V* red, int rl, int t) {
-    constexpr int W = T < 32 ? T : 32;
-#pragma unroll
-    for (int o = W / 2; o >= 1; o >>= 1) v = op(v, __shfl_xor_sync(0xffffffffu, v, o));
-    if constexpr (T > 32) {
-      if ((t & 31) == 0) red[rl * WPR + (t >> 5)] = v;
-      __syncthreads();
-      v = red[rl * WPR];
-#pragma unroll
-      for (int w = 1; w < WPR; ++w) v = op(v, red[rl * WPR + w]);
-    }
-    return v;
-  }
-};
-
-struct AddF {
-  __device__ __forceinline__ float operator()(float a, float b) const { return a + b; }
-};
-struct AddD {
-  __device__ __forceinline__ double operator()(double a, double b) const { return a + b; }
-};
-struct MaxF {
-  __device__ __forceinline__ float operator()(float a, float b) const { return fmaxf(a, b); }
-};
-
-__device__ __forceinline__ void bf16x8_to_f32(const uint4& u, float* o) {
-  o[0] = __uint_as_float(u.x << 16);
-  o[1] = __uint_as_float(u.x & 0xffff0000u);
-  o[2] = __uint_as_float(u.y << 16);
-  o[3] = __uint_as_float(u.y & 0xffff0000u);
-  o[4] = __uint_as_float(u.z << 16);
-  o[5] = __uint_as_float(u.z & 0xffff0000u);
-  o[6] = __uint_as_float(u.w << 16);
-  o[7] = __uint_as_float(u.w & 0xffff0000u);
-}
-
-template <bool BF16>
-__device__ __forceinline__ void load8(const void* xrow, int i, float* o) {
-  if constexpr (BF16) {
-    uint4 u = __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(xrow) + i));
-    bf16x8_to_f32(u, o);
-  } else {
-    const float4* p = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(xrow) + i);
-    float4 a = __ldg(p), b = __ldg(p + 1);
-    o[0] = a.x; o[1] = a.y; o[2] = a.z; o[3] = a.w;
-    o[4] = b.x; o[5] = b.y; o[6] = b.z; o[7] = b.w;
-  }
 }
 
 // Thread bit j of pass 2 -> index bit: {PB .. 5} then {k-3, k-2, k-1}.
@@ -301,6 +209,7 @@ ln_fht_quant_kernel(const void* __restrict__ x, int64_t M, float sK, void* __res
   const size_t esz = BF16 ? 2 : 4;
   const void* xrow = reinterpret_cast<const unsigned char*>(x) + (size_t)(active ? row : 0) * K * esz;
   const int row_off = rl * S::STRIDE;
+  constexpr bool kLN = MODE != K1_FHT_F32;  // the plain transform mode has no LayerNorm
 
   float e[64];
 
@@ -324,7 +233,7 @@ ln_fht_quant_kernel(const void* __restrict__ x, int64_t M, float sK, void* __res
       lo = fminf(lo, f8[u]);
       hi = fmaxf(hi, f8[u]);
     }
-    if (fabsf(mu) > hi - lo) {
+    if (kLN && fabsf(mu) > hi - lo) {
 #pragma unroll
       for (int r = 0; r < 64; r += 2) sub2(e[r], e[r + 1], mu);
     }
@@ -357,20 +266,23 @@ ln_fht_quant_kernel(const void* __restrict__ x, int64_t M, float sK, void* __res
   stage_range(e, 3, LOGK - 3 < 6 ? LOGK - 3 : 6);
 
   // ---- LayerNorm statistics from the transform: K^2 var = sum_{i>=1} Y_i^2
-  float s0 = 0.0f, s1 = 0.0f;
-  const float e0 = e[0];
-  if (t == 0) e[0] = 0.0f;
+  float cmul = sK;
+  if constexpr (kLN) {
+    float s0 = 0.0f, s1 = 0.0f;
+    const float e0 = e[0];
+    if (t == 0) e[0] = 0.0f;
 #pragma unroll
-  for (int r = 0; r < 64; r += 2) sq_acc2(s0, s1, e[r], e[r + 1]);
-  if (t == 0) e[0] = e0;
-  const float ss = RowReduce<T, S::WPR>::run(s0 + s1, AddF(), reinterpret_cast<float*>(red1), rl, t);
-  const float var = ss * (1.0f / ((float)K * (float)K));
-  const float cmul = __fmul_rn(__fdiv_rn(1.0f, sqrtf(__fadd_rn(var, 1e-5f))), sK);
+    for (int r = 0; r < 64; r += 2) sq_acc2(s0, s1, e[r], e[r + 1]);
+    if (t == 0) e[0] = e0;
+    const float ss = RowReduce<T, S::WPR>::run(s0 + s1, AddF(), reinterpret_cast<float*>(red1), rl, t);
+    const float var = ss * (1.0f / ((float)K * (float)K));
+    cmul = __fmul_rn(__fdiv_rn(1.0f, sqrtf(__fadd_rn(var, 1e-5f))), sK);
+  }
 #pragma unroll
   for (int r = 0; r < 64; r += 2) mul2(e[r], e[r + 1], cmul);
-  if (t == 0) e[0] = 0.0f;
+  if (kLN && t == 0) e[0] = 0.0f;
 
-  if constexpr (MODE == K1_T_F32) {
+  if constexpr (MODE == K1_T_F32 || MODE == K1_FHT_F32) {
     if (active) {
       float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(out) + (size_t)row * K + base);
 #pragma unroll
@@ -447,6 +359,7 @@ cudaError_t launch_mode(const void* x, int64_t M, K1Mode mode, void* out, float*
     case K1_Q4_PACKED: return launch_one<LOGK, BF16, K1_Q4_PACKED>(x, M, out, scales, s);
     case K1_Q4_I8: return launch_one<LOGK, BF16, K1_Q4_I8>(x, M, out, scales, s);
     case K1_Q8_I8: return launch_one<LOGK, BF16, K1_Q8_I8>(x, M, out, scales, s);
+    case K1_FHT_F32: return launch_one<LOGK, BF16, K1_FHT_F32>(x, M, out, scales, s);
   }
   return cudaErrorInvalidValue;
 }

@@ -47,6 +47,12 @@ hbl_status check_n(int64_t N) {
   return HBL_OK;
 }
 
+hbl_status check_norm_k(int64_t K) {
+  if (K <= 0) return HBL_ERR_INVALID_ARG;
+  if (K < 256 || K > 32768 || (K & (K - 1))) return HBL_ERR_UNSUPPORTED;
+  return HBL_OK;
+}
+
 struct ForwardLayout {
   size_t a_off, s_off, b_off, total;
 };
@@ -173,6 +179,66 @@ hbl_status hbl_gemm_dequant(const int8_t* A, const int8_t* w, int64_t M, int64_t
   if (s != HBL_OK) return s;
   if ((s = check_n(N)) != HBL_OK) return s;
   return cuda_status(hbl::launch_gemm_i8(A, w, M, N, K, yt == HBL_BF16 ? 2 : 1, y, scales, alpha_dev, stream));
+}
+
+hbl_status hbl_fht(const void* x, hbl_dtype xt, int64_t M, int64_t K, float* t, cudaStream_t stream) {
+  if (!x || !t || !dtype_ok(xt)) return HBL_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(t, 16)) return HBL_ERR_INVALID_ARG;
+  int l;
+  hbl_status s = check_k(K, &l);
+  if (s != HBL_OK) return s;
+  if ((s = check_rows(M)) != HBL_OK) return s;
+  return cuda_status(hbl::launch_ln_fht_quant(x, xt == HBL_BF16, M, l, hbl::K1_FHT_F32, t, nullptr, stream));
+}
+
+size_t hbl_pack_ternary_rotated_workspace_bytes(int64_t K, int64_t N) {
+  const size_t base = hbl_pack_ternary_workspace_bytes(K, N);
+  if (base == 0) return 0;
+  return align256((size_t)N * (size_t)K * 4) + base;
+}
+
+hbl_status hbl_pack_ternary_rotated(const void* W, hbl_dtype wt, int64_t K, int64_t N, uint8_t* packed,
+                                    float* alpha_dev, void* workspace, size_t workspace_bytes,
+                                    cudaStream_t stream) {
+  if (!W || !packed || !alpha_dev || !dtype_ok(wt)) return HBL_ERR_INVALID_ARG;
+  if (!aligned(W, 16) || !aligned(packed, 16) || !aligned(alpha_dev, 4)) return HBL_ERR_INVALID_ARG;
+  int l;
+  hbl_status s = check_k(K, &l);
+  if (s != HBL_OK) return s;
+  if ((s = check_n(N)) != HBL_OK) return s;
+  const size_t need = hbl_pack_ternary_rotated_workspace_bytes(K, N);
+  if (!workspace || !aligned(workspace, 256) || workspace_bytes < need) return HBL_ERR_WORKSPACE;
+  float* rotated = reinterpret_cast<float*>(workspace);
+  double* partials = reinterpret_cast<double*>(reinterpret_cast<uint8_t*>(workspace) +
+                                               align256((size_t)N * (size_t)K * 4));
+  cudaError_t e = hbl::launch_ln_fht_quant(W, wt == HBL_BF16, N, l, hbl::K1_FHT_F32, rotated, nullptr, stream);
+  if (e == cudaSuccess) e = hbl::launch_pack_ternary(rotated, false, N, K, packed, alpha_dev, partials, stream);
+  return cuda_status(e);
+}
+
+hbl_status hbl_norm_quant(const void* x, hbl_dtype xt, int64_t M, int64_t K, hbl_norm norm, int bits,
+                          uint8_t* codes, float* scales, cudaStream_t stream) {
+  if (!x || !codes || !scales || !dtype_ok(xt) || (bits != 4 && bits != 8) ||
+      (norm != HBL_NORM_LAYER && norm != HBL_NORM_RMS))
+    return HBL_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(codes, 16) || !aligned(scales, 4)) return HBL_ERR_INVALID_ARG;
+  hbl_status s = check_norm_k(K);
+  if (s != HBL_OK) return s;
+  if ((s = check_rows(M)) != HBL_OK) return s;
+  const K1Mode mode = bits == 4 ? hbl::K1_Q4_PACKED : hbl::K1_Q8_I8;
+  return cuda_status(hbl::launch_norm_quant(x, xt == HBL_BF16, M, K, norm == HBL_NORM_RMS, mode, codes, scales,
+                                            stream));
+}
+
+hbl_status hbl_debug_norm(const void* x, hbl_dtype xt, int64_t M, int64_t K, hbl_norm norm, float* t,
+                          cudaStream_t stream) {
+  if (!x || !t || !dtype_ok(xt) || (norm != HBL_NORM_LAYER && norm != HBL_NORM_RMS)) return HBL_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(t, 16)) return HBL_ERR_INVALID_ARG;
+  hbl_status s = check_norm_k(K);
+  if (s != HBL_OK) return s;
+  if ((s = check_rows(M)) != HBL_OK) return s;
+  return cuda_status(hbl::launch_norm_quant(x, xt == HBL_BF16, M, K, norm == HBL_NORM_RMS, hbl::K1_T_F32, t,
+                                            nullptr, stream));
 }
 
 hbl_status hbl_debug_ln_fht(const void* x, hbl_dtype xt, int64_t M, int64_t K, float* t, cudaStream_t stream) {

@@ -23,18 +23,11 @@ constexpr float kSqrt7 = 2.6457513110645906f;  // sqrt(7) rounded to float
 constexpr float kMagic = 12582912.0f;          // 1.5 * 2^23
 constexpr int kMagicBits = 0x4B400000;
 
-// |t| as a double, for the absmean accumulation, built with integer
-// operations instead of a float->double conversion (which runs on the
-// quarter-rate conversion pipe): for a normal float the double has the same
-// sign, exponent + 896 and the mantissa shifted by 29, so the value is exact.
-// Zero maps to zero.  |t| below 2^-126 (subnormal) maps into [2^-127, 2^-126),
-// i.e. it is counted with an absolute error below 2^-126 -- invisible at float
-// resolution for any row whose sum of |t| exceeds 2^-100.
-__device__ __forceinline__ double abs_f64(float t) {
-  const uint32_t b = __float_as_uint(t) & 0x7fffffffu;
-  const uint32_t hi = b ? (b >> 3) + 0x38000000u : 0u;
-  return __hiloint2double((int)hi, (int)(b << 29));
-}
+// |t| as a double, for the absmean accumulation: an exact float -> double
+// conversion (it runs on the conversion pipe, which the kernels otherwise
+// leave idle, and costs one issue slot) whose absolute value the double add
+// takes as an operand modifier.
+__device__ __forceinline__ double abs_f64(float t) { return fabs((double)t); }
 
 struct RowParams {
   float r;      // multiplier applied to t before rounding

@@ -123,17 +123,13 @@ __device__ __forceinline__ uint4 widen16(uint32_t w) {
                     __byte_perm(kLut, 0u, hi & 0xffffu), __byte_perm(kLut, 0u, hi >> 16));
 }
 
-// 64 codes (four words) per thread -> 64 int8 bytes.
+// One word (16 codes -> 16 bytes) per thread and iteration: consecutive
+// threads take consecutive words, so every store instruction of a warp writes
+// 512 contiguous bytes.
 __global__ void __launch_bounds__(kThreads)
-widen_kernel(const uint4* __restrict__ packed, int64_t nquads, uint4* __restrict__ out) {
-  for (int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x; i < nquads; i += (int64_t)gridDim.x * kThreads) {
-    const uint4 w = __ldg(packed + i);
-    uint4* o = out + 4 * i;
-    o[0] = widen16(w.x);
-    o[1] = widen16(w.y);
-    o[2] = widen16(w.z);
-    o[3] = widen16(w.w);
-  }
+widen_kernel(const uint32_t* __restrict__ packed, int64_t nwords, uint4* __restrict__ out) {
+  for (int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x; i < nwords; i += (int64_t)gridDim.x * kThreads)
+    out[i] = widen16(__ldg(packed + i));
 }
 
 int grid_for(int64_t work) {
@@ -164,8 +160,8 @@ cudaError_t launch_pack_ternary(const void* W, bool in_bf16, int64_t N, int64_t 
 }
 
 cudaError_t launch_widen_ternary(const uint8_t* packed, int64_t N, int64_t K, int8_t* out, cudaStream_t stream) {
-  const int64_t nquads = N * K / 64;  // N K is a multiple of 1024 (K >= 64, N % 16 == 0)
-  widen_kernel<<<grid_for(nquads), kThreads, 0, stream>>>(reinterpret_cast<const uint4*>(packed), nquads,
+  const int64_t nwords = N * K / 16;  // N K is a multiple of 1024 (K >= 64, N % 16 == 0)
+  widen_kernel<<<grid_for(nwords), kThreads, 0, stream>>>(reinterpret_cast<const uint32_t*>(packed), nwords,
                                                           reinterpret_cast<uint4*>(out));
   return cudaGetLastError();
 }

@@ -95,6 +95,14 @@ def test_hook_validation(L):
     assert L.hbl_debug_ln_fht(FAKE, 1, 8, 96, FAKE, S0) == hbl.HBL_ERR_UNSUPPORTED
 
 
+def test_norm_quant_validation(L):
+    assert L.hbl_norm_quant(FAKE, 1, 8, 128, 0, 4, FAKE, FAKE, S0) == hbl.HBL_ERR_UNSUPPORTED
+    assert L.hbl_norm_quant(FAKE, 1, 8, 65536, 0, 4, FAKE, FAKE, S0) == hbl.HBL_ERR_UNSUPPORTED
+    assert L.hbl_norm_quant(FAKE, 1, 8, 1024, 2, 4, FAKE, FAKE, S0) == hbl.HBL_ERR_INVALID_ARG
+    assert L.hbl_norm_quant(FAKE, 1, 8, 1024, 1, 6, FAKE, FAKE, S0) == hbl.HBL_ERR_INVALID_ARG
+    assert L.hbl_debug_norm(FAKE, 1, 0, 1024, 1, FAKE, S0) == hbl.HBL_ERR_INVALID_ARG
+
+
 def test_status_strings(L):
     assert hbl.status_string(hbl.HBL_OK) == "HBL_OK"
     assert hbl.status_string(hbl.HBL_ERR_TIMEOUT) == "HBL_ERR_TIMEOUT"

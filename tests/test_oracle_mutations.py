@@ -16,6 +16,7 @@ SRC = os.path.join(ROOT, "oracle", "hbl_oracle.c")
 # (name, text in hbl_oracle.c, replacement)
 MUTANTS = [
     ("drop 1/sqrt(K)", "double sc = 1.0 / sqrt((double)K);", "double sc = 1.0;"),
+    ("plain FHT without 1/sqrt(K)", "double inv_sqrt_k = 1.0 / sqrt((double)K);", "double inv_sqrt_k = 1.0;"),
     ("butterfly difference sign", "v[j + h] = a - b;", "v[j + h] = b - a;"),
     ("skip the last butterfly stage", "for (int64_t h = 1; h < n; h *= 2)", "for (int64_t h = 1; h < n / 2; h *= 2)"),
     ("unbiased variance", "v /= (double)K;", "v /= (double)(K - 1);"),
@@ -32,6 +33,8 @@ MUTANTS = [
     ("ternary clip to 2", "if (q > 1.0) q = 1.0;", "if (q > 2.0) q = 2.0;"),
     ("transposed GEMM operand", "s += (int64_t)A[m * K + k] * (int64_t)B[n * K + k];",
      "s += (int64_t)A[m * K + k] * (int64_t)B[k * N + n];"),
+    ("RMSNorm without the square", "for (int64_t i = 0; i < K; ++i) s += x[i] * x[i];",
+     "for (int64_t i = 0; i < K; ++i) s += x[i];"),
     ("dequant without alpha", "volatile float sa = scales[m] * alpha;", "volatile float sa = scales[m];"),
     ("nibbles swapped", "out[m * (K / 2) + j] = (uint8_t)(lo | (hi << 4));",
      "out[m * (K / 2) + j] = (uint8_t)(hi | (lo << 4));"),

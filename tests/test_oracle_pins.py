@@ -333,3 +333,50 @@ def test_forward_rows_is_the_composition(orc, bits):
     assert np.array_equal(q2, q) and np.array_equal(s2, s) and np.array_equal(y, want)
     ysel, _, _ = orc.forward_rows(x, w, a, bits, rows=[5, 2])
     assert np.array_equal(ysel, want[[5, 2]])
+
+
+# ----------------------------------------------------------------- BitLinear without the transform
+
+@pytest.mark.parametrize("K", [4, 64, 3000])
+def test_rmsnorm_matches_torch(orc, K):
+    import torch
+    x = np.random.default_rng(K).standard_normal(K) * 2.0 + 0.5
+    want = torch.nn.functional.rms_norm(torch.from_numpy(x), (K,), eps=1e-5).numpy()
+    np.testing.assert_allclose(orc.rmsnorm_row(x), want, rtol=1e-12, atol=1e-12)
+
+
+def test_rmsnorm_hand_example(orc):
+    # x = [3, 4]: mean x^2 = 12.5, u = x / sqrt(12.5 + 1e-5)
+    u = orc.rmsnorm_row(np.array([3.0, 4.0]))
+    np.testing.assert_allclose(u, [3 / math.sqrt(12.50001), 4 / math.sqrt(12.50001)], rtol=1e-14)
+
+
+@pytest.mark.parametrize("norm", [0, 1])
+def test_norm_rows_is_the_row_norm(orc, norm):
+    import torch
+    x = (np.random.default_rng(9).standard_normal((5, 96)) * 3 + 1).astype(np.float32)
+    t64, t32 = orc.norm_rows(x, norm)
+    xt = torch.from_numpy(x.astype(np.float64))
+    want = (torch.nn.functional.layer_norm(xt, (96,), eps=1e-5) if norm == 0
+            else torch.nn.functional.rms_norm(xt, (96,), eps=1e-5)).numpy()
+    np.testing.assert_allclose(t64, want, rtol=1e-12, atol=1e-12)
+    assert np.array_equal(t32, t64.astype(np.float32))
+
+
+# ----------------------------------------------------------------- rotated weights
+
+def test_rotation_preserves_dot_products(orc):
+    # H/sqrt(K) is orthogonal: (H x).(H w) = x.w -- why rotating weights and activations
+    rng = np.random.default_rng(12)
+    x = rng.standard_normal((3, 256)).astype(np.float32)
+    W = rng.standard_normal((5, 256)).astype(np.float32)
+    hx, _ = orc.fht_rows(x)
+    hw, _ = orc.fht_rows(W)
+    np.testing.assert_allclose(hx @ hw.T, x.astype(np.float64) @ W.astype(np.float64).T, rtol=1e-12, atol=1e-11)
+
+
+def test_fht_rows_matches_scipy(orc):
+    x = np.random.default_rng(2).standard_normal((2, 64)).astype(np.float32)
+    t64, t32 = orc.fht_rows(x)
+    np.testing.assert_allclose(t64, x.astype(np.float64) @ scipy.linalg.hadamard(64).T / 8.0, atol=1e-12)
+    assert np.array_equal(t32, t64.astype(np.float32))
