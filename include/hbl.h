@@ -244,6 +244,14 @@ hbl_status hbl_debug_raise_device_error(cudaStream_t stream);
 /* Static string for a status code. */
 const char* hbl_status_string(hbl_status status);
 
+/* The CUDA runtime error code (a cudaError_t value) behind the most recent
+ * HBL_ERR_CUDA returned on this host thread, 0 if there was none.  Reading it
+ * does not clear it. */
+int hbl_last_cuda_error(void);
+
+/* Static name of a CUDA runtime error code, e.g. "cudaErrorInvalidValue". */
+const char* hbl_cuda_error_name(int code);
+
 #ifdef __cplusplus
 }
 #endif

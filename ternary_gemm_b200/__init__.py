@@ -29,7 +29,12 @@ _lib = None
 class HBLError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
-        super().__init__("%s failed: %s" % (where, status_string(status)))
+        self.cuda_error = None
+        msg = "%s failed: %s" % (where, status_string(status))
+        if status == HBL_ERR_CUDA:
+            self.cuda_error = int(lib().hbl_last_cuda_error())
+            msg += " (%s)" % lib().hbl_cuda_error_name(self.cuda_error).decode()
+        super().__init__(msg)
 
 
 def declared_symbols():
@@ -93,6 +98,10 @@ def lib():
             L.hbl_debug_raise_device_error.restype = i32
             L.hbl_status_string.argtypes = [i32]
             L.hbl_status_string.restype = ctypes.c_char_p
+            L.hbl_last_cuda_error.argtypes = []
+            L.hbl_last_cuda_error.restype = ctypes.c_int
+            L.hbl_cuda_error_name.argtypes = [ctypes.c_int]
+            L.hbl_cuda_error_name.restype = ctypes.c_char_p
             _lib = L
     return _lib
 

@@ -29,6 +29,13 @@ constexpr int kMaxLogK = 15;  // K = 32768
 cudaError_t launch_ln_fht_quant(const void* x, bool in_bf16, int64_t M, int log2k, K1Mode mode,
                                 void* out, float* scales, cudaStream_t stream);
 
+// The same operation with the high Hadamard factor on the tensor cores
+// (bf16 input, K in [128, 16384], 16-byte aligned x and out, not
+// K1_FHT_F32); launch_ln_fht_quant dispatches to it when supported.
+bool ln_fht_quant_tc_supports(bool in_bf16, int log2k, K1Mode mode, const void* x, const void* out);
+cudaError_t launch_ln_fht_quant_tc(const void* x, int64_t M, int log2k, K1Mode mode, void* out, float* scales,
+                                   cudaStream_t stream);
+
 // LayerNorm (rms = false) or RMSNorm (rms = true) then the quantizer, without
 // the Hadamard transform; K a power of two in [256, 32768].
 cudaError_t launch_norm_quant(const void* x, bool in_bf16, int64_t M, int64_t K, bool rms, K1Mode mode,
@@ -58,6 +65,9 @@ cudaError_t launch_gemm_i8(const int8_t* A, const int8_t* B, int64_t M, int64_t 
 // Device error word (bounded-wait timeouts) -- lives in gemm_i8.cu; kernels in
 // other translation units receive its device address.
 int* device_error_word();
+// Records e as the thread's last CUDA error (hbl_last_cuda_error) and maps it
+// to a status: HBL_OK for cudaSuccess, else HBL_ERR_CUDA.
+hbl_status note_cuda_error(cudaError_t e);
 cudaError_t read_and_clear_device_error(cudaStream_t stream, int* value);
 cudaError_t raise_device_error(cudaStream_t stream);
 

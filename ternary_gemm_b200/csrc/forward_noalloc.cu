@@ -63,6 +63,7 @@ extern "C" hbl_status hbl_forward_noalloc(const void* x, hbl_dtype xt, int64_t M
   if (s != HBL_ERR_WORKSPACE) return s;
   if (hbl_forward_workspace_bytes(M, K, N, bits) > kNoAllocScratchBytes) return HBL_ERR_WORKSPACE;
   void* scratch = nullptr;
-  if (scratch_address(&scratch) != cudaSuccess) return HBL_ERR_CUDA;
+  cudaError_t e = scratch_address(&scratch);
+  if (e != cudaSuccess) return hbl::note_cuda_error(e);
   return hbl_forward(x, xt, M, K, packed, alpha_dev, N, bits, y, yt, scratch, kNoAllocScratchBytes, stream);
 }

@@ -24,7 +24,13 @@ size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
 bool dtype_ok(hbl_dtype t) { return t == HBL_F32 || t == HBL_BF16; }
 
-hbl_status cuda_status(cudaError_t e) { return e == cudaSuccess ? HBL_OK : HBL_ERR_CUDA; }
+thread_local int g_last_cuda_error = 0;
+
+hbl_status cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return HBL_OK;
+  g_last_cuda_error = (int)e;
+  return HBL_ERR_CUDA;
+}
 
 // K a power of two in [64, 32768] -> log2 K, else -1 / -2 (unsupported)
 hbl_status check_k(int64_t K, int* log2k) {
@@ -67,6 +73,10 @@ ForwardLayout forward_layout(int64_t M, int64_t K, int64_t N) {
 }
 
 }  // namespace
+
+namespace hbl {
+hbl_status note_cuda_error(cudaError_t e) { return cuda_status(e); }
+}  // namespace hbl
 
 extern "C" {
 
@@ -277,7 +287,7 @@ hbl_status hbl_gemm_i8_i32(const int8_t* A, const int8_t* B, int64_t M, int64_t 
 hbl_status hbl_last_device_error(cudaStream_t stream) {
   int v = 0;
   cudaError_t e = hbl::read_and_clear_device_error(stream, &v);
-  if (e != cudaSuccess) return HBL_ERR_CUDA;
+  if (e != cudaSuccess) return cuda_status(e);
   return v ? HBL_ERR_TIMEOUT : HBL_OK;
 }
 
@@ -296,5 +306,9 @@ const char* hbl_status_string(hbl_status status) {
   }
   return "HBL_ERR_UNKNOWN";
 }
+
+int hbl_last_cuda_error(void) { return g_last_cuda_error; }
+
+const char* hbl_cuda_error_name(int code) { return cudaGetErrorName((cudaError_t)code); }
 
 }  // extern "C"

@@ -109,6 +109,13 @@ def test_status_strings(L):
     assert hbl.status_string(99) == "HBL_ERR_UNKNOWN"
 
 
+def test_cuda_error_reporting(L):
+    # argument errors are not CUDA errors: nothing is recorded
+    assert L.hbl_fht_quant(None, 1, 8, 1024, 4, FAKE, FAKE, S0) == hbl.HBL_ERR_INVALID_ARG
+    assert L.hbl_last_cuda_error() == 0
+    assert L.hbl_cuda_error_name(1) == b"cudaErrorInvalidValue"
+
+
 def test_binding_fails_loudly_without_library(monkeypatch):
     monkeypatch.setattr(hbl, "_lib", None)
     monkeypatch.setattr(hbl, "LIB_PATH", "/nonexistent/libhbl.so")
