@@ -4,49 +4,69 @@
 // 1-bit LLMs", section "H-BitLinear": the Hadamard-transform definition and
 // the activation-quantization formula).  bf16 input, K = 128 .. 16384.
 //
-// Sylvester's matrix factors over the index bits: with i = 128 i_hi + i_lo,
-// j = 128 j_hi + j_lo and KH = K / 128,
-//   H_K[i][j] = H_KH[i_hi][j_hi] * H_128[i_lo][j_lo],
+// Sylvester's matrix factors over the index bits: with i = C i_hi + i_lo,
+// j = C j_hi + j_lo and KH = K / C,
+//   H_K[i][j] = H_KH[i_hi][j_hi] * H_C[i_lo][j_lo],
 // so Y = H_K x is two smaller transforms.  The high one is a dense
 // contraction whose operands are exact in bf16 (x itself and +-1), so it runs
-// on the tensor cores; the low one (7 butterfly stages) runs in registers:
+// on the tensor cores; the low one runs as butterflies in registers.  The
+// chunk width is C = 64 for K <= 8192 (KH = 2 .. 128) and C = 128 for
+// K = 16384 (KH = 128), so KH never exceeds the MMA's 128:
 //
-//   x viewed as chunk rows Xc[M*KH][128] (row-major, no copy);
-//   tile    = 128 consecutive chunk rows = 128/KH token rows;
-//   MMA     D[m][n] = sum_k A[m][k] Xc[tile*128 + k][n],
-//           A = blockdiag(H_KH, ..., H_KH) (128 x 128, bf16 +-1/0),
-//           tcgen05.mma kind::f16, M = N = 128, K = 16 x 8, f32 in TMEM;
-//           lane m = (token row r = m / KH, i_hi = m % KH), column n = j_lo;
-//   thread  m loads its 128 columns (one TMEM lane), runs the 7 stages over
-//           j_lo in registers and owns Y[r][128 i_hi .. 128 i_hi + 127],
-//           a contiguous slice of the transformed row.
-// The tensor-core sums are exact whenever the 128 bf16 terms span < 2^9 in
-// magnitude (their common unit in the last place then divides the result),
-// and otherwise round in float like the butterflies would.
+//   x viewed as chunk rows Xc[M*KH][C] (row-major, no copy);
+//   box     = 128 chunk rows x 64 columns of bf16 (16 KB), one TMA copy;
+//   group   = two boxes side by side: C = 64, two consecutive 128-row units;
+//             C = 128, the two column halves of one 128-row tile;
+//   MMA     D[m][n] = sum_k A[m][k] B[k][n], tcgen05.mma kind::f16,
+//           M = 128, N = 128 (the group's two boxes), K = 8 x 16, f32
+//           accumulator in TMEM; A = blockdiag(H_KH, ..., H_KH) (+-1 / 0)
+//           is written into TMEM once, so the tensor core reads only x from
+//           shared memory.  Lane m of a box = (token row m / KH, i_hi =
+//           m % KH).  Wide MMAs matter: an N = 64 MMA costs about as long as
+//           an N = 128 one, and at N = 64 the MMA time did not hide under
+//           the loads.
+//   C = 64  each 64-column half of D is one unit, taken by one epilogue
+//           warpgroup: 64 columns per thread, 6 butterfly stages.
+//   C = 128 a pair of epilogue warpgroups shares the tile: warpgroup h loads
+//           columns 64h .. 64h + 63 of its lanes, runs the 6 stages of the
+//           low 6 column bits, keeps columns 32h .. 32h + 31 and
+//           64 + 32h .. 95 + 32h, and swaps the other 32 with its partner
+//           through TMEM (behind a pair barrier) for the stage on column
+//           bit 6.  Each thread ends with 64 values.
+// The tensor-core sums are exact whenever the bf16 terms of a sum span < 2^9
+// in magnitude (their common unit in the last place then divides the
+// result), and otherwise round in float like the butterflies would.
 //
-// LayerNorm is folded around the transform as in the register kernel: row 0
-// of H is all ones, so sum_{i>=1} Y_i^2 = K^2 var and t_i = Y_i / sqrt(K (var
-// + eps_ln)) for i >= 1, t_0 = 0.  A large row mean only reaches the lanes
-// with i_hi = 0 (the other rows of H_KH sum to zero); those subtract their own
-// column-0 value from all 128 columns before the butterflies, which changes
-// only Y_0 (discarded) and keeps the float sums on the deviations.
+// LayerNorm is folded around the transform: row 0 of H is all ones, so
+// sum_{i>=1} Y_i^2 = K^2 var and t_i = Y_i / sqrt(K (var + eps_ln)) for
+// i >= 1, t_0 = 0.  A large row mean only reaches the lanes with i_hi = 0
+// (the other rows of H_KH sum to zero); those subtract their own column-0
+// value from all C columns before the butterflies, which changes only Y_0
+// (discarded) and keeps the float sums on the deviations.
 //
-// CTA (one per SM, persistent over tiles), three warpgroups:
-//   warp 0     TMA producer: two 64-element-wide 128B-swizzled boxes per
-//              tile (the MN-major B operand) into a 4-stage ring;
-//   warp 1     TMEM allocation (4 accumulators x 128 columns) and one thread
-//              issuing the 8 MMAs of a tile;
+// CTA (one per SM, persistent over groups), five warpgroups:
+//   warp 0     TMA producer: two boxes per group into a 4-group ring;
+//   warp 1     TMEM allocation (512 columns: A in the last 64, three
+//              128-column accumulator regions) and one thread issuing the
+//              MMAs of a group;
 //   warps 2-3  idle (registers are granted to whole warpgroups);
-//   warps 4-11 two epilogue warpgroups taking alternate tiles: TMEM -> 128
-//              registers, butterflies, LayerNorm statistics, quantizer, codes
-//              into a swizzled staging tile that one TMA store writes out
-//              (the tile's codes are contiguous in the output).
-// Registers are allocated for 4-warp groups, so the block is launched with
-// 168 per thread and rebalanced with setmaxnreg: the first warpgroup gives
-// its share down to 40, the epilogue warpgroups take 208 each (the host
-// checks that the launch count covers this split before launching).
-// Every mbarrier wait is bounded (2 s, then the CTA abort flag and the device
-// error word are set and every role leaves its loop).
+//   warps 4-19 four epilogue warpgroups in two pairs; pair p takes every
+//              other group: TMEM -> registers, butterflies, LayerNorm
+//              statistics, quantizer, codes into a swizzled staging tile that
+//              a TMA store writes out.
+// Row statistics reduce over the threads of a token row: warp shuffles, then
+// per-warp slots behind a named barrier of the row's warpgroup (pair).  The
+// INT4 absmean is summed in float (trees of depth <= 22, so beta is within
+// 1.3e-6 relative of a double sum; a double per-element sum cost about a
+// fifth of the kernel's time), INT8 absmax is exact.  INT4 codes widened to
+// int8 are clipped on packed 16-bit halves when the row bound ||t|| r keeps
+// every code below 2^15, else on 32-bit values.
+// The block is launched with at most 96 registers per thread and rebalanced
+// with setmaxnreg: the first warpgroup gives its share down to 40, the
+// epilogue warpgroups take 104 each (the host checks that the launch count
+// covers this split before launching).  Every mbarrier wait is bounded (2 s,
+// then the CTA abort flag and the device error word are set and every role
+// leaves its loop).
 #include <cstdint>
 
 #include "common.cuh"
@@ -60,98 +80,193 @@ namespace {
 using namespace sm100;
 using namespace rowkit;
 
-constexpr int kTileChunks = 128;                      // chunk rows per tile (MMA K)
-constexpr int kTileBytes = kTileChunks * 128 * 2;     // 32 KB of bf16
-constexpr int kStages = 4;
-constexpr int kABytes = 128 * 128 * 2;                // blockdiag(H_KH) in bf16
-constexpr int kOutBytes = kTileChunks * 128;          // int8 codes of a tile
-constexpr int kEpiGroups = 2;
+constexpr int kBoxCols = 64;                         // bf16 columns per box (one 128-byte swizzle row)
+constexpr int kBoxRows = 128;                        // chunk rows per box (MMA M and K)
+constexpr int kBoxBytes = kBoxRows * kBoxCols * 2;   // 16 KB
+constexpr int kSlots = 4;                            // ring slots of two boxes (one group)
+constexpr int kSlotBytes = 2 * kBoxBytes;
+constexpr int kStageOutBytes = kBoxRows * kBoxCols;  // int8 codes of a box (the largest staged form)
+constexpr int kEpiGroups = 4;                        // epilogue warpgroups
 constexpr int kThreads = 128 + 128 * kEpiGroups;
-constexpr int kCtrlRegs = 40;   // registers per thread of the first warpgroup after setmaxnreg
-constexpr int kEpiRegs = 208;   // registers per thread of an epilogue warpgroup after setmaxnreg
-constexpr int kAcc = 4;
-constexpr uint32_t kTmemCols = 128 * kAcc;
-constexpr size_t kSmemBytes = 1024 + kABytes + (size_t)kStages * kTileBytes + kEpiGroups * kOutBytes + 512;
+constexpr int kCtrlRegs = 40;  // registers per thread of the first warpgroup after setmaxnreg
+constexpr int kEpiRegs = 104;  // registers per thread of an epilogue warpgroup after setmaxnreg
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kAcol = 448;  // TMEM column of A (64 columns: 128 bf16 per lane)
+constexpr int kRegions = 3;      // 128-column accumulators below kAcol
+constexpr size_t kSmemBytes = 1024 + (size_t)kSlots * kSlotBytes + (size_t)kEpiGroups * kStageOutBytes + 1024;
 
 // instruction descriptor, kind::f16: D f32, A and B bf16, A K-major, B
 // MN-major, N = 128, M = 128
-constexpr uint32_t kIdesc =
-    (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
+constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
 
 struct TcParams {
   int64_t M;         // token rows
-  int num_tiles;     // ceil(M * KH / 128)
+  int64_t nchunk;    // chunk rows, M * KH
+  int num_groups;    // MMA groups
   float sK;          // 1 / sqrt(K) rounded to float
   float* t_out;      // K1_T_F32: t [M][K]
   float* scales;     // [M]
   int* err;          // device error word
 };
 
-__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t accumulate) {
+// D (TMEM) (+)= A (TMEM) x B (shared memory descriptor)
+__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b, uint32_t accumulate) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
-      "l"(a), "l"(b), "r"(kIdesc), "r"(accumulate));
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b), "r"(kIdesc), "r"(accumulate));
 }
 
-// Butterfly over register-index bit B of a 128-float array.
-template <int B>
-__device__ __forceinline__ void stage128(float (&e)[128]) {
+// one TMEM column of this warp's lane quarter
+__device__ __forceinline__ uint32_t tmem_ld1(uint32_t taddr) {
+  uint32_t v;
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(v) : "r"(taddr));
+  return v;
+}
+
+// Butterfly over register-index bit B of an N-float array.
+template <int B, int N>
+__device__ __forceinline__ void stage(float (&e)[N]) {
   if constexpr (B == 0) {
 #pragma unroll
-    for (int r = 0; r < 128; r += 2) {
+    for (int r = 0; r < N; r += 2) {
       const float a = e[r], c = e[r + 1];
       e[r] = a + c;
       e[r + 1] = a - c;
     }
   } else {
 #pragma unroll
-    for (int r = 0; r < 128; r += 2)
+    for (int r = 0; r < N; r += 2)
       if (!(r & (1 << B))) bfly2(e[r], e[r + 1], e[r | (1 << B)], e[(r | (1 << B)) + 1]);
   }
 }
 
-// All-reduce over the KH consecutive TMEM lanes (threads) of one token row.
-// Every thread of the row ends with the identical value.  Rows wider than a
-// warp combine warp partials through `slots` behind the warpgroup's barrier.
-template <int KH, typename V, typename Op>
-__device__ __forceinline__ V group_reduce(V v, Op op, V* slots, int quarter, int lane, int bar_id) {
-  constexpr int W = KH < 32 ? KH : 32;
+// All-reduce over the RT threads of one token row: RT consecutive lanes when
+// RT <= 32, else RT / 32 whole warps numbered wq (their slots) inside the
+// barrier's `bar_n` threads.  Every thread of the row ends with the identical
+// value.  Each reduction of a group uses its own `slots`.
+template <int RT, typename V, typename Op>
+__device__ __forceinline__ V group_reduce(V v, Op op, V* slots, int wq, int lane, int bar_id, int bar_n) {
+  constexpr int W = RT < 32 ? RT : 32;
 #pragma unroll
   for (int o = W / 2; o >= 1; o >>= 1) v = op(v, __shfl_xor_sync(0xffffffffu, v, o));
-  if constexpr (KH > 32) {
-    if (lane == 0) slots[quarter] = v;
-    named_bar_sync(bar_id, 128);
-    if constexpr (KH == 128)
-      v = op(op(slots[0], slots[1]), op(slots[2], slots[3]));
-    else
-      v = op(slots[quarter & 2], slots[(quarter & 2) | 1]);
+  if constexpr (RT > 32) {
+    constexpr int NW = RT / 32;
+    if (lane == 0) slots[wq] = v;
+    named_bar_sync(bar_id, bar_n);
+    const int w0 = wq & ~(NW - 1);
+    v = slots[w0];
+#pragma unroll
+    for (int i = 1; i < NW; ++i) v = op(v, slots[w0 + i]);
   }
   return v;
 }
 
-// blockdiag(H_KH) as bf16 in the K-major 128B-swizzled layout: two 64-column
-// blocks of 128 rows x 128 bytes; 16-byte chunk c of row m sits at chunk
-// position c ^ (m & 7).
-template <int KH>
-__device__ __forceinline__ void build_a(uint8_t* sA, int tid, int nthreads) {
-  for (int c = tid; c < 2048; c += nthreads) {
-    const int blk = c >> 10, m = (c >> 3) & 127, cc = c & 7;
-    uint32_t w[4];
+// Per-thread reductions over y[0..63] with 8 independent accumulators (8
+// short dependency chains) and a final tree, so they do not serialize on
+// the add latency.
+__device__ __forceinline__ float sum_sq64(const float (&y)[64]) {
+  float s[8];
 #pragma unroll
-    for (int u = 0; u < 8; u += 2) {
-      uint32_t h[2];
+  for (int a = 0; a < 8; ++a) s[a] = 0.0f;
+#pragma unroll
+  for (int r = 0; r < 64; r += 2) sq_acc2(s[(r >> 1) & 6], s[((r >> 1) & 6) + 1], y[r], y[r + 1]);
+#pragma unroll
+  for (int w = 4; w >= 1; w >>= 1)
+#pragma unroll
+    for (int a = 0; a < w; ++a) s[a] += s[a + w];
+  return s[0];
+}
+
+// sum |y| in float (the |.| is an operand modifier of the adds)
+__device__ __forceinline__ float sum_abs64(const float (&y)[64]) {
+  float v[8];
+#pragma unroll
+  for (int a = 0; a < 8; ++a) v[a] = fabsf(y[a]);
+#pragma unroll
+  for (int r = 8; r < 64; ++r) v[r & 7] += fabsf(y[r]);
+#pragma unroll
+  for (int w = 4; w >= 1; w >>= 1)
+#pragma unroll
+    for (int a = 0; a < w; ++a) v[a] += v[a + w];
+  return v[0];
+}
+
+// max |y| (order-free and exact)
+__device__ __forceinline__ float max_abs64(const float (&y)[64]) {
+  float v[8];
+#pragma unroll
+  for (int a = 0; a < 8; ++a) v[a] = fabsf(y[a]);
+#pragma unroll
+  for (int r = 8; r < 64; ++r) v[r & 7] = fmaxf(v[r & 7], fabsf(y[r]));
+#pragma unroll
+  for (int w = 4; w >= 1; w >>= 1)
+#pragma unroll
+    for (int a = 0; a < w; ++a) v[a] = fmaxf(v[a], v[a + w]);
+  return v[0];
+}
+
+// Row m of A = blockdiag(H_KH, ..., H_KH) (128 x 128, bf16 +-1 / 0) as 64
+// TMEM words: word c holds A[m][2c] in its low half and A[m][2c + 1] in its
+// high half; written by the warp that owns lane m.
+template <int KH>
+__device__ __forceinline__ void store_a_row(uint32_t taddr, int m) {
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+    uint32_t w[32];
+#pragma unroll
+    for (int c = 0; c < 32; ++c) {
+      uint32_t hv[2];
 #pragma unroll
       for (int v = 0; v < 2; ++v) {
-        const int k = blk * 64 + cc * 8 + u + v;
+        const int k = 64 * half + 2 * c + v;
         const bool same = (m / KH) == (k / KH);
-        h[v] = !same ? 0u : ((__popc((m % KH) & (k % KH)) & 1) ? 0xBF80u : 0x3F80u);
+        hv[v] = !same ? 0u : (0x3F80u ^ ((uint32_t)(__popc((m % KH) & (k % KH)) & 1) << 15));
       }
-      w[u >> 1] = h[0] | (h[1] << 16);
+      w[c] = hv[0] | (hv[1] << 16);
     }
-    *reinterpret_cast<uint4*>(sA + blk * 16384 + m * 128 + ((cc ^ (m & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+    tmem_st32(taddr + (uint32_t)(32 * half), w);
   }
+}
+
+// 16 int8 codes of y[0..15] (INT8 absmax, or INT4 codes widened to int8).
+// INT4 with S16: clip on packed 16-bit halves (every |code| < 2^15).
+template <int MODE, bool S16 = false>
+__device__ __forceinline__ uint4 codes16_i8(const float* y, float r) {
+  uint32_t w[4];
+#pragma unroll
+  for (int hh = 0; hh < 4; ++hh) {
+    uint32_t mm[4];
+    magic2(y[4 * hh], y[4 * hh + 1], r, mm[0], mm[1]);
+    magic2(y[4 * hh + 2], y[4 * hh + 3], r, mm[2], mm[3]);
+    if constexpr (MODE == K1_Q4_I8 && S16) {
+      w[hh] = __byte_perm(q::clip_pair_int4_s16(mm[0], mm[1]), q::clip_pair_int4_s16(mm[2], mm[3]), 0x6420);
+    } else {
+      if constexpr (MODE == K1_Q4_I8) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) mm[u] = q::clip_magic_int4(mm[u]);
+      }
+      w[hh] = q::gather_low_bytes(mm[0], mm[1], mm[2], mm[3]);
+    }
+  }
+  return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// 32 INT4 codes of y[0..31] as packed nibbles (y[0] in the lowest nibble)
+__device__ __forceinline__ uint4 codes32_s4(const float* y, float r) {
+  uint32_t w[4];
+#pragma unroll
+  for (int hh = 0; hh < 4; ++hh) {
+    uint32_t mm[8];
+#pragma unroll
+    for (int u = 0; u < 8; u += 2) magic2(y[8 * hh + u], y[8 * hh + u + 1], r, mm[u], mm[u + 1]);
+    int n[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) n[u] = (int)mm[u] - q::kMagicBits;
+    w[hh] = q::pack_s4x8(n);
+  }
+  return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
 template <int LOGK, int MODE>
@@ -159,236 +274,315 @@ __global__ void __launch_bounds__(kThreads, 1)
 ln_fht_quant_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmOut,
                        TcParams p) {
   constexpr int K = 1 << LOGK;
-  constexpr int KH = K / 128;
+  constexpr int C = LOGK >= 14 ? 128 : 64;  // chunk width
+  constexpr int KH = K / C;                 // chunk rows per token row
+  static_assert(KH >= 2 && KH <= 128, "K out of range");
+  constexpr bool PAIR = C == 128;           // a warpgroup pair shares each tile
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-  uint8_t* sA = base;
-  uint8_t* sB = sA + kABytes;
-  uint8_t* sOut = sB + kStages * kTileBytes;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sOut + kEpiGroups * kOutBytes);
-  uint64_t* empty = full + kStages;
-  uint64_t* tfull = empty + kStages;
-  uint64_t* tempty = tfull + kAcc;
-  uint64_t* drain = tempty + kAcc;
-  double* red_d = reinterpret_cast<double*>(drain + 1);     // [kEpiGroups][4]
-  float* red_f = reinterpret_cast<float*>(red_d + 4 * kEpiGroups);  // [kEpiGroups][4]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(red_f + 4 * kEpiGroups);
+  uint8_t* sB = base;
+  uint8_t* sOut = sB + kSlots * kSlotBytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sOut + kEpiGroups * kStageOutBytes);
+  uint64_t* empty = full + kSlots;
+  uint64_t* tfull = empty + kSlots;
+  uint64_t* tempty = tfull + kRegions;
+  uint64_t* drain = tempty + kRegions;
+  float* red_f = reinterpret_cast<float*>(drain + 1);    // [pair][16]: squares; |t| sums or maxima
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(red_f + 32);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < kSlots; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    for (int a = 0; a < kAcc; ++a) {
+    for (int a = 0; a < kRegions; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 4);
+      mbar_init(&tempty[a], 8);  // the 8 warps of the pair that reads the region
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 1) tmem_alloc(tmem_slot, kTmemCols);
-  if (warp >= 4) {
-    build_a<KH>(sA, threadIdx.x - 128, kThreads - 128);
-    fence_proxy_async_smem();
-  }
   fence_before();
   __syncthreads();
   fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // A into TMEM: the first epilogue warpgroup writes its four lane quarters
+  if (warp >= 4 && warp < 8) {
+    store_a_row<KH>(tmem_base + kAcol + ((uint32_t)((warp & 3) * 32) << 16), (warp & 3) * 32 + lane);
+    tmem_wait_st();
+  }
+  fence_before();
+  __syncthreads();
+  fence_after();
 
   if (warp < 4) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kCtrlRegs));
-  if (warp == 0) {
-    // ------------------------------------------------ TMA producer
-    if (lane == 0) {
-      prefetch_tensormap(&tmX);
-      int stage = 0;
-      uint32_t phase = 0;
-      bool ok = true;
-      for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
-        if (!wait_bounded(&empty[stage], phase ^ 1u, abort_flag, p.err)) { ok = false; break; }
-        mbar_expect_tx(&full[stage], (uint32_t)kTileBytes);
-        uint8_t* dst = sB + stage * kTileBytes;
-        tma_load_2d(dst, &tmX, 0, tile * kTileChunks, &full[stage]);
-        tma_load_2d(dst + kTileBytes / 2, &tmX, 64, tile * kTileChunks, &full[stage]);
-        if (++stage == kStages) { stage = 0; phase ^= 1u; }
-      }
-      if (!ok) {
-        // give the copies already issued time to land before the CTA exits
-        const uint64_t t0 = globaltimer();
-        while (globaltimer() - t0 < 20000000ull) {
-        }
-      }
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
-      const uint32_t a_addr = smem_u32(sA);
-      for (int it = 0, tile = blockIdx.x; tile < p.num_tiles; ++it, tile += gridDim.x) {
-        const int acc = it & (kAcc - 1);
-        const uint32_t acc_phase = (uint32_t)(it / kAcc) & 1u;
-        if (!wait_bounded(&tempty[acc], acc_phase ^ 1u, abort_flag, p.err)) break;
-        if (!wait_bounded(&full[stage], phase, abort_flag, p.err)) break;
-        fence_after();
-        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * 128);
-        const uint64_t b0 = sdesc_mn_sw128(smem_u32(sB + stage * kTileBytes), kTileBytes / 2);
+    if (warp == 0) {
+      // ---------------------------------------------- TMA producer
+      if (lane == 0) {
+        prefetch_tensormap(&tmX);
+        bool ok = true;
+        for (int j = 0;; ++j) {
+          const int q = blockIdx.x + j * gridDim.x;
+          if (q >= p.num_groups) break;
+          const int slot = j % kSlots;
+          if (!wait_bounded(&empty[slot], ((uint32_t)(j / kSlots) & 1u) ^ 1u, abort_flag, p.err)) {
+            ok = false;
+            break;
+          }
+          mbar_expect_tx(&full[slot], (uint32_t)kSlotBytes);
+          uint8_t* dst = sB + slot * kSlotBytes;
 #pragma unroll
-        for (int s = 0; s < 8; ++s) {
-          // A: K-major, 32 bytes per K=16 step inside a 64-column block
-          const uint64_t a = sdesc_k_sw128(a_addr + (uint32_t)((s >> 2) * 16384)) + (uint64_t)(2 * (s & 3));
-          // B: MN-major, 16 chunk rows (2048 bytes) per K=16 step
-          mma_bf16(d_tmem, a, b0 + (uint64_t)(128 * s), s > 0 ? 1u : 0u);
+          for (int u = 0; u < 2; ++u) {
+            if constexpr (PAIR)
+              tma_load_2d(dst + u * kBoxBytes, &tmX, kBoxCols * u, q * kBoxRows, &full[slot]);
+            else
+              tma_load_2d(dst + u * kBoxBytes, &tmX, 0, (2 * q + u) * kBoxRows, &full[slot]);
+          }
         }
-        umma_commit(&empty[stage]);
-        umma_commit(&tfull[acc]);
-        if (++stage == kStages) { stage = 0; phase ^= 1u; }
+        if (!ok) {
+          // give the copies already issued time to land before the CTA exits
+          const uint64_t t0 = globaltimer();
+          while (globaltimer() - t0 < 20000000ull) {
+          }
+        }
       }
-      // all MMAs issued by this thread are complete once this commit arrives
-      umma_commit(drain);
-      const uint64_t t0 = globaltimer();
-      while (!mbar_try_wait(drain, 0) && globaltimer() - t0 < 200000000ull) {
+    } else if (warp == 1) {
+      // ---------------------------------------------- MMA issuer
+      if (lane == 0) {
+        const uint32_t a_tm = tmem_base + kAcol;
+        for (int j = 0;; ++j) {
+          const int q = blockIdx.x + j * gridDim.x;
+          if (q >= p.num_groups) break;
+          const int slot = j % kSlots, region = j % kRegions;
+          if (!wait_bounded(&tempty[region], ((uint32_t)(j / kRegions) & 1u) ^ 1u, abort_flag, p.err)) break;
+          if (!wait_bounded(&full[slot], (uint32_t)(j / kSlots) & 1u, abort_flag, p.err)) break;
+          fence_after();
+          const uint32_t d = tmem_base + (uint32_t)(region * 128);
+          // B: MN-major, the two boxes are the two 64-column atoms (16 KB
+          // apart); 16 chunk rows (2048 bytes) per K=16 step.  A: 8 TMEM
+          // columns (16 bf16 per lane) per K=16 step.
+          const uint64_t b = sdesc_mn_sw128(smem_u32(sB + slot * kSlotBytes), kBoxBytes);
+#pragma unroll
+          for (int s = 0; s < 8; ++s) mma_bf16_ts(d, a_tm + 8u * s, b + (uint64_t)(128 * s), s > 0 ? 1u : 0u);
+          umma_commit(&empty[slot]);
+          umma_commit(&tfull[region]);
+        }
+        // all MMAs issued by this thread are complete once this commit arrives
+        umma_commit(drain);
+        const uint64_t t0 = globaltimer();
+        while (!mbar_try_wait(drain, 0) && globaltimer() - t0 < 200000000ull) {
+        }
       }
     }
-  }
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kEpiRegs));
     // ------------------------------------------------ epilogue warpgroups
-    const int grp = (warp - 4) >> 2;
-    const int quarter = warp & 3;
-    const int m = quarter * 32 + lane;  // TMEM lane = (token row in tile, i_hi)
-    const int r_loc = m / KH;
-    const int i_hi = m % KH;
-    const int bar_id = 1 + grp;
-    const bool issuer = (warp == 4 + 4 * grp) && lane == 0;
-    uint8_t* stg = sOut + grp * kOutBytes;
-    double* slot_d = red_d + 4 * grp;
-    float* slot_f = red_f + 4 * grp;
-    for (int it = grp, tile = blockIdx.x + grp * gridDim.x; tile < p.num_tiles;
-         it += kEpiGroups, tile += kEpiGroups * gridDim.x) {
-      const int acc = it & (kAcc - 1);
-      const uint32_t acc_phase = (uint32_t)(it / kAcc) & 1u;
-      // the previous TMA store of this group has finished reading the staging tile
+    const int g = (warp - 4) >> 2;    // epilogue warpgroup
+    const int quarter = warp & 3;     // its TMEM lane quarter
+    const int pr = g >> 1;            // pair: groups j = pr, pr + 2, ...
+    const int h = g & 1;              // column half of the group's accumulator
+    const int m = quarter * 32 + lane;
+    const int bar_wg = 1 + g;
+    const int bar_pair = 1 + kEpiGroups + pr;
+    constexpr int RT = PAIR ? 256 : KH;          // threads of a token row
+    const int bar_row = PAIR ? bar_pair : bar_wg;
+    const int bar_row_n = PAIR ? 256 : 128;
+    const int wq = PAIR ? 4 * h + quarter : quarter;  // warp number among the row's warps
+    const bool issuer = quarter == 0 && lane == 0 && (!PAIR || h == 0);
+    // PAIR: the pair's two staging buffers form one 16 KB tile
+    uint8_t* stg = sOut + (PAIR ? pr * 2 : g) * kStageOutBytes;
+    float* slot_ss = red_f + 16 * pr + (PAIR ? 0 : 4 * h);
+    float* slot_mx = slot_ss + 8;
+    const int i_hi = PAIR ? m : m % KH;
+    for (int j = pr;; j += 2) {
+      const int q = blockIdx.x + j * gridDim.x;
+      if (q >= p.num_groups) break;
+      const int region = j % kRegions;
+      // the previous TMA store of this staging tile has finished reading it
       if (issuer) bulk_wait_read_all();
       int ok = 1;
-      if (lane == 0) ok = wait_bounded(&tfull[acc], acc_phase, abort_flag, p.err) ? 1 : 0;
+      if (lane == 0) ok = wait_bounded(&tfull[region], (uint32_t)(j / kRegions) & 1u, abort_flag, p.err) ? 1 : 0;
       ok = __shfl_sync(0xffffffffu, ok, 0);
-      if (named_bar_any(bar_id, 128, ok == 0)) break;
+      if (named_bar_any(bar_row, bar_row_n, ok == 0)) break;
       fence_after();
+      const uint32_t tl = tmem_base + (uint32_t)(region * 128) + ((uint32_t)(quarter * 32) << 16);
 
-      float y[128];
-      {
-        const uint32_t taddr = tmem_base + (uint32_t)(acc * 128) + ((uint32_t)(quarter * 32) << 16);
-        uint32_t u[128];
+      float y[64];
+      int64_t row;     // token row of this thread's values
+      int64_t unit0;   // first chunk row of the box this warpgroup stores (C = 64)
+      if constexpr (!PAIR) {
+        const int unit = 2 * q + h;
+        unit0 = (int64_t)unit * kBoxRows;
+        row = (int64_t)unit * (kBoxRows / KH) + m / KH;
+        {
+          uint32_t u[64];
+          tmem_ld32_nowait(tl + (uint32_t)(64 * h), &u[0]);
+          tmem_ld32_nowait(tl + (uint32_t)(64 * h + 32), &u[32]);
+          tmem_wait_ld();
 #pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld32_nowait(taddr + (uint32_t)(32 * c), &u[32 * c]);
-        tmem_wait_ld();
+          for (int r = 0; r < 64; ++r) y[r] = __uint_as_float(u[r]);
+        }
+        fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tempty[region]);
+        // a large row mean sits only in the i_hi = 0 lanes: remove it there
+        if (i_hi == 0) {
+          const float c0 = y[0];
 #pragma unroll
-        for (int r = 0; r < 128; ++r) y[r] = __uint_as_float(u[r]);
+          for (int r = 0; r < 64; r += 2) sub2(y[r], y[r + 1], c0);
+        }
+        stage<0>(y);
+        stage<1>(y);
+        stage<2>(y);
+        stage<3>(y);
+        stage<4>(y);
+        stage<5>(y);
+        if (i_hi == 0) y[0] = 0.0f;  // t_0 = 0 (the mean's coefficient)
+      } else {
+        unit0 = 0;
+        row = q;
+        {
+          uint32_t u[64];
+          uint32_t c0w = 0;
+          tmem_ld32_nowait(tl + (uint32_t)(64 * h), &u[0]);
+          tmem_ld32_nowait(tl + (uint32_t)(64 * h + 32), &u[32]);
+          if (h == 1 && quarter == 0) c0w = tmem_ld1(tl);  // column 0 of lane 0 for the mean removal
+          tmem_wait_ld();
+#pragma unroll
+          for (int r = 0; r < 64; ++r) y[r] = __uint_as_float(u[r]);
+          if (m == 0) {
+            const float c0 = h == 0 ? y[0] : __uint_as_float(c0w);
+#pragma unroll
+            for (int r = 0; r < 64; r += 2) sub2(y[r], y[r + 1], c0);
+          }
+        }
+        // column bits 0..5
+        stage<0>(y);
+        stage<1>(y);
+        stage<2>(y);
+        stage<3>(y);
+        stage<4>(y);
+        stage<5>(y);
+        // Exchange through TMEM: warpgroup 0 keeps columns 0..31 and hands
+        // over 32..63; warpgroup 1 keeps 96..127 and hands over 64..95.
+        // Column 0 is never rewritten (warpgroup 1 read it above).
+        if (h == 0) {
+          uint32_t u[32];
+#pragma unroll
+          for (int r = 0; r < 32; ++r) u[r] = __float_as_uint(y[32 + r]);
+          tmem_st32(tl + 32u, u);
+        } else {
+          uint32_t u[32];
+#pragma unroll
+          for (int r = 0; r < 32; ++r) u[r] = __float_as_uint(y[r]);
+          tmem_st32(tl + 64u, u);
+        }
+        tmem_wait_st();
+        fence_before();
+        named_bar_sync(bar_pair, 256);
+        fence_after();
+        if (h == 0) {
+          uint32_t u[32];
+          tmem_ld32_nowait(tl + 64u, u);
+          tmem_wait_ld();
+#pragma unroll
+          for (int r = 0; r < 32; ++r) y[32 + r] = __uint_as_float(u[r]);
+        } else {
+          uint32_t u[32];
+          tmem_ld32_nowait(tl + 32u, u);
+          tmem_wait_ld();
+#pragma unroll
+          for (int r = 0; r < 32; ++r) y[r] = __uint_as_float(u[r]);
+        }
+        fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tempty[region]);
+        // column bit 6: y[r] = column 32h + r, y[32 + r] = column 64 + 32h + r
+#pragma unroll
+        for (int r = 0; r < 32; r += 2) bfly2(y[r], y[r + 1], y[32 + r], y[33 + r]);
+        if (m == 0 && h == 0) y[0] = 0.0f;  // t_0 = 0
       }
-      fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&tempty[acc]);
-
-      // a large row mean sits only in the i_hi = 0 lanes: remove it there
-      if (i_hi == 0) {
-        const float c0 = y[0];
-#pragma unroll
-        for (int r = 0; r < 128; r += 2) sub2(y[r], y[r + 1], c0);
-      }
-      stage128<0>(y);
-      stage128<1>(y);
-      stage128<2>(y);
-      stage128<3>(y);
-      stage128<4>(y);
-      stage128<5>(y);
-      stage128<6>(y);
-      if (i_hi == 0) y[0] = 0.0f;  // t_0 = 0 (the mean's coefficient)
 
       // LayerNorm statistics: K^2 var = sum_{i>=1} Y_i^2
-      float s0 = 0.0f, s1 = 0.0f;
-#pragma unroll
-      for (int r = 0; r < 128; r += 2) sq_acc2(s0, s1, y[r], y[r + 1]);
-      const float ss = group_reduce<KH>(s0 + s1, AddF(), slot_f, quarter, lane, bar_id);
+      const float ss = group_reduce<RT>(sum_sq64(y), AddF(), slot_ss, wq, lane, bar_row, bar_row_n);
       const float var = ss * (1.0f / ((float)K * (float)K));
       const float cmul = __fmul_rn(__fdiv_rn(1.0f, sqrtf(__fadd_rn(var, 1e-5f))), p.sK);
 #pragma unroll
-      for (int r = 0; r < 128; r += 2) mul2(y[r], y[r + 1], cmul);
+      for (int r = 0; r < 64; r += 2) mul2(y[r], y[r + 1], cmul);
 
-      const int64_t row = (int64_t)tile * (128 / KH) + r_loc;
       const bool row_ok = row < p.M;
       if constexpr (MODE == K1_T_F32) {
         if (row_ok) {
-          float4* dst = reinterpret_cast<float4*>(p.t_out + (size_t)row * K + (size_t)i_hi * 128);
+          float* trow = p.t_out + (size_t)row * K;
 #pragma unroll
-          for (int j = 0; j < 32; ++j) dst[j] = make_float4(y[4 * j], y[4 * j + 1], y[4 * j + 2], y[4 * j + 3]);
+          for (int half = 0; half < 2; ++half) {
+            // C = 64: columns 64 i_hi + 32 half + r; C = 128: 128 i_hi + 64 half + 32 h + r
+            const size_t col = PAIR ? (size_t)i_hi * 128 + 64 * half + 32 * h : (size_t)i_hi * 64 + 32 * half;
+            float4* dst = reinterpret_cast<float4*>(trow + col);
+#pragma unroll
+            for (int jj = 0; jj < 8; ++jj) {
+              const int r = 32 * half + 4 * jj;
+              dst[jj] = make_float4(y[r], y[r + 1], y[r + 2], y[r + 3]);
+            }
+          }
         }
       } else {
         q::RowParams qp;
         if constexpr (MODE == K1_Q8_I8) {
-          float g = 0.0f;
-#pragma unroll
-          for (int r = 0; r < 128; ++r) g = fmaxf(g, fabsf(y[r]));
-          qp = q::params_int8(group_reduce<KH>(g, MaxF(), slot_f, quarter, lane, bar_id));
+          qp = q::params_int8(group_reduce<RT>(max_abs64(y), MaxF(), slot_mx, wq, lane, bar_row, bar_row_n));
         } else {
-          double a0 = 0.0, a1 = 0.0;
-#pragma unroll
-          for (int r = 0; r < 128; r += 2) {
-            a0 += q::abs_f64(y[r]);
-            a1 += q::abs_f64(y[r + 1]);
-          }
-          qp = q::params_int4(group_reduce<KH>(a0 + a1, AddD(), slot_d, quarter, lane, bar_id), K);
+          // beta from a float tree sum (the quantizer-only kernel sums in
+          // double); the INT8 maximum slots are free in INT4 mode
+          qp = q::params_int4_f32(group_reduce<RT>(sum_abs64(y), AddF(), slot_mx, wq, lane, bar_row, bar_row_n), K);
         }
-        if (row_ok && i_hi == 0) p.scales[row] = qp.scale;
+        if (row_ok && i_hi == 0 && (!PAIR || h == 0)) p.scales[row] = qp.scale;
         if constexpr (MODE == K1_Q4_PACKED) {
-          // 64 bytes per thread, 16-byte chunk c at position c ^ ((m >> 1) & 3) (64B swizzle)
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            const uint4 v = codes32_s4(&y[32 * c], qp.r);
+            if constexpr (PAIR) {
+              // 64-byte rows (64B swizzle): 16-byte chunk h (c = 0) or 2 + h (c = 1)
+              const int lc = 2 * c + h;
+              *reinterpret_cast<uint4*>(stg + m * 64 + ((lc ^ ((m >> 1) & 3)) << 4)) = v;
+            } else {
+              // 32-byte rows (32B swizzle)
+              *reinterpret_cast<uint4*>(stg + m * 32 + ((c ^ ((m >> 2) & 1)) << 4)) = v;
+            }
+          }
+        } else {
+          // INT4 codes fit 16 bits when ||t|| r < 2^15 (|t_i| <= ||t||); with
+          // ||t||^2 = ss cmul^2 and a margin for the roundings
+          const bool s16 = MODE == K1_Q4_I8 && sqrtf(ss) * cmul * qp.r < 30000.0f;
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
-            uint32_t w[4];
-#pragma unroll
-            for (int h = 0; h < 4; ++h) {
-              const int r0 = 32 * c + 8 * h;
-              uint32_t mm[8];
-#pragma unroll
-              for (int u = 0; u < 8; u += 2) magic2(y[r0 + u], y[r0 + u + 1], qp.r, mm[u], mm[u + 1]);
-              int n[8];
-#pragma unroll
-              for (int u = 0; u < 8; ++u) n[u] = (int)mm[u] - q::kMagicBits;
-              w[h] = q::pack_s4x8(n);
+            const uint4 v = s16 ? codes16_i8<MODE, true>(&y[16 * c], qp.r) : codes16_i8<MODE>(&y[16 * c], qp.r);
+            if constexpr (PAIR) {
+              // 128-byte rows (128B swizzle): chunks 2h, 2h+1 (c < 2), 4 + 2h, 5 + 2h (c >= 2)
+              const int lc = (c < 2 ? 2 * h + c : 4 + 2 * h + (c - 2));
+              *reinterpret_cast<uint4*>(stg + m * 128 + ((lc ^ (m & 7)) << 4)) = v;
+            } else {
+              // 64-byte rows (64B swizzle)
+              *reinterpret_cast<uint4*>(stg + m * 64 + ((c ^ ((m >> 1) & 3)) << 4)) = v;
             }
-            *reinterpret_cast<uint4*>(stg + m * 64 + ((c ^ ((m >> 1) & 3)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
-          }
-        } else {
-          // 128 bytes per thread, 16-byte chunk c at position c ^ (m & 7) (128B swizzle)
-#pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            uint32_t w[4];
-#pragma unroll
-            for (int h = 0; h < 4; ++h) {
-              const int r0 = 16 * c + 4 * h;
-              uint32_t mm[4];
-              magic2(y[r0], y[r0 + 1], qp.r, mm[0], mm[1]);
-              magic2(y[r0 + 2], y[r0 + 3], qp.r, mm[2], mm[3]);
-              if constexpr (MODE == K1_Q4_I8) {
-#pragma unroll
-                for (int u = 0; u < 4; ++u) mm[u] = q::clip_magic_int4(mm[u]);
-              }
-              w[h] = q::gather_low_bytes(mm[0], mm[1], mm[2], mm[3]);
-            }
-            *reinterpret_cast<uint4*>(stg + m * 128 + ((c ^ (m & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
           }
         }
         fence_proxy_async_smem();
-        named_bar_sync(bar_id, 128);
+        named_bar_sync(bar_row, bar_row_n);
         if (issuer) {
-          tma_store_2d(&tmOut, stg, 0, tile * kTileChunks);
-          bulk_commit();
+          if constexpr (PAIR) {
+            tma_store_2d(&tmOut, stg, 0, q * kBoxRows);
+            bulk_commit();
+          } else if (unit0 < p.nchunk) {
+            tma_store_2d(&tmOut, stg, 0, (int)unit0);
+            bulk_commit();
+          }
         }
       }
     }
@@ -403,26 +597,31 @@ ln_fht_quant_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_con
 
 template <int LOGK, int MODE>
 cudaError_t launch_tc(const void* x, int64_t M, void* out, float* scales, int* err, cudaStream_t stream) {
-  constexpr int KH = (1 << LOGK) / 128;
+  constexpr int C = LOGK >= 14 ? 128 : 64;
+  constexpr int KH = (1 << LOGK) / C;
+  constexpr bool PAIR = C == 128;
   const int64_t nchunk = M * KH;
+  const int64_t groups = PAIR ? nchunk / kBoxRows : (nchunk + 2 * kBoxRows - 1) / (2 * kBoxRows);
+  if (groups > (int64_t)INT32_MAX / 4 || nchunk > (int64_t)INT32_MAX / 2) return cudaErrorInvalidValue;
   CUtensorMap tmX, tmOut;
-  if (!sm100_host::encode_2d(&tmX, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, 128, (uint64_t)nchunk, 256, 64, kTileChunks,
-                             CU_TENSOR_MAP_SWIZZLE_128B))
+  if (!sm100_host::encode_2d(&tmX, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, C, (uint64_t)nchunk, C * 2, kBoxCols,
+                             kBoxRows, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
   if constexpr (MODE == K1_Q4_PACKED) {
-    if (!sm100_host::encode_2d(&tmOut, CU_TENSOR_MAP_DATA_TYPE_UINT8, out, 64, (uint64_t)nchunk, 64, 64, kTileChunks,
-                               CU_TENSOR_MAP_SWIZZLE_64B))
+    if (!sm100_host::encode_2d(&tmOut, CU_TENSOR_MAP_DATA_TYPE_UINT8, out, C / 2, (uint64_t)nchunk, C / 2, C / 2,
+                               kBoxRows, PAIR ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B))
       return cudaErrorInvalidValue;
   } else if constexpr (MODE == K1_Q4_I8 || MODE == K1_Q8_I8) {
-    if (!sm100_host::encode_2d(&tmOut, CU_TENSOR_MAP_DATA_TYPE_UINT8, out, 128, (uint64_t)nchunk, 128, 128,
-                               kTileChunks, CU_TENSOR_MAP_SWIZZLE_128B))
+    if (!sm100_host::encode_2d(&tmOut, CU_TENSOR_MAP_DATA_TYPE_UINT8, out, C, (uint64_t)nchunk, C, C, kBoxRows,
+                               PAIR ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B))
       return cudaErrorInvalidValue;
   } else {
     tmOut = tmX;  // unused
   }
   TcParams p;
   p.M = M;
-  p.num_tiles = (int)((nchunk + kTileChunks - 1) / kTileChunks);
+  p.nchunk = nchunk;
+  p.num_groups = (int)groups;
   p.sK = (float)(1.0 / sqrt((double)(1 << LOGK)));
   p.t_out = reinterpret_cast<float*>(out);
   p.scales = scales;
@@ -439,7 +638,7 @@ cudaError_t launch_tc(const void* x, int64_t M, void* out, float* scales, int* e
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
   if (e != cudaSuccess) return e;
   const int nsm = sm100_host::sm_count();
-  const int grid = p.num_tiles < nsm ? p.num_tiles : nsm;
+  const int grid = p.num_groups < nsm ? p.num_groups : nsm;
   kern<<<grid, kThreads, kSmemBytes, stream>>>(tmX, tmOut, p);
   return cudaGetLastError();
 }

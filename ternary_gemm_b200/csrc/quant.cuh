@@ -43,6 +43,18 @@ __device__ __forceinline__ RowParams params_int4(double abs_sum, int64_t K) {
   return p;
 }
 
+// beta from a float sum of |t| over K elements (K a power of two, so the
+// division is exact).  Used by the fused tensor-core kernel, whose sum is a
+// float tree (relative error at most ~15 float units in the last place);
+// the quantizer-only kernel keeps the double sum above.
+__device__ __forceinline__ RowParams params_int4_f32(float abs_sum, int64_t K) {
+  const float beta = abs_sum * (1.0f / (float)K);
+  RowParams p;
+  p.r = __fdiv_rn(kSqrt7, __fadd_rn(beta, kEps));
+  p.scale = __fdiv_rn(beta, kSqrt7);
+  return p;
+}
+
 // gamma = max |t| (exact, order free).
 __device__ __forceinline__ RowParams params_int8(float gamma) {
   RowParams p;
@@ -87,6 +99,17 @@ __device__ __forceinline__ int clip_int4(int n) { return max(-8, min(7, n)); }
 // the bits clips the code, and the low byte is the code as an int8.
 __device__ __forceinline__ uint32_t clip_magic_int4(uint32_t m) {
   return (uint32_t)max(kMagicBits - 8, min(kMagicBits + 7, (int)m));
+}
+
+// Two codes from the magic-FMA bits of a pair, clipped to the INT4 range,
+// as two int16 halves (lo in the low half).  The low 16 bits of the bits are
+// the code itself (kMagicBits has zero low halves), so this is exact when
+// every |code| < 2^15, which the caller guarantees per row.
+__device__ __forceinline__ uint32_t clip_pair_int4_s16(uint32_t m_lo, uint32_t m_hi) {
+  uint32_t v = __byte_perm(m_lo, m_hi, 0x5410);
+  asm("max.s16x2 %0, %0, %1;" : "+r"(v) : "r"(0xFFF8FFF8u));
+  asm("min.s16x2 %0, %0, %1;" : "+r"(v) : "r"(0x00070007u));
+  return v;
 }
 
 // Low bytes of four words -> one word, a in the lowest byte.

@@ -64,6 +64,24 @@ def check_codes_near(q_gpu, q_orc, t_orc32, scale_orc, bits, min_agree=0.9999, h
     return agree
 
 
+# The fused tensor-core kernel (bf16 input, K in [128, 16384]) takes the INT4
+# absmean beta from a float tree sum of depth <= 22 (10 levels inside a thread,
+# 5 shuffle levels, 7 slot additions), so beta is within 22 units in the last
+# place (1.3e-6) of the double sum; r = sqrt(7)/(beta+eps) moves as much.  A
+# code can then change only where the exact t*r (|t*r| <= 8.5 for unclipped
+# codes) lies within 8.5 * 1.3e-6 = 1.1e-5 of a half-integer.
+FUSED_BETA_REL = 2e-6
+FUSED_HALF_TOL = 2e-5
+
+
+def check_fused_int4(q_gpu, scales_gpu, q_orc, scales_orc, t32):
+    """Fused INT4 codes and scales against the oracle's quantizer on the same t."""
+    s = np.asarray(scales_gpu, np.float64)
+    so = np.asarray(scales_orc, np.float64)
+    assert np.all(np.abs(s - so) <= FUSED_BETA_REL * np.abs(so)), np.max(np.abs(s - so) / np.maximum(so, 1e-30))
+    return check_codes_near(q_gpu, q_orc, t32, scales_orc, 4, min_agree=0.9999, half_tol=FUSED_HALF_TOL)
+
+
 def rel_fro(a, b):
     a = np.asarray(a, np.float64)
     b = np.asarray(b, np.float64)

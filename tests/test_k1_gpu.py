@@ -10,7 +10,7 @@ Tolerances (stated by the path's definition):
 import numpy as np
 import pytest
 
-from helpers import check_codes_near, check_t, to_device, to_host, unpack_nibbles
+from helpers import check_fused_int4, check_codes_near, check_t, to_device, to_host, unpack_nibbles
 from ternary_gemm_b200.inputs import WORKLOADS, f32_to_bf16_bits, make_x, make_x_rows, sample_rows
 
 pytestmark = pytest.mark.gpu
@@ -116,15 +116,20 @@ def test_quant_hook_any_length(H, orc, K, bits):
 @pytest.mark.parametrize("bits", [4, 8])
 @pytest.mark.parametrize("K", KS)
 def test_fused_equals_quant_of_hook_t(H, orc, K, bits):
-    """The fused kernel's codes are exactly the quantizer applied to its own t."""
+    """The fused kernel quantizes its own t: bit for bit, except INT4 on the
+    tensor-core kernel (bf16, K in [128, 16384]), whose absmean is a float
+    sum (scales within 2e-6, codes off by one only at rounding boundaries)."""
     x = x_for(K, "bf16")
     xd = to_device(x)
     t = to_host(H.hbl_debug_ln_fht(xd))
     codes, scales = H.hbl_fht_quant(xd, bits)
     q = unpack_nibbles(to_host(codes), K) if bits == 4 else to_host(codes)
     qo, so = orc.quant(t, bits)
-    assert np.array_equal(q, qo)
-    assert np.array_equal(to_host(scales), so)
+    if bits == 4 and 128 <= K <= 16384:
+        check_fused_int4(q, to_host(scales), qo, so, t)
+    else:
+        assert np.array_equal(q, qo)
+        assert np.array_equal(to_host(scales), so)
 
 
 @pytest.mark.parametrize("bits", [4, 8])

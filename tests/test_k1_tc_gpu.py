@@ -1,17 +1,19 @@
 """GPU parity of the tensor-core split of the fused LN -> Hadamard -> quantize
 kernel (bf16 input, K in [128, 16384]): the high Hadamard factor as a tcgen05
-MMA, the low 7 stages in registers.
+MMA, the low 6 stages (7 at K = 16384) in registers.
 
 The shapes here run many tiles per CTA (every shared-memory stage and TMEM
 accumulator is reused several times) with a ragged last tile, and the inputs
 include bf16 rows whose mean is far above their spread.  Tolerances are the
-fused kernel's: t within 1e-5 relative of the oracle; codes and scales
-bit-exact against the oracle's quantizer applied to the kernel's own t.
+fused kernel's: t within 1e-5 relative of the oracle; INT8 codes and scales
+bit-exact against the oracle's quantizer applied to the kernel's own t; INT4
+scales within 2e-6 relative of it (the kernel sums |t| in float) and codes
+equal except off by one where t*r is within 2e-5 of a rounding boundary.
 """
 import numpy as np
 import pytest
 
-from helpers import check_t, to_device, to_host, unpack_nibbles
+from helpers import check_fused_int4, check_t, to_device, to_host, unpack_nibbles
 from ternary_gemm_b200.inputs import WORKLOADS, f32_to_bf16_bits, make_x, make_x_rows, sample_rows
 
 pytestmark = pytest.mark.gpu
@@ -29,11 +31,14 @@ def H():
     return hbl
 
 
-def many_tile_rows(K, tiles_per_cta=9, extra_chunks=3):
-    """Rows giving tiles_per_cta tiles per CTA on a full GPU plus a ragged tile."""
-    kh = K // 128
-    chunks = 128 * SMS * tiles_per_cta + extra_chunks * kh
-    return chunks // kh
+def many_tile_rows(K, groups_per_cta=9, extra_rows=3):
+    """Rows giving about groups_per_cta MMA groups (256 chunk rows of 64
+    columns, or 128 of 128 at K = 16384) per CTA on a full GPU, plus a ragged
+    last group."""
+    chunk = 128 if K >= 16384 else 64
+    group_chunks = 128 if K >= 16384 else 256
+    kh = K // chunk
+    return (group_chunks * SMS * groups_per_cta) // kh + extra_rows
 
 
 @pytest.mark.parametrize("K", [128, 2048, 16384])
@@ -46,16 +51,19 @@ def test_tc_many_tiles(H, orc, K):
     rows = sample_rows(M, 24)
     check_t(t[rows], orc.ln_fht(make_x_rows(wl, rows))[0])
     # codes and scales: the oracle's quantizer on the kernel's own t, every row
-    for bits in (4, 8):
-        qo, so = orc.quant(t, bits)
-        codes, scales = H.hbl_fht_quant(xd, bits)
-        q = unpack_nibbles(to_host(codes), K) if bits == 4 else to_host(codes)
-        assert np.array_equal(q, qo)
-        assert np.array_equal(to_host(scales), so)
-    codes_i8, scales_i8 = H.hbl_fht_quant_i8(xd, 4)
+    qo, so = orc.quant(t, 8)
+    codes, scales = H.hbl_fht_quant(xd, 8)
+    assert np.array_equal(to_host(codes), qo)
+    assert np.array_equal(to_host(scales), so)
     qo, so = orc.quant(t, 4)
-    assert np.array_equal(to_host(codes_i8), qo)
-    assert np.array_equal(to_host(scales_i8), so)
+    codes, scales = H.hbl_fht_quant(xd, 4)
+    q4 = unpack_nibbles(to_host(codes), K)
+    s4 = to_host(scales)
+    check_fused_int4(q4, s4, qo, so, t)
+    # the int8-widened INT4 codes are the packed ones, byte for byte
+    codes_i8, scales_i8 = H.hbl_fht_quant_i8(xd, 4)
+    assert np.array_equal(to_host(codes_i8), q4)
+    assert np.array_equal(to_host(scales_i8), s4)
 
 
 @pytest.mark.parametrize("K", [128, 256, 4096, 16384])
@@ -86,7 +94,10 @@ def test_tc_constant_and_zero_rows_bf16(H, orc, K, bits):
     t = to_host(H.hbl_debug_ln_fht(to_device(xb)))
     check_t(t, t64)
     qo, so = orc.quant(t, bits)
-    assert np.array_equal(q, qo) and np.array_equal(s, so)
+    if bits == 8:
+        assert np.array_equal(q, qo) and np.array_equal(s, so)
+    else:
+        check_fused_int4(q, s, qo, so, t)
 
 
 def test_tc_single_row_and_partial_tile(H, orc):
@@ -99,5 +110,4 @@ def test_tc_single_row_and_partial_tile(H, orc):
         check_t(t, orc.ln_fht(x)[0])
         codes, scales = H.hbl_fht_quant(xd, 4)
         qo, so = orc.quant(t, 4)
-        assert np.array_equal(unpack_nibbles(to_host(codes), K), qo)
-        assert np.array_equal(to_host(scales), so)
+        check_fused_int4(unpack_nibbles(to_host(codes), K), to_host(scales), qo, so, t)
