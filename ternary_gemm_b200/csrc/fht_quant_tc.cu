@@ -52,15 +52,22 @@
 //   warps 2-3  idle (registers are granted to whole warpgroups);
 //   warps 4-19 four epilogue warpgroups in two pairs; pair p takes every
 //              other group: TMEM -> registers, butterflies, LayerNorm
-//              statistics, quantizer, codes into a swizzled staging tile that
-//              a TMA store writes out.
+//              statistics, quantizer, codes stored straight to global memory
+//              (each warp writes whole consecutive chunk rows).
 // Row statistics reduce over the threads of a token row: warp shuffles, then
-// per-warp slots behind a named barrier of the row's warpgroup (pair).  The
-// INT4 absmean is summed in float (trees of depth <= 22, so beta is within
-// 1.3e-6 relative of a double sum; a double per-element sum cost about a
-// fifth of the kernel's time), INT8 absmax is exact.  INT4 codes widened to
-// int8 are clipped on packed 16-bit halves when the row bound ||t|| r keeps
-// every code below 2^15, else on 32-bit values.
+// per-warp slots behind a named barrier of the row's warpgroup (pair), one
+// round for both statistics: sum Y^2, and sum |y| (INT4) or max |y| (INT8)
+// of the transformed but unscaled y, since t = cmul y.  INT8 then stays
+// exact: gamma = fl(cmul max|y|) = max|t| (rounding is monotone) and the
+// codes are rint(fl(cmul y) r).  INT4 takes beta = fl(cmul sum|y|) / K with
+// the sum in float (trees of depth <= 22) and codes rint(y fl(cmul r)): beta
+// within ~24 units in the last place (1.5e-6) of the double sum over t, and
+// y fl(cmul r) within 2 units of t r, so a code can differ from the
+// quantizer-on-t value only where t r is within ~1.5e-5 of a half-integer
+// (a double per-element sum and a second reduction round cost about a
+// quarter of the kernel's time).  INT4 codes widened to int8 are clipped on
+// packed 16-bit halves when the row bound ||t|| r keeps every code below
+// 2^15, else on 32-bit values.
 // The block is launched with at most 96 registers per thread and rebalanced
 // with setmaxnreg: the first warpgroup gives its share down to 40, the
 // epilogue warpgroups take 104 each (the host checks that the launch count
@@ -85,7 +92,6 @@ constexpr int kBoxRows = 128;                        // chunk rows per box (MMA 
 constexpr int kBoxBytes = kBoxRows * kBoxCols * 2;   // 16 KB
 constexpr int kSlots = 4;                            // ring slots of two boxes (one group)
 constexpr int kSlotBytes = 2 * kBoxBytes;
-constexpr int kStageOutBytes = kBoxRows * kBoxCols;  // int8 codes of a box (the largest staged form)
 constexpr int kEpiGroups = 4;                        // epilogue warpgroups
 constexpr int kThreads = 128 + 128 * kEpiGroups;
 constexpr int kCtrlRegs = 40;  // registers per thread of the first warpgroup after setmaxnreg
@@ -93,7 +99,7 @@ constexpr int kEpiRegs = 104;  // registers per thread of an epilogue warpgroup 
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kAcol = 448;  // TMEM column of A (64 columns: 128 bf16 per lane)
 constexpr int kRegions = 3;      // 128-column accumulators below kAcol
-constexpr size_t kSmemBytes = 1024 + (size_t)kSlots * kSlotBytes + (size_t)kEpiGroups * kStageOutBytes + 1024;
+constexpr size_t kSmemBytes = 1024 + (size_t)kSlots * kSlotBytes + 1024;
 
 // instruction descriptor, kind::f16: D f32, A and B bf16, A K-major, B
 // MN-major, N = 128, M = 128
@@ -105,6 +111,8 @@ struct TcParams {
   int num_groups;    // MMA groups
   float sK;          // 1 / sqrt(K) rounded to float
   float* t_out;      // K1_T_F32: t [M][K]
+  uint8_t* codes;    // quantizing modes: codes [M][K/2] (packed) or [M][K] (int8)
+  int codes_al32;    // codes 32-byte aligned (256-bit stores allowed)
   float* scales;     // [M]
   int* err;          // device error word
 };
@@ -116,6 +124,13 @@ __device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, ui
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
       "r"(a_tmem), "l"(b), "r"(kIdesc), "r"(accumulate));
+}
+
+// 32 bytes to global memory in one 256-bit store (p 32-byte aligned)
+__device__ __forceinline__ void st_global_32B(void* p, const uint4& a, const uint4& b) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(a.x), "r"(a.y), "r"(a.z),
+               "r"(a.w), "r"(b.x), "r"(b.y), "r"(b.z), "r"(b.w)
+               : "memory");
 }
 
 // one TMEM column of this warp's lane quarter
@@ -142,15 +157,21 @@ __device__ __forceinline__ void stage(float (&e)[N]) {
   }
 }
 
-// All-reduce over the RT threads of one token row: RT consecutive lanes when
-// RT <= 32, else RT / 32 whole warps numbered wq (their slots) inside the
-// barrier's `bar_n` threads.  Every thread of the row ends with the identical
-// value.  Each reduction of a group uses its own `slots`.
-template <int RT, typename V, typename Op>
-__device__ __forceinline__ V group_reduce(V v, Op op, V* slots, int wq, int lane, int bar_id, int bar_n) {
+// All-reduce of a pair of values over the RT threads of one token row, in
+// one round: .x summed, .y summed or, with MAXY, maximized.  RT consecutive
+// lanes when RT <= 32, else RT / 32 whole warps numbered wq (their slots)
+// inside the barrier's `bar_n` threads.  Every thread of the row ends with
+// the identical pair.
+template <int RT, bool MAXY>
+__device__ __forceinline__ float2 group_reduce2(float2 v, float2* slots, int wq, int lane, int bar_id, int bar_n) {
   constexpr int W = RT < 32 ? RT : 32;
 #pragma unroll
-  for (int o = W / 2; o >= 1; o >>= 1) v = op(v, __shfl_xor_sync(0xffffffffu, v, o));
+  for (int o = W / 2; o >= 1; o >>= 1) {
+    const float a = __shfl_xor_sync(0xffffffffu, v.x, o);
+    const float b = __shfl_xor_sync(0xffffffffu, v.y, o);
+    v.x += a;
+    v.y = MAXY ? fmaxf(v.y, b) : v.y + b;
+  }
   if constexpr (RT > 32) {
     constexpr int NW = RT / 32;
     if (lane == 0) slots[wq] = v;
@@ -158,7 +179,11 @@ __device__ __forceinline__ V group_reduce(V v, Op op, V* slots, int wq, int lane
     const int w0 = wq & ~(NW - 1);
     v = slots[w0];
 #pragma unroll
-    for (int i = 1; i < NW; ++i) v = op(v, slots[w0 + i]);
+    for (int i = 1; i < NW; ++i) {
+      const float2 u = slots[w0 + i];
+      v.x += u.x;
+      v.y = MAXY ? fmaxf(v.y, u.y) : v.y + u.y;
+    }
   }
   return v;
 }
@@ -271,8 +296,7 @@ __device__ __forceinline__ uint4 codes32_s4(const float* y, float r) {
 
 template <int LOGK, int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
-ln_fht_quant_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmOut,
-                       TcParams p) {
+ln_fht_quant_tc_kernel(const __grid_constant__ CUtensorMap tmX, TcParams p) {
   constexpr int K = 1 << LOGK;
   constexpr int C = LOGK >= 14 ? 128 : 64;  // chunk width
   constexpr int KH = K / C;                 // chunk rows per token row
@@ -281,14 +305,13 @@ ln_fht_quant_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_con
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   uint8_t* sB = base;
-  uint8_t* sOut = sB + kSlots * kSlotBytes;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sOut + kEpiGroups * kStageOutBytes);
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + kSlots * kSlotBytes);
   uint64_t* empty = full + kSlots;
   uint64_t* tfull = empty + kSlots;
   uint64_t* tempty = tfull + kRegions;
   uint64_t* drain = tempty + kRegions;
-  float* red_f = reinterpret_cast<float*>(drain + 1);    // [pair][16]: squares; |t| sums or maxima
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(red_f + 32);
+  float2* red2 = reinterpret_cast<float2*>(drain + 1);   // [pair][8]: (sum of squares, |y| sum or max)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(red2 + 16);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -395,18 +418,12 @@ ln_fht_quant_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_con
     const int bar_row = PAIR ? bar_pair : bar_wg;
     const int bar_row_n = PAIR ? 256 : 128;
     const int wq = PAIR ? 4 * h + quarter : quarter;  // warp number among the row's warps
-    const bool issuer = quarter == 0 && lane == 0 && (!PAIR || h == 0);
-    // PAIR: the pair's two staging buffers form one 16 KB tile
-    uint8_t* stg = sOut + (PAIR ? pr * 2 : g) * kStageOutBytes;
-    float* slot_ss = red_f + 16 * pr + (PAIR ? 0 : 4 * h);
-    float* slot_mx = slot_ss + 8;
+    float2* slot2 = red2 + 8 * pr + (PAIR ? 0 : 4 * h);
     const int i_hi = PAIR ? m : m % KH;
     for (int j = pr;; j += 2) {
       const int q = blockIdx.x + j * gridDim.x;
       if (q >= p.num_groups) break;
       const int region = j % kRegions;
-      // the previous TMA store of this staging tile has finished reading it
-      if (issuer) bulk_wait_read_all();
       int ok = 1;
       if (lane == 0) ok = wait_bounded(&tfull[region], (uint32_t)(j / kRegions) & 1u, abort_flag, p.err) ? 1 : 0;
       ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -510,15 +527,25 @@ ln_fht_quant_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_con
         if (m == 0 && h == 0) y[0] = 0.0f;  // t_0 = 0
       }
 
-      // LayerNorm statistics: K^2 var = sum_{i>=1} Y_i^2
-      const float ss = group_reduce<RT>(sum_sq64(y), AddF(), slot_ss, wq, lane, bar_row, bar_row_n);
+      // Row statistics in one reduction round: K^2 var = sum_{i>=1} Y_i^2,
+      // and the quantizer's statistic of y (t = cmul y): sum |y| for INT4
+      // (sum |t| = cmul sum |y| up to the roundings of t), max |y| for INT8
+      // (max |t| = fl(cmul max |y|) exactly, rounding being monotone).
+      float stat_part = 0.0f;
+      if constexpr (MODE == K1_Q8_I8) stat_part = max_abs64(y);
+      if constexpr (MODE == K1_Q4_PACKED || MODE == K1_Q4_I8) stat_part = sum_abs64(y);
+      const float2 red = group_reduce2<RT, MODE == K1_Q8_I8>(make_float2(sum_sq64(y), stat_part), slot2, wq, lane,
+                                                              bar_row, bar_row_n);
+      const float ss = red.x;
       const float var = ss * (1.0f / ((float)K * (float)K));
       const float cmul = __fmul_rn(__fdiv_rn(1.0f, sqrtf(__fadd_rn(var, 1e-5f))), p.sK);
-#pragma unroll
-      for (int r = 0; r < 64; r += 2) mul2(y[r], y[r + 1], cmul);
-
       const bool row_ok = row < p.M;
+      // this thread's chunk row: C = 64, unit row m; C = 128, tile row m
+      const int64_t crow = (PAIR ? (int64_t)q * kBoxRows : unit0) + m;
+
       if constexpr (MODE == K1_T_F32) {
+#pragma unroll
+        for (int r = 0; r < 64; r += 2) mul2(y[r], y[r + 1], cmul);
         if (row_ok) {
           float* trow = p.t_out + (size_t)row * K;
 #pragma unroll
@@ -535,58 +562,53 @@ ln_fht_quant_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_con
         }
       } else {
         q::RowParams qp;
+        float cq;  // multiplier from y to the value rounded to a code
         if constexpr (MODE == K1_Q8_I8) {
-          qp = q::params_int8(group_reduce<RT>(max_abs64(y), MaxF(), slot_mx, wq, lane, bar_row, bar_row_n));
+          qp = q::params_int8(__fmul_rn(cmul, red.y));
+          // INT8 keeps the exact order: t = fl(cmul y), then rint(t r)
+#pragma unroll
+          for (int r = 0; r < 64; r += 2) mul2(y[r], y[r + 1], cmul);
+          cq = qp.r;
         } else {
-          // beta from a float tree sum (the quantizer-only kernel sums in
-          // double); the INT8 maximum slots are free in INT4 mode
-          qp = q::params_int4_f32(group_reduce<RT>(sum_abs64(y), AddF(), slot_mx, wq, lane, bar_row, bar_row_n), K);
+          // INT4: beta from cmul sum|y| (float), codes rint(y * fl(cmul r))
+          qp = q::params_int4_f32(__fmul_rn(cmul, red.y), K);
+          cq = __fmul_rn(cmul, qp.r);
         }
         if (row_ok && i_hi == 0 && (!PAIR || h == 0)) p.scales[row] = qp.scale;
-        if constexpr (MODE == K1_Q4_PACKED) {
+        if (row_ok) {
+          uint8_t* crow_out = p.codes + crow * (MODE == K1_Q4_PACKED ? C / 2 : C);
+          if constexpr (MODE == K1_Q4_PACKED) {
+            // 32 codes (16 bytes) per half: C = 64 at bytes 0 and 16 of the
+            // 32-byte chunk row; C = 128 at 16h and 32 + 16h of 64 bytes
+            uint4* d0 = reinterpret_cast<uint4*>(crow_out + (PAIR ? 16 * h : 0));
+            uint4* d1 = reinterpret_cast<uint4*>(crow_out + (PAIR ? 32 + 16 * h : 16));
+            *d0 = codes32_s4(&y[0], cq);
+            *d1 = codes32_s4(&y[32], cq);
+          } else {
+            // 16 codes per 16 bytes: C = 64 at 0, 16, 32, 48; C = 128 at
+            // 32h, 32h + 16, 64 + 32h, 80 + 32h
+            const bool s16 = MODE == K1_Q4_I8 && sqrtf(ss) * cq < 30000.0f;
+            if (PAIR && p.codes_al32) {
+              // two whole 32-byte sectors per thread, not four half sectors
 #pragma unroll
-          for (int c = 0; c < 2; ++c) {
-            const uint4 v = codes32_s4(&y[32 * c], qp.r);
-            if constexpr (PAIR) {
-              // 64-byte rows (64B swizzle): 16-byte chunk h (c = 0) or 2 + h (c = 1)
-              const int lc = 2 * c + h;
-              *reinterpret_cast<uint4*>(stg + m * 64 + ((lc ^ ((m >> 1) & 3)) << 4)) = v;
+              for (int c = 0; c < 4; c += 2) {
+                const uint4 v0 = s16 ? codes16_i8<MODE, true>(&y[16 * c], cq) : codes16_i8<MODE>(&y[16 * c], cq);
+                const uint4 v1 =
+                    s16 ? codes16_i8<MODE, true>(&y[16 * c + 16], cq) : codes16_i8<MODE>(&y[16 * c + 16], cq);
+                st_global_32B(crow_out + (c == 0 ? 32 * h : 64 + 32 * h), v0, v1);
+              }
             } else {
-              // 32-byte rows (32B swizzle)
-              *reinterpret_cast<uint4*>(stg + m * 32 + ((c ^ ((m >> 2) & 1)) << 4)) = v;
-            }
-          }
-        } else {
-          // INT4 codes fit 16 bits when ||t|| r < 2^15 (|t_i| <= ||t||); with
-          // ||t||^2 = ss cmul^2 and a margin for the roundings
-          const bool s16 = MODE == K1_Q4_I8 && sqrtf(ss) * cmul * qp.r < 30000.0f;
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            const uint4 v = s16 ? codes16_i8<MODE, true>(&y[16 * c], qp.r) : codes16_i8<MODE>(&y[16 * c], qp.r);
-            if constexpr (PAIR) {
-              // 128-byte rows (128B swizzle): chunks 2h, 2h+1 (c < 2), 4 + 2h, 5 + 2h (c >= 2)
-              const int lc = (c < 2 ? 2 * h + c : 4 + 2 * h + (c - 2));
-              *reinterpret_cast<uint4*>(stg + m * 128 + ((lc ^ (m & 7)) << 4)) = v;
-            } else {
-              // 64-byte rows (64B swizzle)
-              *reinterpret_cast<uint4*>(stg + m * 64 + ((c ^ ((m >> 1) & 3)) << 4)) = v;
+              for (int c = 0; c < 4; ++c) {
+                const int off = PAIR ? (c < 2 ? 32 * h + 16 * c : 64 + 32 * h + 16 * (c - 2)) : 16 * c;
+                const uint4 v = s16 ? codes16_i8<MODE, true>(&y[16 * c], cq) : codes16_i8<MODE>(&y[16 * c], cq);
+                *reinterpret_cast<uint4*>(crow_out + off) = v;
+              }
             }
-          }
-        }
-        fence_proxy_async_smem();
-        named_bar_sync(bar_row, bar_row_n);
-        if (issuer) {
-          if constexpr (PAIR) {
-            tma_store_2d(&tmOut, stg, 0, q * kBoxRows);
-            bulk_commit();
-          } else if (unit0 < p.nchunk) {
-            tma_store_2d(&tmOut, stg, 0, (int)unit0);
-            bulk_commit();
           }
         }
       }
     }
-    if (issuer) bulk_wait_all();
   }
 
   fence_before();
@@ -603,27 +625,18 @@ cudaError_t launch_tc(const void* x, int64_t M, void* out, float* scales, int* e
   const int64_t nchunk = M * KH;
   const int64_t groups = PAIR ? nchunk / kBoxRows : (nchunk + 2 * kBoxRows - 1) / (2 * kBoxRows);
   if (groups > (int64_t)INT32_MAX / 4 || nchunk > (int64_t)INT32_MAX / 2) return cudaErrorInvalidValue;
-  CUtensorMap tmX, tmOut;
+  CUtensorMap tmX;
   if (!sm100_host::encode_2d(&tmX, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, C, (uint64_t)nchunk, C * 2, kBoxCols,
                              kBoxRows, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
-  if constexpr (MODE == K1_Q4_PACKED) {
-    if (!sm100_host::encode_2d(&tmOut, CU_TENSOR_MAP_DATA_TYPE_UINT8, out, C / 2, (uint64_t)nchunk, C / 2, C / 2,
-                               kBoxRows, PAIR ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B))
-      return cudaErrorInvalidValue;
-  } else if constexpr (MODE == K1_Q4_I8 || MODE == K1_Q8_I8) {
-    if (!sm100_host::encode_2d(&tmOut, CU_TENSOR_MAP_DATA_TYPE_UINT8, out, C, (uint64_t)nchunk, C, C, kBoxRows,
-                               PAIR ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B))
-      return cudaErrorInvalidValue;
-  } else {
-    tmOut = tmX;  // unused
-  }
   TcParams p;
   p.M = M;
   p.nchunk = nchunk;
   p.num_groups = (int)groups;
   p.sK = (float)(1.0 / sqrt((double)(1 << LOGK)));
   p.t_out = reinterpret_cast<float*>(out);
+  p.codes = reinterpret_cast<uint8_t*>(out);
+  p.codes_al32 = (reinterpret_cast<uintptr_t>(out) & 31u) == 0;
   p.scales = scales;
   p.err = err;
   auto kern = ln_fht_quant_tc_kernel<LOGK, MODE>;
@@ -639,7 +652,7 @@ cudaError_t launch_tc(const void* x, int64_t M, void* out, float* scales, int* e
   if (e != cudaSuccess) return e;
   const int nsm = sm100_host::sm_count();
   const int grid = p.num_groups < nsm ? p.num_groups : nsm;
-  kern<<<grid, kThreads, kSmemBytes, stream>>>(tmX, tmOut, p);
+  kern<<<grid, kThreads, kSmemBytes, stream>>>(tmX, p);
   return cudaGetLastError();
 }
 
