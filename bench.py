@@ -341,14 +341,15 @@ def bench_ours(args):
     achieved_tops = ops / t_gm / 1e12
     k1_bytes = M * K * (2 if wl.dtype == "bf16" else 4) + M * K + 4 * M
     k1_gbs = k1_bytes / t_k1 / 1e9
-    roofline = {"bound": "tensor", "kernel": "gemm_i8_kernel (tcgen05 kind::i8 + dequant epilogue)",
+    roofline = {"bound": "tensor", "kernel": "gemm_i8_2sm_kernel (tcgen05 kind::i8, cta_group::2, dequant epilogue)",
                 "achieved": achieved_tops, "peak": int8_peak, "unit": "TFLOP/s", "frac": achieved_tops / int8_peak,
                 "traffic": measured_traffic("gemm_7b_wdown"),
                 "peak_source": "%s bf16 burst %.1f TFLOP/s x %.0f (nominal int8/bf16 dense ratio)"
                                % (peak_kind, peaks["bf16_tflops"], INT8_OVER_BF16),
                 "algorithmic_ops_per_launch": ops, "launch_ms": t_gm * 1e3,
                 "frac_of_nominal_4500": achieved_tops / 4500.0}
-    k1 = {"bound": "hbm", "kernel": "ln_fht_quant_kernel (INT%d, int8 codes out)" % bits, "achieved": k1_gbs,
+    k1 = {"bound": "hbm", "kernel": "ln_fht_quant_tc_kernel (tcgen05 high Hadamard factor; INT%d, int8 codes out)"
+          % bits, "achieved": k1_gbs,
           "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": k1_gbs / peaks["hbm_gbs"],
           "traffic": measured_traffic("k1_7b_wdown"),
           "algorithmic_bytes_per_launch": k1_bytes, "launch_ms": t_k1 * 1e3}
@@ -403,155 +404,6 @@ def bench_ours(args):
                "h2d_bytes_per_step": x.numel() * x.element_size(),
                "d2h_bytes_per_step": y.numel() * y.element_size(), "ms_per_step": e2e_ms,
                "pipeline": "%d row chunks, upload / hbl_forward / download on three streams" % chunks}
-
-    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": int(os.environ.get("WORLD_SIZE", "1")),
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3 / args.steps,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
-            "impl": "reference",
-            "config": {"workload": wl.name, "M": wl.M, "K": wl.K, "N": wl.N, "bits": args.bits,
-                       "x_dtype": wl.dtype, "parallelism": "replicas"},
-            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": sample},
-            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
-    print(json.dumps(line), flush=True)
-    return 0
-
-
-# ------------------------------------------------------------------ ours
-
-def _to_device(a):
-    import numpy as np
-    import torch
-    if a.dtype == np.uint16:
-        return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).cuda()
-    return torch.from_numpy(a).cuda()
-
-
-def bench_ours(args):
-    import numpy as np
-    import torch
-    from ternary_gemm_b200 import build as hbl_build
-    hbl_build.build()
-    import ternary_gemm_b200 as hbl
-    from ternary_gemm_b200.inputs import WORKLOADS, make_w, make_x
-
-    ranks = Ranks("nccl")
-    torch.cuda.set_device(ranks.local)
-    dev = torch.device("cuda", ranks.local)
-    wl = WORKLOADS[args.workload]
-    M, K, N, bits = wl.M, wl.K, wl.N, args.bits
-    peaks, peak_kind = load_peaks()
-
-    # CPU baseline first, before any GPU work in this process (rank 0, N = 1 only)
-    cpu = None
-    if ranks.rank == 0 and ranks.world == 1 and not args.no_cpu_baseline:
-        v, n, dt = oracle_rows_per_second(wl, bits, args.cpu_seconds)
-        cpu = {"value": v, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-               "sample": "%d rows of %s (K=%d, N=%d, INT%d) through LN+FHT+quant+GEMM+dequant, single-threaded C "
-                         "oracle, %.1f s" % (n, wl.name, K, N, bits, dt)}
-
-    x = _to_device(make_x(wl))
-    W = _to_device(make_w(wl))
-    stream = torch.cuda.current_stream()
-    packed, alpha = hbl.hbl_pack_ternary(W)
-    del W
-    y = torch.empty((M, N), dtype=x.dtype, device=dev)
-    ws = torch.empty((hbl.hbl_forward_workspace_bytes(M, K, N, bits),), dtype=torch.uint8, device=dev)
-
-    def step():
-        hbl.hbl_forward(x, packed, alpha, N, bits, y=y, workspace=ws)
-
-    gpu_uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
-    clocks = ClockSampler(gpu_uuid)
-    clocks.start()
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize()
-
-    # -------- headline: K whole forwards
-    ranks.barrier()
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.steps):
-        step()
-    e1.record(stream)
-    e1.synchronize()
-    ranks.barrier()
-    torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1) / args.steps
-    ms_max = ranks.max(ms, dev)
-    value = aggregate_value(M, ranks.world, ms_max / 1e3)
-
-    # -------- per-kernel times through the stage entry points (same kernels as hbl_forward)
-    A = torch.empty((M, K), dtype=torch.int8, device=dev)
-    sc = torch.empty((M,), dtype=torch.float32, device=dev)
-    Wi = torch.empty((N, K), dtype=torch.int8, device=dev)
-    nst = max(20, min(args.steps, 200))
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(nst)]
-    for _ in range(3):
-        hbl.hbl_fht_quant_i8(x, bits, codes=A, scales=sc)
-        hbl.hbl_widen_ternary(packed, K, w=Wi)
-        hbl.hbl_gemm_dequant(A, Wi, sc, alpha, y=y)
-    torch.cuda.synchronize()
-    for i in range(nst):
-        evs[i][0].record(stream)
-        hbl.hbl_fht_quant_i8(x, bits, codes=A, scales=sc)
-        evs[i][1].record(stream)
-        hbl.hbl_widen_ternary(packed, K, w=Wi)
-        evs[i][2].record(stream)
-        hbl.hbl_gemm_dequant(A, Wi, sc, alpha, y=y)
-        evs[i][3].record(stream)
-    torch.cuda.synchronize()
-    clk = clocks.stop()
-    t_k1 = statistics.mean(e[0].elapsed_time(e[1]) for e in evs) / 1e3
-    t_wd = statistics.mean(e[1].elapsed_time(e[2]) for e in evs) / 1e3
-    t_gm = statistics.mean(e[2].elapsed_time(e[3]) for e in evs) / 1e3
-    t_gm = ranks.max(t_gm, dev)
-    t_k1 = ranks.max(t_k1, dev)
-
-    ops = 2.0 * M * N * K
-    int8_peak = peaks["bf16_tflops"] * INT8_OVER_BF16
-    achieved_tops = ops / t_gm / 1e12
-    k1_bytes = M * K * (2 if wl.dtype == "bf16" else 4) + M * K + 4 * M
-    k1_gbs = k1_bytes / t_k1 / 1e9
-    roofline = {"bound": "tensor", "kernel": "gemm_i8_kernel (tcgen05 kind::i8 + dequant epilogue)",
-                "achieved": achieved_tops, "peak": int8_peak, "unit": "TFLOP/s", "frac": achieved_tops / int8_peak,
-                "traffic": measured_traffic("gemm_7b_wdown"),
-                "peak_source": "%s bf16 burst %.1f TFLOP/s x %.0f (nominal int8/bf16 dense ratio)"
-                               % (peak_kind, peaks["bf16_tflops"], INT8_OVER_BF16),
-                "algorithmic_ops_per_launch": ops, "launch_ms": t_gm * 1e3,
-                "frac_of_nominal_4500": achieved_tops / 4500.0}
-    k1 = {"bound": "hbm", "kernel": "ln_fht_quant_kernel (INT%d, int8 codes out)" % bits, "achieved": k1_gbs,
-          "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": k1_gbs / peaks["hbm_gbs"],
-          "traffic": measured_traffic("k1_7b_wdown"),
-          "algorithmic_bytes_per_launch": k1_bytes, "launch_ms": t_k1 * 1e3}
-
-    # -------- end to end through host memory (pinned), the public call
-    e2e = None
-    if not args.no_e2e:
-        xh = torch.empty(x.shape, dtype=x.dtype, pin_memory=True)
-        xh.copy_(x)
-        yh = torch.empty(y.shape, dtype=y.dtype, pin_memory=True)
-        xd = torch.empty_like(x)
-        for _ in range(2):
-            xd.copy_(xh, non_blocking=True)
-            hbl.hbl_forward(xd, packed, alpha, N, bits, y=y, workspace=ws)
-            yh.copy_(y, non_blocking=True)
-        torch.cuda.synchronize()
-        ranks.barrier()
-        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        f0.record(stream)
-        for _ in range(args.e2e_steps):
-            xd.copy_(xh, non_blocking=True)
-            hbl.hbl_forward(xd, packed, alpha, N, bits, y=y, workspace=ws)
-            yh.copy_(y, non_blocking=True)
-        f1.record(stream)
-        f1.synchronize()
-        ranks.barrier()
-        e2e_ms = ranks.max(f0.elapsed_time(f1) / args.e2e_steps, dev)
-        e2e = {"value": aggregate_value(M, ranks.world, e2e_ms / 1e3), "unit": "tokens/s",
-               "h2d_bytes_per_step": x.numel() * x.element_size(),
-               "d2h_bytes_per_step": y.numel() * y.element_size(), "ms_per_step": e2e_ms}
 
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ranks.world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True, "scaling": "weak",
