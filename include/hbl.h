@@ -167,9 +167,11 @@ hbl_status hbl_debug_norm(const void* x, hbl_dtype xt, int64_t M, int64_t K, hbl
                           cudaStream_t stream);
 
 /* ---------------------------------------------------------------- forward stages
- * hbl_forward is exactly these three calls on slices of its workspace; they
- * are public so that callers can keep the widened weight resident, overlap
- * stages, or time each kernel on their own stream. */
+ * hbl_forward is exactly these three calls on slices of its workspace (for
+ * decode-sized batches, M <= 4 and M * K <= 65536, the first call and then
+ * hbl_gemv_ternary_dequant, whose y is identical); they are public so that
+ * callers can keep the widened weight resident, overlap stages, or time each
+ * kernel on their own stream. */
 
 /* Activation path with one int8 per code (the layout the tensor cores read):
  * the same LN -> H -> quantizer as hbl_fht_quant, codes device int8 [M][K]
@@ -188,6 +190,19 @@ hbl_status hbl_widen_ternary(const uint8_t* packed, int64_t K, int64_t N, int8_t
 hbl_status hbl_gemm_dequant(const int8_t* A, const int8_t* w, int64_t M, int64_t N, int64_t K,
                             const float* scales, const float* alpha_dev, void* y, hbl_dtype yt,
                             cudaStream_t stream);
+
+/* The same product and dequantisation for decode-sized batches, straight
+ * from the packed 2-bit weights (no widened copy): y[m][n] = (float)(sum_k
+ * A[m][k] w[n][k]) * (scales[m] * alpha_dev[0]) with w the ternary codes of
+ * packed [N][K/4] (hbl_pack_ternary's layout).  The int32 sums are exact and
+ * the rescaling is hbl_gemm_dequant's, so y is bit-identical to it.  A device
+ * int8 [M][K] (16-byte aligned), packed device (16-byte aligned), scales,
+ * alpha_dev, y as in hbl_gemm_dequant.  Requires M <= 4, M * K <= 65536 and
+ * K a power of two in [64, 32768] (HBL_ERR_UNSUPPORTED otherwise), N a
+ * multiple of 16. */
+hbl_status hbl_gemv_ternary_dequant(const int8_t* A, const uint8_t* packed, int64_t M, int64_t N, int64_t K,
+                                    const float* scales, const float* alpha_dev, void* y, hbl_dtype yt,
+                                    cudaStream_t stream);
 
 /* ---------------------------------------------------------------- no caller workspace
  * The paper has no counterpart to this entry point; it exists for callers

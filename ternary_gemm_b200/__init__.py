@@ -86,6 +86,8 @@ def lib():
             L.hbl_widen_ternary.restype = i32
             L.hbl_gemm_dequant.argtypes = [p, p, i64, i64, i64, p, p, p, i32, p]
             L.hbl_gemm_dequant.restype = i32
+            L.hbl_gemv_ternary_dequant.argtypes = [p, p, i64, i64, i64, p, p, p, i32, p]
+            L.hbl_gemv_ternary_dequant.restype = i32
             L.hbl_debug_ln_fht.argtypes = [p, i32, i64, i64, p, p]
             L.hbl_debug_ln_fht.restype = i32
             L.hbl_quant_from_f32.argtypes = [p, i64, i64, i32, p, p, p]
@@ -317,6 +319,20 @@ def hbl_gemm_dequant(A, w, scales, alpha, y=None, y_dtype=None, stream=None):
         y = torch.empty((M, N), dtype=y_dtype or torch.bfloat16, device=A.device)
     _check(lib().hbl_gemm_dequant(_ptr(A), _ptr(w), M, N, K, _ptr(scales), _ptr(alpha), _ptr(y), _dtype_code(y),
                                   _stream(stream)), "hbl_gemm_dequant")
+    return y
+
+
+def hbl_gemv_ternary_dequant(A, packed, scales, alpha, y=None, y_dtype=None, stream=None):
+    """int8 A [M][K], packed ternary [N][K/4] -> y = (A w^T) * (scales[m] * alpha) [M][N]
+    (decode-sized M: M <= 4, M * K <= 65536)."""
+    torch = _torch()
+    _need_cuda(A, packed, scales, alpha)
+    M, K = A.shape
+    N = packed.shape[0]
+    if y is None:
+        y = torch.empty((M, N), dtype=y_dtype or torch.bfloat16, device=A.device)
+    _check(lib().hbl_gemv_ternary_dequant(_ptr(A), _ptr(packed), M, N, K, _ptr(scales), _ptr(alpha), _ptr(y),
+                                          _dtype_code(y), _stream(stream)), "hbl_gemv_ternary_dequant")
     return y
 
 

@@ -62,6 +62,15 @@ cudaError_t launch_gemm_i8(const int8_t* A, const int8_t* B, int64_t M, int64_t 
                            int y_mode, void* y, const float* scales, const float* alpha,
                            cudaStream_t stream);
 
+// Small-M product straight from the packed 2-bit weights with the same
+// dequantisation (y_mode 1 float, 2 bf16): M <= kGemvMaxRows and
+// M * K <= kGemvMaxCodeBytes (the code rows stay in L1), K % 64 == 0.
+constexpr int64_t kGemvMaxRows = 4;
+constexpr int64_t kGemvMaxCodeBytes = 65536;
+bool gemv_ternary_supports(int64_t M, int64_t K);
+cudaError_t launch_gemv_ternary(const int8_t* A, const float* scales, const uint8_t* packed, const float* alpha,
+                                int64_t M, int64_t N, int64_t K, int y_mode, void* y, cudaStream_t stream);
+
 // Device error word (bounded-wait timeouts) -- lives in gemm_i8.cu; kernels in
 // other translation units receive its device address.
 int* device_error_word();

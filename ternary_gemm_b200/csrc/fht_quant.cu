@@ -38,6 +38,7 @@
 #include <cstdint>
 
 #include "common.cuh"
+#include "sm100.cuh"
 #include "quant.cuh"
 #include "rowkit.cuh"
 
@@ -210,6 +211,9 @@ ln_fht_quant_kernel(const void* __restrict__ x, int64_t M, float sK, void* __res
   const void* xrow = reinterpret_cast<const unsigned char*>(x) + (size_t)(active ? row : 0) * K * esz;
   const int row_off = rl * S::STRIDE;
   constexpr bool kLN = MODE != K1_FHT_F32;  // the plain transform mode has no LayerNorm
+  // a programmatic dependent of this kernel may start now (it waits for this
+  // kernel's results itself before reading them)
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   float e[64];
 
@@ -344,7 +348,8 @@ template <int LOGK, bool BF16, int MODE>
 cudaError_t launch_one(const void* x, int64_t M, void* out, float* scales, cudaStream_t stream) {
   using S = Shape<LOGK>;
   auto kern = ln_fht_quant_kernel<LOGK, BF16, MODE>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)S::SMEM);
+  static bool smem_set[sm100_host::kMaxDevices] = {false};
+  cudaError_t e = sm100_host::ensure_smem(kern, (int)S::SMEM, smem_set);
   if (e != cudaSuccess) return e;
   const int64_t grid = (M + S::R - 1) / S::R;
   const float sK = (float)(1.0 / sqrt((double)S::K));

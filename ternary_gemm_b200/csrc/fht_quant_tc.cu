@@ -343,6 +343,9 @@ ln_fht_quant_tc_kernel(const __grid_constant__ CUtensorMap tmX, TcParams p) {
   fence_before();
   __syncthreads();
   fence_after();
+  // a programmatic dependent of this kernel may start now (it waits for this
+  // kernel's results itself before reading them)
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   if (warp < 4) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kCtrlRegs));
@@ -648,7 +651,8 @@ cudaError_t launch_tc(const void* x, int64_t M, void* out, float* scales, int* e
     return (int64_t)fa.numRegs * kThreads >= (int64_t)128 * kCtrlRegs + (int64_t)128 * kEpiGroups * kEpiRegs;
   }();
   if (!split_ok) return cudaErrorInvalidConfiguration;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+  static bool smem_set[sm100_host::kMaxDevices] = {false};
+  cudaError_t e = sm100_host::ensure_smem(kern, (int)kSmemBytes, smem_set);
   if (e != cudaSuccess) return e;
   const int nsm = sm100_host::sm_count();
   const int grid = p.num_groups < nsm ? p.num_groups : nsm;

@@ -567,8 +567,8 @@ cudaError_t launch_gemm_i8(const int8_t* A, const int8_t* B, int64_t M, int64_t 
     p.num_m = (int)((M + 255) / 256);
     p.num_n = (int)((N + 255) / 256);
     p.num_tiles = p.num_m * p.num_n;
-    cudaError_t e = cudaFuncSetAttribute(gemm_i8_2sm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)k2SmemBytes);
+    static bool smem_set2[sm100_host::kMaxDevices] = {false};
+    cudaError_t e = sm100_host::ensure_smem(gemm_i8_2sm_kernel, (int)k2SmemBytes, smem_set2);
     if (e != cudaSuccess) return e;
     const int pairs = sm_count() / 2;
     const int nclusters = p.num_tiles < pairs ? p.num_tiles : pairs;
@@ -588,7 +588,8 @@ cudaError_t launch_gemm_i8(const int8_t* A, const int8_t* B, int64_t M, int64_t 
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
   }
-  cudaError_t e = cudaFuncSetAttribute(gemm_i8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+  static bool smem_set[sm100_host::kMaxDevices] = {false};
+  cudaError_t e = sm100_host::ensure_smem(gemm_i8_kernel, (int)kSmemBytes, smem_set);
   if (e != cudaSuccess) return e;
   const int grid = p.num_tiles < sm_count() ? p.num_tiles : sm_count();
   gemm_i8_kernel<<<grid, kThreads, kSmemBytes, stream>>>(ta, tb, p);

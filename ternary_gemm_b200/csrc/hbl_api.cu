@@ -151,6 +151,12 @@ hbl_status hbl_forward(const void* x, hbl_dtype xt, int64_t M, int64_t K, const 
   int8_t* B = reinterpret_cast<int8_t*>(ws + L.b_off);
   const K1Mode mode = bits == 4 ? hbl::K1_Q4_I8 : hbl::K1_Q8_I8;
   cudaError_t e = hbl::launch_ln_fht_quant(x, xt == HBL_BF16, M, l, mode, A, scales, stream);
+  if (hbl::gemv_ternary_supports(M, K)) {
+    // decode-sized batch: the product straight from the packed weights
+    if (e == cudaSuccess)
+      e = hbl::launch_gemv_ternary(A, scales, packed, alpha_dev, M, N, K, yt == HBL_BF16 ? 2 : 1, y, stream);
+    return cuda_status(e);
+  }
   if (e == cudaSuccess) e = hbl::launch_widen_ternary(packed, N, K, B, stream);
   if (e == cudaSuccess) e = hbl::launch_gemm_i8(A, B, M, N, K, yt == HBL_BF16 ? 2 : 1, y, scales, alpha_dev, stream);
   return cuda_status(e);
@@ -189,6 +195,22 @@ hbl_status hbl_gemm_dequant(const int8_t* A, const int8_t* w, int64_t M, int64_t
   if (s != HBL_OK) return s;
   if ((s = check_n(N)) != HBL_OK) return s;
   return cuda_status(hbl::launch_gemm_i8(A, w, M, N, K, yt == HBL_BF16 ? 2 : 1, y, scales, alpha_dev, stream));
+}
+
+hbl_status hbl_gemv_ternary_dequant(const int8_t* A, const uint8_t* packed, int64_t M, int64_t N, int64_t K,
+                                    const float* scales, const float* alpha_dev, void* y, hbl_dtype yt,
+                                    cudaStream_t stream) {
+  if (!A || !packed || !scales || !alpha_dev || !y || !dtype_ok(yt)) return HBL_ERR_INVALID_ARG;
+  if (!aligned(A, 16) || !aligned(packed, 16) || !aligned(scales, 4) || !aligned(alpha_dev, 4) || !aligned(y, 4))
+    return HBL_ERR_INVALID_ARG;
+  int l;
+  hbl_status s = check_k(K, &l);
+  if (s != HBL_OK) return s;
+  if ((s = check_rows(M)) != HBL_OK) return s;
+  if ((s = check_n(N)) != HBL_OK) return s;
+  if (!hbl::gemv_ternary_supports(M, K)) return HBL_ERR_UNSUPPORTED;
+  return cuda_status(hbl::launch_gemv_ternary(A, scales, packed, alpha_dev, M, N, K, yt == HBL_BF16 ? 2 : 1, y,
+                                              stream));
 }
 
 hbl_status hbl_fht(const void* x, hbl_dtype xt, int64_t M, int64_t K, float* t, cudaStream_t stream) {

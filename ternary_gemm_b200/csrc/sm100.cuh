@@ -239,11 +239,30 @@ inline bool encode_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* p
   return r == CUDA_SUCCESS;
 }
 
+constexpr int kMaxDevices = 64;
+
+// SM count of the current device, queried once per device.
 inline int sm_count() {
+  static int cache[kMaxDevices] = {0};
   int dev = 0, n = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (dev >= 0 && dev < kMaxDevices && cache[dev] > 0) return cache[dev];
   if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+  if (dev >= 0 && dev < kMaxDevices) cache[dev] = n;
   return n;
+}
+
+// Dynamic shared memory limit of a kernel, set once per device: `done` is the
+// call site's own per-device flag array (one per kernel instantiation).
+template <typename Kernel>
+inline cudaError_t ensure_smem(Kernel kern, int bytes, bool (&done)[kMaxDevices]) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev >= 0 && dev < kMaxDevices && done[dev]) return cudaSuccess;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && dev >= 0 && dev < kMaxDevices) done[dev] = true;
+  return e;
 }
 
 }  // namespace sm100_host

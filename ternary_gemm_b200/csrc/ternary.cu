@@ -15,6 +15,7 @@
 
 #include "common.cuh"
 #include "quant.cuh"
+#include "ternary.cuh"
 
 namespace hbl {
 namespace {
@@ -104,32 +105,13 @@ pack_kernel(const void* __restrict__ W, int64_t nwords, int64_t count, const dou
   }
 }
 
-// Eight 2-bit fields (the low 16 bits of w) -> eight nibbles, field i in
-// nibble i: three shift-or-mask steps.
-__device__ __forceinline__ uint32_t spread_fields(uint32_t w) {
-  uint32_t y = w & 0xffffu;
-  y = (y | (y << 8)) & 0x00ff00ffu;
-  y = (y | (y << 4)) & 0x0f0f0f0fu;
-  y = (y | (y << 2)) & 0x33333333u;
-  return y;
-}
-
-// 2-bit code -> int8 byte by a byte-permute lookup: the table's bytes are
-// 00 -> 0x00, 01 -> 0x01, 10 -> 0x00 (unused pattern), 11 -> 0xFF (-1).
-__device__ __forceinline__ uint4 widen16(uint32_t w) {
-  constexpr uint32_t kLut = 0xff000100u;
-  const uint32_t lo = spread_fields(w), hi = spread_fields(w >> 16);
-  return make_uint4(__byte_perm(kLut, 0u, lo & 0xffffu), __byte_perm(kLut, 0u, lo >> 16),
-                    __byte_perm(kLut, 0u, hi & 0xffffu), __byte_perm(kLut, 0u, hi >> 16));
-}
-
 // One word (16 codes -> 16 bytes) per thread and iteration: consecutive
 // threads take consecutive words, so every store instruction of a warp writes
 // 512 contiguous bytes.
 __global__ void __launch_bounds__(kThreads)
 widen_kernel(const uint32_t* __restrict__ packed, int64_t nwords, uint4* __restrict__ out) {
   for (int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x; i < nwords; i += (int64_t)gridDim.x * kThreads)
-    out[i] = widen16(__ldg(packed + i));
+    out[i] = tern::widen16(__ldg(packed + i));
 }
 
 int grid_for(int64_t work) {
