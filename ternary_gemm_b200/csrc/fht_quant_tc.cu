@@ -161,9 +161,11 @@ __device__ __forceinline__ void stage(float (&e)[N]) {
 // one round: .x summed, .y summed or, with MAXY, maximized.  RT consecutive
 // lanes when RT <= 32, else RT / 32 whole warps numbered wq (their slots)
 // inside the barrier's `bar_n` threads.  Every thread of the row ends with
-// the identical pair.
+// the identical pair.  `failed` (a bounded wait of this group gave up) is
+// or-ed over the barrier's threads, so they all leave the loop together.
 template <int RT, bool MAXY>
-__device__ __forceinline__ float2 group_reduce2(float2 v, float2* slots, int wq, int lane, int bar_id, int bar_n) {
+__device__ __forceinline__ float2 group_reduce2(float2 v, float2* slots, int wq, int lane, int bar_id, int bar_n,
+                                                bool& failed) {
   constexpr int W = RT < 32 ? RT : 32;
 #pragma unroll
   for (int o = W / 2; o >= 1; o >>= 1) {
@@ -175,7 +177,7 @@ __device__ __forceinline__ float2 group_reduce2(float2 v, float2* slots, int wq,
   if constexpr (RT > 32) {
     constexpr int NW = RT / 32;
     if (lane == 0) slots[wq] = v;
-    named_bar_sync(bar_id, bar_n);
+    failed = named_bar_any(bar_id, bar_n, failed);
     const int w0 = wq & ~(NW - 1);
     v = slots[w0];
 #pragma unroll
@@ -310,8 +312,11 @@ ln_fht_quant_tc_kernel(const __grid_constant__ CUtensorMap tmX, TcParams p) {
   uint64_t* tfull = empty + kSlots;
   uint64_t* tempty = tfull + kRegions;
   uint64_t* drain = tempty + kRegions;
-  float2* red2 = reinterpret_cast<float2*>(drain + 1);   // [pair][8]: (sum of squares, |y| sum or max)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(red2 + 16);
+  // [pair][group parity][8]: (sum of squares, |y| sum or max).  Two sets:
+  // with no barrier between one group's reduction and the next group's, a
+  // fast warp writes the other set while a slow one still reads this one.
+  float2* red2 = reinterpret_cast<float2*>(drain + 1);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(red2 + 32);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -421,16 +426,19 @@ ln_fht_quant_tc_kernel(const __grid_constant__ CUtensorMap tmX, TcParams p) {
     const int bar_row = PAIR ? bar_pair : bar_wg;
     const int bar_row_n = PAIR ? 256 : 128;
     const int wq = PAIR ? 4 * h + quarter : quarter;  // warp number among the row's warps
-    float2* slot2 = red2 + 8 * pr + (PAIR ? 0 : 4 * h);
     const int i_hi = PAIR ? m : m % KH;
     for (int j = pr;; j += 2) {
       const int q = blockIdx.x + j * gridDim.x;
       if (q >= p.num_groups) break;
       const int region = j % kRegions;
+      // A wait that gives up does not leave at once: the group runs on (on
+      // stale TMEM contents, same addresses, bounded waits) to the row
+      // reduction, whose barrier ors the failure over every thread that
+      // shares a barrier with this one, and all of them leave there.
       int ok = 1;
       if (lane == 0) ok = wait_bounded(&tfull[region], (uint32_t)(j / kRegions) & 1u, abort_flag, p.err) ? 1 : 0;
       ok = __shfl_sync(0xffffffffu, ok, 0);
-      if (named_bar_any(bar_row, bar_row_n, ok == 0)) break;
+      bool failed = ok == 0;
       fence_after();
       const uint32_t tl = tmem_base + (uint32_t)(region * 128) + ((uint32_t)(quarter * 32) << 16);
 
@@ -537,8 +545,10 @@ ln_fht_quant_tc_kernel(const __grid_constant__ CUtensorMap tmX, TcParams p) {
       float stat_part = 0.0f;
       if constexpr (MODE == K1_Q8_I8) stat_part = max_abs64(y);
       if constexpr (MODE == K1_Q4_PACKED || MODE == K1_Q4_I8) stat_part = sum_abs64(y);
+      float2* slot2 = red2 + 16 * pr + 8 * ((j >> 1) & 1) + (PAIR ? 0 : 4 * h);
       const float2 red = group_reduce2<RT, MODE == K1_Q8_I8>(make_float2(sum_sq64(y), stat_part), slot2, wq, lane,
-                                                              bar_row, bar_row_n);
+                                                              bar_row, bar_row_n, failed);
+      if (failed) break;
       const float ss = red.x;
       const float var = ss * (1.0f / ((float)K * (float)K));
       const float cmul = __fmul_rn(__fdiv_rn(1.0f, sqrtf(__fadd_rn(var, 1e-5f))), p.sK);
