@@ -35,6 +35,12 @@ cudaError_t launch_ln_fht_quant(const void* x, bool in_bf16, int64_t M, int log2
 bool ln_fht_quant_tc_supports(bool in_bf16, int log2k, K1Mode mode, const void* x, const void* out);
 cudaError_t launch_ln_fht_quant_tc(const void* x, int64_t M, int log2k, K1Mode mode, void* out, float* scales,
                                    cudaStream_t stream);
+// The same launch with the ternary weight widening (2-bit [N][K/4] -> int8
+// [N][K]) done by the kernel's two otherwise idle warps per CTA alongside
+// the transform (hbl_forward's first two stages in one kernel).
+cudaError_t launch_ln_fht_quant_tc_widen(const void* x, int64_t M, int log2k, K1Mode mode, void* out,
+                                         float* scales, const uint8_t* packed, int64_t N, int64_t K, int8_t* w,
+                                         cudaStream_t stream);
 
 // LayerNorm (rms = false) or RMSNorm (rms = true) then the quantizer, without
 // the Hadamard transform; K a power of two in [256, 32768].

@@ -49,7 +49,10 @@
 //   warp 1     TMEM allocation (512 columns: A in the last 64, three
 //              128-column accumulator regions) and one thread issuing the
 //              MMAs of a group;
-//   warps 2-3  idle (registers are granted to whole warpgroups);
+//   warps 2-3  otherwise idle (registers are granted to whole warpgroups);
+//              in hbl_forward they widen the ternary weights to int8 for the
+//              GEMM that follows (a grid-stride loop, 16 codes per thread
+//              and step), which the issue-bound epilogue leaves room for;
 //   warps 4-19 four epilogue warpgroups in two pairs; pair p takes every
 //              other group: TMEM -> registers, butterflies, LayerNorm
 //              statistics, quantizer, codes stored straight to global memory
@@ -80,6 +83,7 @@
 #include "quant.cuh"
 #include "rowkit.cuh"
 #include "sm100.cuh"
+#include "ternary.cuh"
 
 namespace hbl {
 namespace {
@@ -113,6 +117,9 @@ struct TcParams {
   float* t_out;      // K1_T_F32: t [M][K]
   uint8_t* codes;    // quantizing modes: codes [M][K/2] (packed) or [M][K] (int8)
   int codes_al32;    // codes 32-byte aligned (256-bit stores allowed)
+  const uint32_t* wpacked;  // weight widening by the idle warps: 2-bit codes
+  uint4* wout;              // int8 codes out, 16 per uint4
+  int64_t wwords;           // 32-bit words of 2-bit codes (0: no widening)
   float* scales;     // [M]
   int* err;          // device error word
 };
@@ -411,6 +418,11 @@ ln_fht_quant_tc_kernel(const __grid_constant__ CUtensorMap tmX, TcParams p) {
         while (!mbar_try_wait(drain, 0) && globaltimer() - t0 < 200000000ull) {
         }
       }
+    } else {
+      // ---------------------------------------------- warps 2-3: weight widening
+      // (hbl_forward's next stage; the epilogue leaves issue slots to spare)
+      for (int64_t i = (int64_t)blockIdx.x * 64 + (warp - 2) * 32 + lane; i < p.wwords; i += (int64_t)gridDim.x * 64)
+        p.wout[i] = tern::widen16(__ldg(p.wpacked + i));
     }
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kEpiRegs));
@@ -630,8 +642,15 @@ ln_fht_quant_tc_kernel(const __grid_constant__ CUtensorMap tmX, TcParams p) {
   if (warp == 1) tmem_dealloc(tmem_base, kTmemCols);
 }
 
+struct WidenJob {
+  const uint32_t* packed = nullptr;
+  uint4* out = nullptr;
+  int64_t words = 0;
+};
+
 template <int LOGK, int MODE>
-cudaError_t launch_tc(const void* x, int64_t M, void* out, float* scales, int* err, cudaStream_t stream) {
+cudaError_t launch_tc(const void* x, int64_t M, void* out, float* scales, int* err, const WidenJob& wjob,
+                      cudaStream_t stream) {
   constexpr int C = LOGK >= 14 ? 128 : 64;
   constexpr int KH = (1 << LOGK) / C;
   constexpr bool PAIR = C == 128;
@@ -650,6 +669,9 @@ cudaError_t launch_tc(const void* x, int64_t M, void* out, float* scales, int* e
   p.t_out = reinterpret_cast<float*>(out);
   p.codes = reinterpret_cast<uint8_t*>(out);
   p.codes_al32 = (reinterpret_cast<uintptr_t>(out) & 31u) == 0;
+  p.wpacked = wjob.packed;
+  p.wout = wjob.out;
+  p.wwords = wjob.words;
   p.scales = scales;
   p.err = err;
   auto kern = ln_fht_quant_tc_kernel<LOGK, MODE>;
@@ -672,12 +694,12 @@ cudaError_t launch_tc(const void* x, int64_t M, void* out, float* scales, int* e
 
 template <int LOGK>
 cudaError_t launch_tc_mode(const void* x, int64_t M, K1Mode mode, void* out, float* scales, int* err,
-                           cudaStream_t s) {
+                           const WidenJob& w, cudaStream_t s) {
   switch (mode) {
-    case K1_T_F32: return launch_tc<LOGK, K1_T_F32>(x, M, out, scales, err, s);
-    case K1_Q4_PACKED: return launch_tc<LOGK, K1_Q4_PACKED>(x, M, out, scales, err, s);
-    case K1_Q4_I8: return launch_tc<LOGK, K1_Q4_I8>(x, M, out, scales, err, s);
-    case K1_Q8_I8: return launch_tc<LOGK, K1_Q8_I8>(x, M, out, scales, err, s);
+    case K1_T_F32: return launch_tc<LOGK, K1_T_F32>(x, M, out, scales, err, w, s);
+    case K1_Q4_PACKED: return launch_tc<LOGK, K1_Q4_PACKED>(x, M, out, scales, err, w, s);
+    case K1_Q4_I8: return launch_tc<LOGK, K1_Q4_I8>(x, M, out, scales, err, w, s);
+    case K1_Q8_I8: return launch_tc<LOGK, K1_Q8_I8>(x, M, out, scales, err, w, s);
     default: break;
   }
   return cudaErrorInvalidValue;
@@ -690,22 +712,42 @@ bool ln_fht_quant_tc_supports(bool in_bf16, int log2k, K1Mode mode, const void* 
          (reinterpret_cast<uintptr_t>(x) & 15u) == 0 && (reinterpret_cast<uintptr_t>(out) & 15u) == 0;
 }
 
-cudaError_t launch_ln_fht_quant_tc(const void* x, int64_t M, int log2k, K1Mode mode, void* out, float* scales,
-                                   cudaStream_t stream) {
+namespace {
+
+cudaError_t launch_tc_any(const void* x, int64_t M, int log2k, K1Mode mode, void* out, float* scales,
+                          const WidenJob& w, cudaStream_t stream) {
   if (M <= 0) return cudaSuccess;
   int* err = device_error_word();
   if (!err) return cudaErrorInvalidValue;
   switch (log2k) {
-    case 7: return launch_tc_mode<7>(x, M, mode, out, scales, err, stream);
-    case 8: return launch_tc_mode<8>(x, M, mode, out, scales, err, stream);
-    case 9: return launch_tc_mode<9>(x, M, mode, out, scales, err, stream);
-    case 10: return launch_tc_mode<10>(x, M, mode, out, scales, err, stream);
-    case 11: return launch_tc_mode<11>(x, M, mode, out, scales, err, stream);
-    case 12: return launch_tc_mode<12>(x, M, mode, out, scales, err, stream);
-    case 13: return launch_tc_mode<13>(x, M, mode, out, scales, err, stream);
-    case 14: return launch_tc_mode<14>(x, M, mode, out, scales, err, stream);
+    case 7: return launch_tc_mode<7>(x, M, mode, out, scales, err, w, stream);
+    case 8: return launch_tc_mode<8>(x, M, mode, out, scales, err, w, stream);
+    case 9: return launch_tc_mode<9>(x, M, mode, out, scales, err, w, stream);
+    case 10: return launch_tc_mode<10>(x, M, mode, out, scales, err, w, stream);
+    case 11: return launch_tc_mode<11>(x, M, mode, out, scales, err, w, stream);
+    case 12: return launch_tc_mode<12>(x, M, mode, out, scales, err, w, stream);
+    case 13: return launch_tc_mode<13>(x, M, mode, out, scales, err, w, stream);
+    case 14: return launch_tc_mode<14>(x, M, mode, out, scales, err, w, stream);
   }
   return cudaErrorInvalidValue;
+}
+
+}  // namespace
+
+cudaError_t launch_ln_fht_quant_tc(const void* x, int64_t M, int log2k, K1Mode mode, void* out, float* scales,
+                                   cudaStream_t stream) {
+  return launch_tc_any(x, M, log2k, mode, out, scales, WidenJob(), stream);
+}
+
+cudaError_t launch_ln_fht_quant_tc_widen(const void* x, int64_t M, int log2k, K1Mode mode, void* out,
+                                         float* scales, const uint8_t* packed, int64_t N, int64_t K, int8_t* w,
+                                         cudaStream_t stream) {
+  WidenJob job;
+  job.packed = reinterpret_cast<const uint32_t*>(packed);
+  job.out = reinterpret_cast<uint4*>(w);
+  job.words = N * K / 16;
+  if (M <= 0) return launch_widen_ternary(packed, N, K, w, stream);
+  return launch_tc_any(x, M, log2k, mode, out, scales, job, stream);
 }
 
 }  // namespace hbl

@@ -150,14 +150,21 @@ hbl_status hbl_forward(const void* x, hbl_dtype xt, int64_t M, int64_t K, const 
   float* scales = reinterpret_cast<float*>(ws + L.s_off);
   int8_t* B = reinterpret_cast<int8_t*>(ws + L.b_off);
   const K1Mode mode = bits == 4 ? hbl::K1_Q4_I8 : hbl::K1_Q8_I8;
-  cudaError_t e = hbl::launch_ln_fht_quant(x, xt == HBL_BF16, M, l, mode, A, scales, stream);
+  cudaError_t e;
   if (hbl::gemv_ternary_supports(M, K)) {
     // decode-sized batch: the product straight from the packed weights
+    e = hbl::launch_ln_fht_quant(x, xt == HBL_BF16, M, l, mode, A, scales, stream);
     if (e == cudaSuccess)
       e = hbl::launch_gemv_ternary(A, scales, packed, alpha_dev, M, N, K, yt == HBL_BF16 ? 2 : 1, y, stream);
     return cuda_status(e);
   }
-  if (e == cudaSuccess) e = hbl::launch_widen_ternary(packed, N, K, B, stream);
+  if (hbl::ln_fht_quant_tc_supports(xt == HBL_BF16, l, mode, x, A)) {
+    // the weight widening runs inside the quantizer kernel (its idle warps)
+    e = hbl::launch_ln_fht_quant_tc_widen(x, M, l, mode, A, scales, packed, N, K, B, stream);
+  } else {
+    e = hbl::launch_ln_fht_quant(x, xt == HBL_BF16, M, l, mode, A, scales, stream);
+    if (e == cudaSuccess) e = hbl::launch_widen_ternary(packed, N, K, B, stream);
+  }
   if (e == cudaSuccess) e = hbl::launch_gemm_i8(A, B, M, N, K, yt == HBL_BF16 ? 2 : 1, y, scales, alpha_dev, stream);
   return cuda_status(e);
 }
