@@ -24,7 +24,10 @@
 //               committing each stage back to the producer and each finished
 //               accumulator to the epilogue;
 //   warps 2-5   epilogue: tcgen05.ld 32 columns at a time from the TMEM lane
-//               quarter each warp may access, scale, convert, store.
+//               quarter each warp may access, scale, convert, store (as
+//               streaming stores: y is not read again here, and evicting it
+//               early writes it back while this kernel leaves DRAM idle
+//               instead of during the memory-bound kernel that follows).
 // The accumulator double buffer lets the epilogue of tile i overlap the main
 // loop of tile i+1.  Every mbarrier wait is bounded: after ~2 s a thread sets
 // the CTA abort flag and the device error word, every role leaves its loop,
@@ -231,7 +234,7 @@ gemm_i8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
               v.y = __fmul_rn(__int2float_rn((int)r[j + 1]), sa);
               v.z = __fmul_rn(__int2float_rn((int)r[j + 2]), sa);
               v.w = __fmul_rn(__int2float_rn((int)r[j + 3]), sa);
-              *reinterpret_cast<float4*>(yrow + col0 + j) = v;
+              __stcs(reinterpret_cast<float4*>(yrow + col0 + j), v);
             }
           }
         } else {
@@ -244,7 +247,7 @@ gemm_i8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
               v.y = bf16x2(__fmul_rn(__int2float_rn((int)r[j + 2]), sa), __fmul_rn(__int2float_rn((int)r[j + 3]), sa));
               v.z = bf16x2(__fmul_rn(__int2float_rn((int)r[j + 4]), sa), __fmul_rn(__int2float_rn((int)r[j + 5]), sa));
               v.w = bf16x2(__fmul_rn(__int2float_rn((int)r[j + 6]), sa), __fmul_rn(__int2float_rn((int)r[j + 7]), sa));
-              *reinterpret_cast<uint4*>(yrow + col0 + j) = v;
+              __stcs(reinterpret_cast<uint4*>(yrow + col0 + j), v);
             }
           }
         }
@@ -362,7 +365,7 @@ __device__ __forceinline__ void epilogue_tile(const Params& p, uint32_t tbase, i
           v.y = __fmul_rn(__int2float_rn((int)r[j + 1]), sa);
           v.z = __fmul_rn(__int2float_rn((int)r[j + 2]), sa);
           v.w = __fmul_rn(__int2float_rn((int)r[j + 3]), sa);
-          *reinterpret_cast<float4*>(yrow + col0 + j) = v;
+          __stcs(reinterpret_cast<float4*>(yrow + col0 + j), v);
         }
       }
     } else {
@@ -375,7 +378,7 @@ __device__ __forceinline__ void epilogue_tile(const Params& p, uint32_t tbase, i
           v.y = bf16x2(__fmul_rn(__int2float_rn((int)r[j + 2]), sa), __fmul_rn(__int2float_rn((int)r[j + 3]), sa));
           v.z = bf16x2(__fmul_rn(__int2float_rn((int)r[j + 4]), sa), __fmul_rn(__int2float_rn((int)r[j + 5]), sa));
           v.w = bf16x2(__fmul_rn(__int2float_rn((int)r[j + 6]), sa), __fmul_rn(__int2float_rn((int)r[j + 7]), sa));
-          *reinterpret_cast<uint4*>(yrow + col0 + j) = v;
+          __stcs(reinterpret_cast<uint4*>(yrow + col0 + j), v);
         }
       }
     }
