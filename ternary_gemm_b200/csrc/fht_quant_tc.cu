@@ -63,10 +63,11 @@
 // of the transformed but unscaled y, since t = cmul y.  INT8 then stays
 // exact: gamma = fl(cmul max|y|) = max|t| (rounding is monotone) and the
 // codes are rint(fl(cmul y) r).  INT4 takes beta = fl(cmul sum|y|) / K with
-// the sum in float (trees of depth <= 22) and codes rint(y fl(cmul r)): beta
-// within ~24 units in the last place (1.5e-6) of the double sum over t, and
-// y fl(cmul r) within 2 units of t r, so a code can differ from the
-// quantizer-on-t value only where t r is within ~1.5e-5 of a half-integer
+// the sum in float (trees of depth <= 22), r a fast division, the scale
+// beta * fl(1/sqrt 7), and codes rint(y fl(cmul r)): beta within ~24 units
+// in the last place (1.5e-6) of the double sum over t, and y fl(cmul r)
+// within ~30 units of t r, so a code can differ from the quantizer-on-t
+// value only where t r is within ~1.5e-5 of a half-integer
 // (a double per-element sum and a second reduction round cost about a
 // quarter of the kernel's time).  INT4 codes widened to int8 are clipped on
 // packed 16-bit halves when the row bound ||t|| r keeps every code below
@@ -563,7 +564,9 @@ ln_fht_quant_tc_kernel(const __grid_constant__ CUtensorMap tmX, TcParams p) {
       if (failed) break;
       const float ss = red.x;
       const float var = ss * (1.0f / ((float)K * (float)K));
-      const float cmul = __fmul_rn(__fdiv_rn(1.0f, sqrtf(__fadd_rn(var, 1e-5f))), p.sK);
+      // 1 / sqrt(K (var + eps)): a correctly rounded reciprocal square root
+      // (one rounding) times 1/sqrt(K); the debug and quantizing modes share it
+      const float cmul = __fmul_rn(__frsqrt_rn(__fadd_rn(var, 1e-5f)), p.sK);
       const bool row_ok = row < p.M;
       // this thread's chunk row: C = 64, unit row m; C = 128, tile row m
       const int64_t crow = (PAIR ? (int64_t)q * kBoxRows : unit0) + m;
@@ -612,7 +615,7 @@ ln_fht_quant_tc_kernel(const __grid_constant__ CUtensorMap tmX, TcParams p) {
           } else {
             // 16 codes per 16 bytes: C = 64 at 0, 16, 32, 48; C = 128 at
             // 32h, 32h + 16, 64 + 32h, 80 + 32h
-            const bool s16 = MODE == K1_Q4_I8 && sqrtf(ss) * cq < 30000.0f;
+            const bool s16 = MODE == K1_Q4_I8 && ss * cq * cq < 9.0e8f;
             if (PAIR && p.codes_al32) {
               // two whole 32-byte sectors per thread, not four half sectors
 #pragma unroll

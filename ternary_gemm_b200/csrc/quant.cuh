@@ -45,13 +45,16 @@ __device__ __forceinline__ RowParams params_int4(double abs_sum, int64_t K) {
 
 // beta from a float sum of |t| over K elements (K a power of two, so the
 // division is exact).  Used by the fused tensor-core kernel, whose sum is a
-// float tree (relative error at most ~15 float units in the last place);
-// the quantizer-only kernel keeps the double sum above.
+// float tree (relative error at most ~24 float units in the last place);
+// the quantizer-only kernel keeps the double sum above.  With that tolerance
+// the row's divisions need not be correctly rounded: r is one fast division
+// (within 2 ulp) and the scale a product with fl(1/sqrt(7)) (within 1.5 ulp).
+constexpr float kInvSqrt7 = 0.37796447300922722f;  // 1/sqrt(7) rounded to float
 __device__ __forceinline__ RowParams params_int4_f32(float abs_sum, int64_t K) {
   const float beta = abs_sum * (1.0f / (float)K);
   RowParams p;
-  p.r = __fdiv_rn(kSqrt7, __fadd_rn(beta, kEps));
-  p.scale = __fdiv_rn(beta, kSqrt7);
+  p.r = __fdividef(kSqrt7, __fadd_rn(beta, kEps));
+  p.scale = __fmul_rn(beta, kInvSqrt7);
   return p;
 }
 

@@ -68,10 +68,11 @@ def check_codes_near(q_gpu, q_orc, t_orc32, scale_orc, bits, min_agree=0.9999, h
 # from the transformed, unscaled y (t = cmul y): beta = fl(cmul * S) / K with S
 # a float tree sum of |y| of depth <= 22 (10 levels inside a thread, 5 shuffle
 # levels, 7 slot additions), so beta is within 22 + 2 units in the last place
-# (1.5e-6) of the double sum over t; codes are rint(y * fl(cmul r)), within 2
-# more units of t r.  A code can then change only where the exact t*r
-# (|t*r| <= 8.5 for an unclipped code) lies within 8.5 * 28 units (1.5e-5) of
-# a half-integer.
+# (1.5e-6) of the double sum over t, and the scale (beta times fl(1/sqrt 7))
+# within 1.5 more; codes are rint(y * fl(cmul r)) with r a fast division
+# (2 ulp), within 30 units of t r.  A code can then change only where the
+# exact t*r (|t*r| <= 8.5 for an unclipped code) lies within 8.5 * 30 units
+# (1.5e-5) of a half-integer.
 FUSED_BETA_REL = 2e-6
 FUSED_HALF_TOL = 3e-5
 
