@@ -118,9 +118,9 @@ struct TcParams {
   float* t_out;      // K1_T_F32: t [M][K]
   uint8_t* codes;    // quantizing modes: codes [M][K/2] (packed) or [M][K] (int8)
   int codes_al32;    // codes 32-byte aligned (256-bit stores allowed)
-  const uint32_t* wpacked;  // weight widening by the idle warps: 2-bit codes
+  const uint32_t* wpacked;  // weight widening by the idle warps: 2-bit codes (16-byte aligned)
   uint4* wout;              // int8 codes out, 16 per uint4
-  int64_t wwords;           // 32-bit words of 2-bit codes (0: no widening)
+  int64_t wwords;           // 32-bit words of 2-bit codes, a multiple of 4 (0: no widening)
   float* scales;     // [M]
   int* err;          // device error word
 };
@@ -421,9 +421,28 @@ ln_fht_quant_tc_kernel(const __grid_constant__ CUtensorMap tmX, TcParams p) {
       }
     } else {
       // ---------------------------------------------- warps 2-3: weight widening
-      // (hbl_forward's next stage; the epilogue leaves issue slots to spare)
-      for (int64_t i = (int64_t)blockIdx.x * 64 + (warp - 2) * 32 + lane; i < p.wwords; i += (int64_t)gridDim.x * 64)
-        p.wout[i] = tern::widen16(__ldg(p.wpacked + i));
+      // (hbl_forward's next stage; the epilogue leaves issue slots to spare).
+      // Only 64 threads per SM do it, so each keeps two 16-byte loads (128
+      // codes) in flight; every warp store covers 2 KB of contiguous output.
+      constexpr int kU = 2;
+      const uint4* src = reinterpret_cast<const uint4*>(p.wpacked);
+      const int64_t n4 = p.wwords / 4;  // 64 codes per uint4
+      const int64_t stride = (int64_t)gridDim.x * 64;
+      for (int64_t i = (int64_t)blockIdx.x * 64 + (warp - 2) * 32 + lane; i < n4; i += stride * kU) {
+        uint4 v[kU];
+#pragma unroll
+        for (int u = 0; u < kU; ++u) v[u] = i + u * stride < n4 ? __ldg(src + i + u * stride) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+          if (i + u * stride < n4) {
+            uint4* d = p.wout + 4 * (i + u * stride);
+            d[0] = tern::widen16(v[u].x);
+            d[1] = tern::widen16(v[u].y);
+            d[2] = tern::widen16(v[u].z);
+            d[3] = tern::widen16(v[u].w);
+          }
+        }
+      }
     }
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kEpiRegs));
