@@ -2,7 +2,7 @@
 // with the transform split between the tensor cores and the FMA pipe
 // ("BitNet v2: Native 4-bit Activations with Hadamard Transformation for
 // 1-bit LLMs", section "H-BitLinear": the Hadamard-transform definition and
-// the activation-quantization formula).  bf16 input, K = 128 .. 16384.
+// the activation-quantization formula).  bf16 input, K = 128 .. 32768.
 //
 // Sylvester's matrix factors over the index bits: with i = C i_hi + i_lo,
 // j = C j_hi + j_lo and KH = K / C,
@@ -664,6 +664,336 @@ ln_fht_quant_tc_kernel(const __grid_constant__ CUtensorMap tmX, TcParams p) {
   if (warp == 1) tmem_dealloc(tmem_base, kTmemCols);
 }
 
+// ---------------------------------------------------------------- K = 32768
+// 256-column chunks (KH = 128, so the high factor is still H_128): a tile is
+// one token row, 128 chunk rows x 256 columns = four 64-column boxes (64 KB),
+// and one N = 256 MMA per K step.  A (H_128 in bf16) stays in shared memory
+// so that TMEM holds two 256-column accumulators (the MMA of the next tile
+// overlaps this tile's epilogue).  All four epilogue warpgroups share each
+// tile: warpgroup g loads columns 64 g .. 64 g + 63 of its lanes and runs
+// the 6 low stages; two exchange rounds through TMEM, each behind a barrier
+// of the two warpgroups involved, bring the partners of column bit 6 and
+// then of bit 7 together.  In 32-column units u (columns 32 u ..), warpgroup
+// g starts with units {2g, 2g+1}, holds {0,2} {1,3} {4,6} {5,7} after round
+// 1 and the final outputs {g, g+4} after round 2.  Every exchange write goes
+// to a unit nobody reads again except its receiver, and unit 0 (whose first
+// column the i_hi = 0 lanes of every warpgroup read for the mean removal) is
+// never written.
+constexpr int k256Cols = 256;
+constexpr int k256TileBytes = 4 * kBoxBytes;  // 64 KB
+constexpr int k256Slots = 2;
+constexpr int k256ABytes = 128 * 128 * 2;
+constexpr size_t k256SmemBytes = 1024 + (size_t)k256ABytes + (size_t)k256Slots * k256TileBytes + 1024;
+// kind::f16: D f32, A and B bf16, A K-major, B MN-major, N = 256, M = 128
+constexpr uint32_t kIdesc256 =
+    (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) | ((256u >> 3) << 17) | ((128u >> 4) << 24);
+
+__device__ __forceinline__ void mma_bf16_ss(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(kIdesc256), "r"(accumulate));
+}
+
+// H_128 as bf16 in the K-major 128B-swizzled layout: two 64-column blocks of
+// 128 rows x 128 bytes; 16-byte chunk c of row m at chunk position c ^ (m & 7).
+__device__ __forceinline__ void build_h128_smem(uint8_t* sA, int tid, int nthreads) {
+  for (int c = tid; c < 2048; c += nthreads) {
+    const int blk = c >> 10, m = (c >> 3) & 127, cc = c & 7;
+    uint32_t w[4];
+#pragma unroll
+    for (int u = 0; u < 8; u += 2) {
+      uint32_t hv[2];
+#pragma unroll
+      for (int v = 0; v < 2; ++v) {
+        const int k = blk * 64 + cc * 8 + u + v;
+        hv[v] = 0x3F80u ^ ((uint32_t)(__popc(m & k) & 1) << 15);
+      }
+      w[u >> 1] = hv[0] | (hv[1] << 16);
+    }
+    *reinterpret_cast<uint4*>(sA + blk * 16384 + m * 128 + ((cc ^ (m & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+}
+
+// 32 TMEM columns from registers r[0..31] / into them
+__device__ __forceinline__ void tm_put32(uint32_t taddr, const float* r) {
+  uint32_t u[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) u[i] = __float_as_uint(r[i]);
+  tmem_st32(taddr, u);
+}
+__device__ __forceinline__ void tm_get32(uint32_t taddr, float* r) {
+  uint32_t u[32];
+  tmem_ld32_nowait(taddr, u);
+  tmem_wait_ld();
+#pragma unroll
+  for (int i = 0; i < 32; ++i) r[i] = __uint_as_float(u[i]);
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(kThreads, 1)
+ln_fht_quant_tc256_kernel(const __grid_constant__ CUtensorMap tmX, TcParams p) {
+  constexpr int K = 32768;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  uint8_t* sA = base;
+  uint8_t* sB = sA + k256ABytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + k256Slots * k256TileBytes);
+  uint64_t* empty = full + k256Slots;
+  uint64_t* tfull = empty + k256Slots;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  float2* red2 = reinterpret_cast<float2*>(drain + 1);  // [tile parity][16 warps]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(red2 + 32);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s2 = 0; s2 < k256Slots; ++s2) {
+      mbar_init(&full[s2], 1);
+      mbar_init(&empty[s2], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 16);  // every epilogue warp reads every tile
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, kTmemCols);
+  if (warp >= 4) {
+    build_h128_smem(sA, threadIdx.x - 128, kThreads - 128);
+    fence_proxy_async_smem();
+  }
+  fence_before();
+  __syncthreads();
+  fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+
+  if (warp < 4) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kCtrlRegs));
+    if (warp == 0) {
+      if (lane == 0) {
+        prefetch_tensormap(&tmX);
+        bool ok = true;
+        for (int j = 0;; ++j) {
+          const int q = blockIdx.x + j * gridDim.x;
+          if (q >= p.num_groups) break;
+          const int slot = j % k256Slots;
+          if (!wait_bounded(&empty[slot], ((uint32_t)(j / k256Slots) & 1u) ^ 1u, abort_flag, p.err)) {
+            ok = false;
+            break;
+          }
+          mbar_expect_tx(&full[slot], (uint32_t)k256TileBytes);
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+            tma_load_2d(sB + slot * k256TileBytes + u * kBoxBytes, &tmX, kBoxCols * u, q * kBoxRows, &full[slot]);
+        }
+        if (!ok) {
+          const uint64_t t0 = globaltimer();
+          while (globaltimer() - t0 < 20000000ull) {
+          }
+        }
+      }
+    } else if (warp == 1) {
+      if (lane == 0) {
+        const uint32_t a_addr = smem_u32(sA);
+        for (int j = 0;; ++j) {
+          const int q = blockIdx.x + j * gridDim.x;
+          if (q >= p.num_groups) break;
+          const int slot = j % k256Slots, region = j & 1;
+          if (!wait_bounded(&tempty[region], ((uint32_t)(j >> 1) & 1u) ^ 1u, abort_flag, p.err)) break;
+          if (!wait_bounded(&full[slot], (uint32_t)(j / k256Slots) & 1u, abort_flag, p.err)) break;
+          fence_after();
+          const uint32_t d = tmem_base + (uint32_t)(region * k256Cols);
+          // B: four 64-column atoms 16 KB apart, 2048 bytes per K=16 step
+          const uint64_t b = sdesc_mn_sw128(smem_u32(sB + slot * k256TileBytes), kBoxBytes);
+#pragma unroll
+          for (int s2 = 0; s2 < 8; ++s2) {
+            const uint64_t a = sdesc_k_sw128(a_addr + (uint32_t)((s2 >> 2) * 16384)) + (uint64_t)(2 * (s2 & 3));
+            mma_bf16_ss(d, a, b + (uint64_t)(128 * s2), s2 > 0 ? 1u : 0u);
+          }
+          umma_commit(&empty[slot]);
+          umma_commit(&tfull[region]);
+        }
+        umma_commit(drain);
+        const uint64_t t0 = globaltimer();
+        while (!mbar_try_wait(drain, 0) && globaltimer() - t0 < 200000000ull) {
+        }
+      }
+    } else {
+      // warps 2-3: weight widening for hbl_forward's GEMM (see the main kernel)
+      constexpr int kU = 2;
+      const uint4* src = reinterpret_cast<const uint4*>(p.wpacked);
+      const int64_t n4 = p.wwords / 4;
+      const int64_t stride = (int64_t)gridDim.x * 64;
+      for (int64_t i = (int64_t)blockIdx.x * 64 + (warp - 2) * 32 + lane; i < n4; i += stride * kU) {
+        uint4 v[kU];
+#pragma unroll
+        for (int u = 0; u < kU; ++u) v[u] = i + u * stride < n4 ? __ldg(src + i + u * stride) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+          if (i + u * stride < n4) {
+            uint4* dd = p.wout + 4 * (i + u * stride);
+            dd[0] = tern::widen16(v[u].x);
+            dd[1] = tern::widen16(v[u].y);
+            dd[2] = tern::widen16(v[u].z);
+            dd[3] = tern::widen16(v[u].w);
+          }
+        }
+      }
+    }
+  } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kEpiRegs));
+    const int g = (warp - 4) >> 2;    // epilogue warpgroup: starting columns 64 g ..
+    const int quarter = warp & 3;
+    const int m = quarter * 32 + lane;  // lane = i_hi
+    const int wq = 4 * g + quarter;
+    const int h1 = g & 1;               // role in round 1 (pairs {0,1}, {2,3})
+    const int bar_r1 = 1 + (g >> 1);
+    const int bar_r2 = 3 + (g & 1);     // round 2 pairs {0,2}, {1,3}
+    const int bar_row = 5;
+    // round 2: location written, location read, and whether the kept 32
+    // values are y[0..31] (else y[32..63])
+    const int w2 = g == 0 ? 3 : g == 1 ? 1 : g == 2 ? 4 : 7;
+    const int r2 = g == 0 ? 4 : g == 1 ? 7 : g == 2 ? 3 : 1;
+    const bool keep_lo2 = g < 2;
+    for (int j = 0;; ++j) {
+      const int q = blockIdx.x + j * gridDim.x;
+      if (q >= p.num_groups) break;
+      const int region = j & 1;
+      int ok = 1;
+      if (lane == 0) ok = wait_bounded(&tfull[region], (uint32_t)(j >> 1) & 1u, abort_flag, p.err) ? 1 : 0;
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      bool failed = ok == 0;
+      fence_after();
+      const uint32_t tl = tmem_base + (uint32_t)(region * k256Cols) + ((uint32_t)(quarter * 32) << 16);
+
+      float y[64];
+      {
+        uint32_t u[64];
+        uint32_t c0w = 0;
+        tmem_ld32_nowait(tl + (uint32_t)(64 * g), &u[0]);
+        tmem_ld32_nowait(tl + (uint32_t)(64 * g + 32), &u[32]);
+        if (g > 0 && quarter == 0) c0w = tmem_ld1(tl);  // column 0 of lane 0 for the mean removal
+        tmem_wait_ld();
+#pragma unroll
+        for (int r = 0; r < 64; ++r) y[r] = __uint_as_float(u[r]);
+        if (m == 0) {
+          const float c0 = g == 0 ? y[0] : __uint_as_float(c0w);
+#pragma unroll
+          for (int r = 0; r < 64; r += 2) sub2(y[r], y[r + 1], c0);
+        }
+      }
+      stage<0>(y);
+      stage<1>(y);
+      stage<2>(y);
+      stage<3>(y);
+      stage<4>(y);
+      stage<5>(y);
+      // round 1 (column bit 6): units 2g, 2g+1 -> {4(g>>1) + h1, 4(g>>1) + h1 + 2}
+      if (h1 == 0) tm_put32(tl + (uint32_t)(64 * g + 32), &y[32]);  // hand over unit 2g+1
+      else tm_put32(tl + (uint32_t)(64 * g), &y[0]);                 // hand over unit 2g
+      tmem_wait_st();
+      fence_before();
+      named_bar_sync(bar_r1, 256);
+      fence_after();
+      if (h1 == 0) tm_get32(tl + (uint32_t)(64 * g + 64), &y[32]);   // partner's unit 2g+2
+      else tm_get32(tl + (uint32_t)(64 * g - 32), &y[0]);            // partner's unit 2g-1
+#pragma unroll
+      for (int r = 0; r < 32; r += 2) bfly2(y[r], y[r + 1], y[32 + r], y[33 + r]);
+      // round 2 (column bit 7)
+      if (keep_lo2) tm_put32(tl + (uint32_t)(32 * w2), &y[32]);
+      else tm_put32(tl + (uint32_t)(32 * w2), &y[0]);
+      tmem_wait_st();
+      fence_before();
+      named_bar_sync(bar_r2, 256);
+      fence_after();
+      if (keep_lo2) tm_get32(tl + (uint32_t)(32 * r2), &y[32]);
+      else tm_get32(tl + (uint32_t)(32 * r2), &y[0]);
+      fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[region]);
+#pragma unroll
+      for (int r = 0; r < 32; r += 2) bfly2(y[r], y[r + 1], y[32 + r], y[33 + r]);
+      // now y[r] = column 32 g + r, y[32 + r] = column 128 + 32 g + r
+      if (m == 0 && g == 0) y[0] = 0.0f;  // t_0 = 0
+
+      float stat_part = 0.0f;
+      if constexpr (MODE == K1_Q8_I8) stat_part = max_abs64(y);
+      if constexpr (MODE == K1_Q4_PACKED || MODE == K1_Q4_I8) stat_part = sum_abs64(y);
+      float2* slot2 = red2 + 16 * (j & 1);
+      const float2 red = group_reduce2<512, MODE == K1_Q8_I8>(make_float2(sum_sq64(y), stat_part), slot2, wq, lane,
+                                                               bar_row, 512, failed);
+      if (failed) break;
+      const float ss = red.x;
+      const float var = ss * (1.0f / ((float)K * (float)K));
+      const float cmul = __fmul_rn(__frsqrt_rn(__fadd_rn(var, 1e-5f)), p.sK);
+      const int64_t row = q;
+      const int64_t crow = (int64_t)q * kBoxRows + m;
+
+      if constexpr (MODE == K1_T_F32) {
+#pragma unroll
+        for (int r = 0; r < 64; r += 2) mul2(y[r], y[r + 1], cmul);
+        float* trow = p.t_out + (size_t)row * K + (size_t)m * k256Cols;
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          float4* dst = reinterpret_cast<float4*>(trow + 128 * half + 32 * g);
+#pragma unroll
+          for (int jj = 0; jj < 8; ++jj) {
+            const int r = 32 * half + 4 * jj;
+            dst[jj] = make_float4(y[r], y[r + 1], y[r + 2], y[r + 3]);
+          }
+        }
+      } else {
+        q::RowParams qp;
+        float cq;
+        if constexpr (MODE == K1_Q8_I8) {
+          qp = q::params_int8(__fmul_rn(cmul, red.y));
+#pragma unroll
+          for (int r = 0; r < 64; r += 2) mul2(y[r], y[r + 1], cmul);
+          cq = qp.r;
+        } else {
+          qp = q::params_int4_f32(__fmul_rn(cmul, red.y), K);
+          cq = __fmul_rn(cmul, qp.r);
+        }
+        if (m == 0 && g == 0) p.scales[row] = qp.scale;
+        uint8_t* crow_out = p.codes + crow * (MODE == K1_Q4_PACKED ? k256Cols / 2 : k256Cols);
+        if constexpr (MODE == K1_Q4_PACKED) {
+          // 32 codes (16 bytes) per half, at bytes 16 g and 64 + 16 g
+          *reinterpret_cast<uint4*>(crow_out + 16 * g) = codes32_s4(&y[0], cq);
+          *reinterpret_cast<uint4*>(crow_out + 64 + 16 * g) = codes32_s4(&y[32], cq);
+        } else {
+          const bool s16 = MODE == K1_Q4_I8 && ss * cq * cq < 9.0e8f;
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {
+            const uint4 v0 = s16 ? codes16_i8<MODE, true>(&y[32 * half], cq) : codes16_i8<MODE>(&y[32 * half], cq);
+            const uint4 v1 =
+                s16 ? codes16_i8<MODE, true>(&y[32 * half + 16], cq) : codes16_i8<MODE>(&y[32 * half + 16], cq);
+            uint8_t* dst = crow_out + 128 * half + 32 * g;
+            if (p.codes_al32) {
+              st_global_32B(dst, v0, v1);
+            } else {
+              reinterpret_cast<uint4*>(dst)[0] = v0;
+              reinterpret_cast<uint4*>(dst)[1] = v1;
+            }
+          }
+        }
+      }
+    }
+  }
+
+  fence_before();
+  __syncthreads();
+  fence_after();
+  if (warp == 1) tmem_dealloc(tmem_base, kTmemCols);
+}
+
 struct WidenJob {
   const uint32_t* packed = nullptr;
   uint4* out = nullptr;
@@ -714,15 +1044,63 @@ cudaError_t launch_tc(const void* x, int64_t M, void* out, float* scales, int* e
   return cudaGetLastError();
 }
 
+template <int MODE>
+cudaError_t launch_tc256(const void* x, int64_t M, void* out, float* scales, int* err, const WidenJob& wjob,
+                         cudaStream_t stream) {
+  const int64_t nchunk = M * 128;
+  if (M > (int64_t)INT32_MAX / 4) return cudaErrorInvalidValue;
+  CUtensorMap tmX;
+  if (!sm100_host::encode_2d(&tmX, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, k256Cols, (uint64_t)nchunk, k256Cols * 2,
+                             kBoxCols, kBoxRows, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  TcParams p;
+  p.M = M;
+  p.nchunk = nchunk;
+  p.num_groups = (int)M;
+  p.sK = (float)(1.0 / sqrt(32768.0));
+  p.t_out = reinterpret_cast<float*>(out);
+  p.scales = scales;
+  p.err = err;
+  p.codes = reinterpret_cast<uint8_t*>(out);
+  p.codes_al32 = (reinterpret_cast<uintptr_t>(out) & 31u) == 0;
+  p.wpacked = wjob.packed;
+  p.wout = wjob.out;
+  p.wwords = wjob.words;
+  auto kern = ln_fht_quant_tc256_kernel<MODE>;
+  static const bool split_ok = [&]() {
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return false;
+    return (int64_t)fa.numRegs * kThreads >= (int64_t)128 * kCtrlRegs + (int64_t)128 * kEpiGroups * kEpiRegs;
+  }();
+  if (!split_ok) return cudaErrorInvalidConfiguration;
+  static bool smem_set[sm100_host::kMaxDevices] = {false};
+  cudaError_t e = sm100_host::ensure_smem(kern, (int)k256SmemBytes, smem_set);
+  if (e != cudaSuccess) return e;
+  const int nsm = sm100_host::sm_count();
+  const int grid = p.num_groups < nsm ? p.num_groups : nsm;
+  kern<<<grid, kThreads, k256SmemBytes, stream>>>(tmX, p);
+  return cudaGetLastError();
+}
+
 template <int LOGK>
 cudaError_t launch_tc_mode(const void* x, int64_t M, K1Mode mode, void* out, float* scales, int* err,
                            const WidenJob& w, cudaStream_t s) {
-  switch (mode) {
-    case K1_T_F32: return launch_tc<LOGK, K1_T_F32>(x, M, out, scales, err, w, s);
-    case K1_Q4_PACKED: return launch_tc<LOGK, K1_Q4_PACKED>(x, M, out, scales, err, w, s);
-    case K1_Q4_I8: return launch_tc<LOGK, K1_Q4_I8>(x, M, out, scales, err, w, s);
-    case K1_Q8_I8: return launch_tc<LOGK, K1_Q8_I8>(x, M, out, scales, err, w, s);
-    default: break;
+  if constexpr (LOGK == 15) {
+    switch (mode) {
+      case K1_T_F32: return launch_tc256<K1_T_F32>(x, M, out, scales, err, w, s);
+      case K1_Q4_PACKED: return launch_tc256<K1_Q4_PACKED>(x, M, out, scales, err, w, s);
+      case K1_Q4_I8: return launch_tc256<K1_Q4_I8>(x, M, out, scales, err, w, s);
+      case K1_Q8_I8: return launch_tc256<K1_Q8_I8>(x, M, out, scales, err, w, s);
+      default: return cudaErrorInvalidValue;
+    }
+  } else {
+    switch (mode) {
+      case K1_T_F32: return launch_tc<LOGK, K1_T_F32>(x, M, out, scales, err, w, s);
+      case K1_Q4_PACKED: return launch_tc<LOGK, K1_Q4_PACKED>(x, M, out, scales, err, w, s);
+      case K1_Q4_I8: return launch_tc<LOGK, K1_Q4_I8>(x, M, out, scales, err, w, s);
+      case K1_Q8_I8: return launch_tc<LOGK, K1_Q8_I8>(x, M, out, scales, err, w, s);
+      default: break;
+    }
   }
   return cudaErrorInvalidValue;
 }
@@ -730,7 +1108,7 @@ cudaError_t launch_tc_mode(const void* x, int64_t M, K1Mode mode, void* out, flo
 }  // namespace
 
 bool ln_fht_quant_tc_supports(bool in_bf16, int log2k, K1Mode mode, const void* x, const void* out) {
-  return in_bf16 && log2k >= 7 && log2k <= 14 && mode != K1_FHT_F32 &&
+  return in_bf16 && log2k >= 7 && log2k <= 15 && mode != K1_FHT_F32 &&
          (reinterpret_cast<uintptr_t>(x) & 15u) == 0 && (reinterpret_cast<uintptr_t>(out) & 15u) == 0;
 }
 
@@ -750,6 +1128,7 @@ cudaError_t launch_tc_any(const void* x, int64_t M, int log2k, K1Mode mode, void
     case 12: return launch_tc_mode<12>(x, M, mode, out, scales, err, w, stream);
     case 13: return launch_tc_mode<13>(x, M, mode, out, scales, err, w, stream);
     case 14: return launch_tc_mode<14>(x, M, mode, out, scales, err, w, stream);
+    case 15: return launch_tc_mode<15>(x, M, mode, out, scales, err, w, stream);
   }
   return cudaErrorInvalidValue;
 }

@@ -33,14 +33,26 @@ def unpack_nibbles(p, K):
     return out
 
 
+# A float transform rounds every output at least once, and two implementations
+# that order the roundings differently (the kernels and the oracle) differ by
+# a few units in the last place of the value itself.  For a row whose energy
+# sits in one element (e.g. an alternating row, whose transform is a single
+# spike sqrt(K) rms), 1e-5 rms is below one ulp of that element once
+# sqrt(K) > 1e-5 / 2^-24, i.e. at K = 32768; the elementwise bound therefore
+# also allows 4 ulp (2^-21 relative) of the element.
+T_ELEM_ULP = 2.0 ** -21
+
+
 def check_t(t_gpu, t64, rel=1e-5):
-    """Post-transform float values: per row ||dt||/||t|| <= rel and max|dt| <= rel * rms(t)."""
+    """Post-transform float values: per row ||dt||/||t|| <= rel, and every
+    element within rel * rms(t) + 4 ulp of itself."""
     d = t_gpu.astype(np.float64) - t64
     nrm = np.linalg.norm(t64, axis=1)
     rms = nrm / math.sqrt(t64.shape[1])
     nz = nrm > 0
     assert np.all(np.linalg.norm(d, axis=1)[nz] <= rel * nrm[nz]), np.max(np.linalg.norm(d, axis=1)[nz] / nrm[nz])
-    assert np.all(np.abs(d).max(axis=1)[nz] <= rel * rms[nz]), np.max(np.abs(d).max(axis=1)[nz] / rms[nz])
+    bound = rel * rms[:, None] + T_ELEM_ULP * np.abs(t64)
+    assert np.all((np.abs(d) <= bound)[nz]), np.max((np.abs(d) / bound)[nz])
     assert np.all(np.abs(t_gpu[~nz]) == 0)
 
 

@@ -1,6 +1,7 @@
 """GPU parity of the tensor-core split of the fused LN -> Hadamard -> quantize
-kernel (bf16 input, K in [128, 16384]): the high Hadamard factor as a tcgen05
-MMA, the low 6 stages (7 at K = 16384) in registers.
+kernel (bf16 input, K in [128, 32768]): the high Hadamard factor as a tcgen05
+MMA, the low 6 stages (7 at K = 16384, 8 at K = 32768, the last one or two
+through TMEM exchanges between warpgroups) in registers.
 
 The shapes here run many tiles per CTA (every shared-memory stage and TMEM
 accumulator is reused several times) with a ragged last tile, and the inputs
@@ -33,15 +34,15 @@ def H():
 
 def many_tile_rows(K, groups_per_cta=9, extra_rows=3):
     """Rows giving about groups_per_cta MMA groups (256 chunk rows of 64
-    columns, or 128 of 128 at K = 16384) per CTA on a full GPU, plus a ragged
-    last group."""
-    chunk = 128 if K >= 16384 else 64
+    columns; 128 of 128 at K = 16384; 128 of 256 at K = 32768) per CTA on a
+    full GPU, plus a ragged last group."""
+    chunk = 256 if K >= 32768 else (128 if K >= 16384 else 64)
     group_chunks = 128 if K >= 16384 else 256
     kh = K // chunk
     return (group_chunks * SMS * groups_per_cta) // kh + extra_rows
 
 
-@pytest.mark.parametrize("K", [128, 2048, 16384])
+@pytest.mark.parametrize("K", [128, 2048, 16384, 32768])
 def test_tc_many_tiles(H, orc, K):
     M = many_tile_rows(K)
     wl = WORKLOADS["sweep"].with_shape(M, K, 256)
@@ -66,7 +67,7 @@ def test_tc_many_tiles(H, orc, K):
     assert np.array_equal(to_host(scales_i8), s4)
 
 
-@pytest.mark.parametrize("K", [128, 256, 4096, 16384])
+@pytest.mark.parametrize("K", [128, 256, 4096, 16384, 32768])
 def test_tc_large_row_offset_bf16(H, orc, K):
     """bf16 rows with a mean far above the spread keep 1e-5 accuracy."""
     rng = np.random.default_rng(K + 11)
@@ -77,7 +78,7 @@ def test_tc_large_row_offset_bf16(H, orc, K):
 
 
 @pytest.mark.parametrize("bits", [4, 8])
-@pytest.mark.parametrize("K", [128, 1024, 16384])
+@pytest.mark.parametrize("K", [128, 1024, 16384, 32768])
 def test_tc_constant_and_zero_rows_bf16(H, orc, K, bits):
     x = np.zeros((5, K), np.float32)
     x[1] = 3.25
@@ -102,7 +103,7 @@ def test_tc_constant_and_zero_rows_bf16(H, orc, K, bits):
 
 def test_tc_single_row_and_partial_tile(H, orc):
     """M * K / 128 below one tile (1 row of K = 4096 is 32 of 128 chunk rows)."""
-    for M, K in [(1, 4096), (3, 128), (1, 16384), (2, 8192)]:
+    for M, K in [(1, 4096), (3, 128), (1, 16384), (2, 8192), (1, 32768), (3, 32768)]:
         wl = WORKLOADS["sweep"].with_shape(M, K, 256)
         x = make_x(wl)
         xd = to_device(x)
