@@ -37,7 +37,9 @@ cudaError_t launch_ln_fht_quant_tc(const void* x, int64_t M, int log2k, K1Mode m
                                    cudaStream_t stream);
 // The same launch with the ternary weight widening (2-bit [N][K/4] -> int8
 // [N][K]) done by the kernel's two otherwise idle warps per CTA alongside
-// the transform (hbl_forward's first two stages in one kernel).
+// the transform (hbl_forward's first two stages in one kernel) when the
+// kernel has a CTA on every SM; for shorter batches the widening kernel runs
+// after it.
 cudaError_t launch_ln_fht_quant_tc_widen(const void* x, int64_t M, int log2k, K1Mode mode, void* out,
                                          float* scales, const uint8_t* packed, int64_t N, int64_t K, int8_t* w,
                                          cudaStream_t stream);

@@ -1143,11 +1143,19 @@ cudaError_t launch_ln_fht_quant_tc(const void* x, int64_t M, int log2k, K1Mode m
 cudaError_t launch_ln_fht_quant_tc_widen(const void* x, int64_t M, int log2k, K1Mode mode, void* out,
                                          float* scales, const uint8_t* packed, int64_t N, int64_t K, int8_t* w,
                                          cudaStream_t stream) {
+  // The widening needs every SM's idle warps: with fewer CTAs than SMs (a
+  // short batch) it runs as its own kernel instead.
+  const int64_t kh = log2k >= 15 ? 128 : (int64_t)1 << (log2k - (log2k >= 14 ? 7 : 6));
+  const int64_t ctas = log2k >= 14 ? M : (M * kh + 2 * kBoxRows - 1) / (2 * kBoxRows);
+  if (M <= 0 || ctas < sm100_host::sm_count()) {
+    cudaError_t e = launch_tc_any(x, M, log2k, mode, out, scales, WidenJob(), stream);
+    if (e == cudaSuccess) e = launch_widen_ternary(packed, N, K, w, stream);
+    return e;
+  }
   WidenJob job;
   job.packed = reinterpret_cast<const uint32_t*>(packed);
   job.out = reinterpret_cast<uint4*>(w);
   job.words = N * K / 16;
-  if (M <= 0) return launch_widen_ternary(packed, N, K, w, stream);
   return launch_tc_any(x, M, log2k, mode, out, scales, job, stream);
 }
 
