@@ -60,8 +60,11 @@ cudaError_t launch_pack_ternary(const void* W, bool in_bf16, int64_t N, int64_t 
                                 float* alpha, double* partials, cudaStream_t stream);
 
 // 2-bit ternary codes [N][K/4] -> int8 codes [N][K] for the tensor cores.
-cudaError_t launch_widen_ternary(const uint8_t* packed, int64_t N, int64_t K, int8_t* out,
-                                 cudaStream_t stream);
+// With overlap_previous the kernel is a programmatic dependent of the
+// previous kernel of the stream (which it does not read from): it runs
+// alongside it and completes only after it.
+cudaError_t launch_widen_ternary(const uint8_t* packed, int64_t N, int64_t K, int8_t* out, cudaStream_t stream,
+                                 bool overlap_previous = false);
 
 // tcgen05 int8 GEMM: acc[m][n] = sum_k A[m][k] B[n][k].  Epilogue: either the
 // raw int32 (y_mode 0) or y = (float)acc * (scales[m] * alpha[0]) as float

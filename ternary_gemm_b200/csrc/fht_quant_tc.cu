@@ -1149,7 +1149,7 @@ cudaError_t launch_ln_fht_quant_tc_widen(const void* x, int64_t M, int log2k, K1
   const int64_t ctas = log2k >= 14 ? M : (M * kh + 2 * kBoxRows - 1) / (2 * kBoxRows);
   if (M <= 0 || ctas < sm100_host::sm_count()) {
     cudaError_t e = launch_tc_any(x, M, log2k, mode, out, scales, WidenJob(), stream);
-    if (e == cudaSuccess) e = launch_widen_ternary(packed, N, K, w, stream);
+    if (e == cudaSuccess) e = launch_widen_ternary(packed, N, K, w, stream, /*overlap_previous=*/true);
     return e;
   }
   WidenJob job;

@@ -163,7 +163,7 @@ hbl_status hbl_forward(const void* x, hbl_dtype xt, int64_t M, int64_t K, const 
     e = hbl::launch_ln_fht_quant_tc_widen(x, M, l, mode, A, scales, packed, N, K, B, stream);
   } else {
     e = hbl::launch_ln_fht_quant(x, xt == HBL_BF16, M, l, mode, A, scales, stream);
-    if (e == cudaSuccess) e = hbl::launch_widen_ternary(packed, N, K, B, stream);
+    if (e == cudaSuccess) e = hbl::launch_widen_ternary(packed, N, K, B, stream, /*overlap_previous=*/true);
   }
   if (e == cudaSuccess) e = hbl::launch_gemm_i8(A, B, M, N, K, yt == HBL_BF16 ? 2 : 1, y, scales, alpha_dev, stream);
   return cuda_status(e);

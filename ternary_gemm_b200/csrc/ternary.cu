@@ -112,6 +112,11 @@ __global__ void __launch_bounds__(kThreads)
 widen_kernel(const uint32_t* __restrict__ packed, int64_t nwords, uint4* __restrict__ out) {
   for (int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x; i < nwords; i += (int64_t)gridDim.x * kThreads)
     out[i] = tern::widen16(__ldg(packed + i));
+  // Launched as a programmatic dependent of the quantizer kernel (it reads
+  // nothing that kernel writes, so it runs alongside it): finishing only
+  // after that kernel has finished lets the next kernel of the stream rely on
+  // both.  A no-op for an ordinary launch.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
 int grid_for(int64_t work) {
@@ -141,11 +146,20 @@ cudaError_t launch_pack_ternary(const void* W, bool in_bf16, int64_t N, int64_t 
   return cudaGetLastError();
 }
 
-cudaError_t launch_widen_ternary(const uint8_t* packed, int64_t N, int64_t K, int8_t* out, cudaStream_t stream) {
+cudaError_t launch_widen_ternary(const uint8_t* packed, int64_t N, int64_t K, int8_t* out, cudaStream_t stream,
+                                 bool overlap_previous) {
   const int64_t nwords = N * K / 16;  // N K is a multiple of 1024 (K >= 64, N % 16 == 0)
-  widen_kernel<<<grid_for(nwords), kThreads, 0, stream>>>(reinterpret_cast<const uint32_t*>(packed), nwords,
-                                                          reinterpret_cast<uint4*>(out));
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid_for(nwords), 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = overlap_previous ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, widen_kernel, reinterpret_cast<const uint32_t*>(packed), nwords,
+                            reinterpret_cast<uint4*>(out));
 }
 
 }  // namespace hbl
