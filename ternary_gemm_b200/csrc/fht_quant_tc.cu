@@ -304,6 +304,32 @@ __device__ __forceinline__ uint4 codes32_s4(const float* y, float r) {
   return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
+// Warps 2-3 (w = 0, 1) widen the ternary weights to int8 for hbl_forward's
+// GEMM (its next stage; the issue-bound epilogue leaves slots to spare).  Only
+// 64 threads per SM do it, so each keeps two 16-byte loads (128 codes) in
+// flight; every warp store covers 2 KB of contiguous output.
+__device__ __forceinline__ void widen_in_idle_warps(const TcParams& p, int w, int lane) {
+  constexpr int kU = 2;
+  const uint4* src = reinterpret_cast<const uint4*>(p.wpacked);
+  const int64_t n4 = p.wwords / 4;  // 64 codes per uint4
+  const int64_t stride = (int64_t)gridDim.x * 64;
+  for (int64_t i = (int64_t)blockIdx.x * 64 + w * 32 + lane; i < n4; i += stride * kU) {
+    uint4 v[kU];
+#pragma unroll
+    for (int u = 0; u < kU; ++u) v[u] = i + u * stride < n4 ? __ldg(src + i + u * stride) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      if (i + u * stride < n4) {
+        uint4* d = p.wout + 4 * (i + u * stride);
+        d[0] = tern::widen16(v[u].x);
+        d[1] = tern::widen16(v[u].y);
+        d[2] = tern::widen16(v[u].z);
+        d[3] = tern::widen16(v[u].w);
+      }
+    }
+  }
+}
+
 template <int LOGK, int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
 ln_fht_quant_tc_kernel(const __grid_constant__ CUtensorMap tmX, TcParams p) {
@@ -356,8 +382,13 @@ ln_fht_quant_tc_kernel(const __grid_constant__ CUtensorMap tmX, TcParams p) {
   fence_before();
   __syncthreads();
   fence_after();
-  // a programmatic dependent of this kernel may start now (it waits for this
-  // kernel's results itself before reading them)
+  // Launched as a programmatic dependent, the setup above overlapped the
+  // previous kernel's tail; global memory is touched only after that kernel
+  // completes (x may be its output, the codes and weights its input).  Only
+  // then may this kernel's own dependents start (they wait for this kernel's
+  // results themselves): a trigger before the wait would let them run beside
+  // the kernel before this one.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   if (warp < 4) {
@@ -420,29 +451,7 @@ ln_fht_quant_tc_kernel(const __grid_constant__ CUtensorMap tmX, TcParams p) {
         }
       }
     } else {
-      // ---------------------------------------------- warps 2-3: weight widening
-      // (hbl_forward's next stage; the epilogue leaves issue slots to spare).
-      // Only 64 threads per SM do it, so each keeps two 16-byte loads (128
-      // codes) in flight; every warp store covers 2 KB of contiguous output.
-      constexpr int kU = 2;
-      const uint4* src = reinterpret_cast<const uint4*>(p.wpacked);
-      const int64_t n4 = p.wwords / 4;  // 64 codes per uint4
-      const int64_t stride = (int64_t)gridDim.x * 64;
-      for (int64_t i = (int64_t)blockIdx.x * 64 + (warp - 2) * 32 + lane; i < n4; i += stride * kU) {
-        uint4 v[kU];
-#pragma unroll
-        for (int u = 0; u < kU; ++u) v[u] = i + u * stride < n4 ? __ldg(src + i + u * stride) : make_uint4(0u, 0u, 0u, 0u);
-#pragma unroll
-        for (int u = 0; u < kU; ++u) {
-          if (i + u * stride < n4) {
-            uint4* d = p.wout + 4 * (i + u * stride);
-            d[0] = tern::widen16(v[u].x);
-            d[1] = tern::widen16(v[u].y);
-            d[2] = tern::widen16(v[u].z);
-            d[3] = tern::widen16(v[u].w);
-          }
-        }
-      }
+      widen_in_idle_warps(p, warp - 2, lane);
     }
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kEpiRegs));
@@ -773,6 +782,7 @@ ln_fht_quant_tc256_kernel(const __grid_constant__ CUtensorMap tmX, TcParams p) {
   __syncthreads();
   fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  asm volatile("griddepcontrol.wait;" ::: "memory");  // as in ln_fht_quant_tc_kernel
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   if (warp < 4) {
@@ -827,26 +837,7 @@ ln_fht_quant_tc256_kernel(const __grid_constant__ CUtensorMap tmX, TcParams p) {
         }
       }
     } else {
-      // warps 2-3: weight widening for hbl_forward's GEMM (see the main kernel)
-      constexpr int kU = 2;
-      const uint4* src = reinterpret_cast<const uint4*>(p.wpacked);
-      const int64_t n4 = p.wwords / 4;
-      const int64_t stride = (int64_t)gridDim.x * 64;
-      for (int64_t i = (int64_t)blockIdx.x * 64 + (warp - 2) * 32 + lane; i < n4; i += stride * kU) {
-        uint4 v[kU];
-#pragma unroll
-        for (int u = 0; u < kU; ++u) v[u] = i + u * stride < n4 ? __ldg(src + i + u * stride) : make_uint4(0u, 0u, 0u, 0u);
-#pragma unroll
-        for (int u = 0; u < kU; ++u) {
-          if (i + u * stride < n4) {
-            uint4* dd = p.wout + 4 * (i + u * stride);
-            dd[0] = tern::widen16(v[u].x);
-            dd[1] = tern::widen16(v[u].y);
-            dd[2] = tern::widen16(v[u].z);
-            dd[3] = tern::widen16(v[u].w);
-          }
-        }
-      }
+      widen_in_idle_warps(p, warp - 2, lane);
     }
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kEpiRegs));
@@ -1040,8 +1031,7 @@ cudaError_t launch_tc(const void* x, int64_t M, void* out, float* scales, int* e
   if (e != cudaSuccess) return e;
   const int nsm = sm100_host::sm_count();
   const int grid = p.num_groups < nsm ? p.num_groups : nsm;
-  kern<<<grid, kThreads, kSmemBytes, stream>>>(tmX, p);
-  return cudaGetLastError();
+  return sm100_host::launch_pdl(kern, (unsigned)grid, kThreads, kSmemBytes, stream, 1, tmX, p);
 }
 
 template <int MODE>
@@ -1078,8 +1068,7 @@ cudaError_t launch_tc256(const void* x, int64_t M, void* out, float* scales, int
   if (e != cudaSuccess) return e;
   const int nsm = sm100_host::sm_count();
   const int grid = p.num_groups < nsm ? p.num_groups : nsm;
-  kern<<<grid, kThreads, k256SmemBytes, stream>>>(tmX, p);
-  return cudaGetLastError();
+  return sm100_host::launch_pdl(kern, (unsigned)grid, kThreads, k256SmemBytes, stream, 1, tmX, p);
 }
 
 template <int LOGK>
@@ -1145,8 +1134,7 @@ cudaError_t launch_ln_fht_quant_tc_widen(const void* x, int64_t M, int log2k, K1
                                          cudaStream_t stream) {
   // The widening needs every SM's idle warps: with fewer CTAs than SMs (a
   // short batch) it runs as its own kernel instead.
-  const int64_t kh = log2k >= 15 ? 128 : (int64_t)1 << (log2k - (log2k >= 14 ? 7 : 6));
-  const int64_t ctas = log2k >= 14 ? M : (M * kh + 2 * kBoxRows - 1) / (2 * kBoxRows);
+  const int64_t ctas = log2k >= 14 ? M : (M * ((int64_t)1 << (log2k - 6)) + 2 * kBoxRows - 1) / (2 * kBoxRows);
   if (M <= 0 || ctas < sm100_host::sm_count()) {
     cudaError_t e = launch_tc_any(x, M, log2k, mode, out, scales, WidenJob(), stream);
     if (e == cudaSuccess) e = launch_widen_ternary(packed, N, K, w, stream, /*overlap_previous=*/true);

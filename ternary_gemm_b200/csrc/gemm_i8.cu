@@ -134,6 +134,12 @@ gemm_i8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   __syncthreads();
   fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // Launched as a programmatic dependent, the setup above overlapped the
+  // previous kernel's tail; its results (the codes, the weights) are read
+  // only after this wait, and this kernel's own dependents may start only
+  // after it (so none of them runs beside the kernel before this one).
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   if (warp == 0) {
     // ------------------------------------------------ TMA producer
@@ -432,6 +438,8 @@ gemm_i8_2sm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
   cluster_sync_all();
   fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  asm volatile("griddepcontrol.wait;" ::: "memory");  // as in gemm_i8_kernel
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   if (warp == 0) {
     if (lane == 0) {
@@ -575,28 +583,14 @@ cudaError_t launch_gemm_i8(const int8_t* A, const int8_t* B, int64_t M, int64_t 
     if (e != cudaSuccess) return e;
     const int pairs = sm_count() / 2;
     const int nclusters = p.num_tiles < pairs ? p.num_tiles : pairs;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(2 * nclusters), 1, 1);
-    cfg.blockDim = dim3(kThreads, 1, 1);
-    cfg.dynamicSmemBytes = k2SmemBytes;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, gemm_i8_2sm_kernel, ta, tb2, p);
-    if (e != cudaSuccess) return e;
-    return cudaGetLastError();
+    return sm100_host::launch_pdl(gemm_i8_2sm_kernel, (unsigned)(2 * nclusters), kThreads, k2SmemBytes, stream, 2,
+                                  ta, tb2, p);
   }
   static bool smem_set[sm100_host::kMaxDevices] = {false};
   cudaError_t e = sm100_host::ensure_smem(gemm_i8_kernel, (int)kSmemBytes, smem_set);
   if (e != cudaSuccess) return e;
   const int grid = p.num_tiles < sm_count() ? p.num_tiles : sm_count();
-  gemm_i8_kernel<<<grid, kThreads, kSmemBytes, stream>>>(ta, tb, p);
-  return cudaGetLastError();
+  return sm100_host::launch_pdl(gemm_i8_kernel, (unsigned)grid, kThreads, kSmemBytes, stream, 1, ta, tb, p);
 }
 
 int* device_error_word() {

@@ -265,5 +265,37 @@ inline cudaError_t ensure_smem(Kernel kern, int bytes, bool (&done)[kMaxDevices]
   return e;
 }
 
+// Launch as a programmatic dependent of the stream's previous kernel: the
+// grid may be scheduled once that kernel's blocks have all issued
+// griddepcontrol.launch_dependents (or exited), so this kernel's setup
+// overlaps the other's tail.  The kernel itself must execute
+// griddepcontrol.wait before it touches memory the previous kernel reads or
+// writes.  `cluster` > 1 adds a cluster dimension.
+template <typename Kernel, typename... Args>
+inline cudaError_t launch_pdl(Kernel kern, unsigned grid, unsigned block, size_t smem, cudaStream_t stream,
+                              unsigned cluster, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid, 1, 1);
+  cfg.blockDim = dim3(block, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  unsigned n = 1;
+  if (cluster > 1) {
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = cluster;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    n = 2;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, args...);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
 }  // namespace sm100_host
 }  // namespace hbl
