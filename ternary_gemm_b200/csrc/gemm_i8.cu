@@ -12,8 +12,10 @@
 // they reach this kernel (sm_100 has no int4 or ternary integer MMA); int8
 // products accumulate exactly in int32 (|acc| <= 127 * 32768 < 2^31).
 //
-// Two variants share the helpers below: the 2-SM kernel (M >= 256, described
-// above gemm_i8_2sm_kernel) and this 1-SM kernel for short M.
+// Three variants share the helpers below: the 2-SM kernel (M >= 256, described
+// above gemm_i8_2sm_kernel), this 1-SM kernel for short M, and its split-K
+// form for short M with few output tiles (described above
+// gemm_i8_splitk_kernel).
 //
 // 1-SM design (one CTA per SM, persistent over 128 x 256 output tiles):
 //   warp 0      TMA producer: 128-byte-swizzled boxes of A (128 x 128 B) and
@@ -545,6 +547,232 @@ gemm_i8_2sm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
   }
 }
 
+// ---------------------------------------------------------------- split-K variant
+// Short batches with few output tiles (M < 256 and fewer than half as many
+// 128 x 256 tiles as SMs) leave most SMs idle and give each CTA the whole K
+// loop.  Here a cluster of S CTAs (S = 2, 4 or 8) shares one tile and splits
+// its k-blocks: rank r runs the same TMA / MMA pipeline as the 1-SM kernel
+// over k-blocks [r num_kb / S, (r + 1) num_kb / S) into one 256-column TMEM
+// accumulator, and its epilogue warps copy the int32 partial into the
+// CTA's own (now idle) stage ring: 128 rows of 256 words, rows padded to
+// 1040 bytes so that a warp's 16-byte stores of 32 rows spread over the
+// banks.  Then rank r sums the S partials of columns [256 r / S, 256 (r + 1)
+// / S) through distributed shared memory (ld.shared::cluster) and applies
+// the same dequantisation as the other kernels; the int32 sums are exact, so
+// y is identical.  Two cluster barrier phases separate writing the partials,
+// reading them and leaving; every bounded wait of the pipeline comes before
+// them, so each thread reaches both.
+constexpr int kSplitMax = 8;
+constexpr int kPartRowBytes = 256 * 4 + 16;
+constexpr uint32_t kSplitTmemCols = 256;
+static_assert(128 * kPartRowBytes <= kStages * kStageBytes, "partial must fit in the stage ring");
+
+// cluster-wide barrier phase: this thread's shared-memory writes are visible
+// to every CTA of the cluster after it, and its reads of other CTAs' shared
+// memory are complete before any of them passes the next one.  Every thread
+// of every CTA takes each phase once; every wait before it is bounded.
+__device__ __forceinline__ void cluster_phase() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ uint4 ld_cluster_v4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared::cluster.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(addr)
+               : "memory");
+  return v;
+}
+
+// y[row][col .. col + 3] from four int32 sums (col + 3 < N, 16-byte-aligned rows)
+__device__ __forceinline__ void store_y4(const Params& p, int row, int col, const int (&v)[4], float sa) {
+  if (p.y_mode == 0) {
+    *reinterpret_cast<int4*>(reinterpret_cast<int32_t*>(p.y) + (size_t)row * p.N + col) =
+        make_int4(v[0], v[1], v[2], v[3]);
+  } else if (p.y_mode == 1) {
+    float4 o;
+    o.x = __fmul_rn(__int2float_rn(v[0]), sa);
+    o.y = __fmul_rn(__int2float_rn(v[1]), sa);
+    o.z = __fmul_rn(__int2float_rn(v[2]), sa);
+    o.w = __fmul_rn(__int2float_rn(v[3]), sa);
+    __stcs(reinterpret_cast<float4*>(reinterpret_cast<float*>(p.y) + (size_t)row * p.N + col), o);
+  } else {
+    uint2 o;
+    o.x = bf16x2(__fmul_rn(__int2float_rn(v[0]), sa), __fmul_rn(__int2float_rn(v[1]), sa));
+    o.y = bf16x2(__fmul_rn(__int2float_rn(v[2]), sa), __fmul_rn(__int2float_rn(v[3]), sa));
+    __stcs(reinterpret_cast<uint2*>(reinterpret_cast<uint16_t*>(p.y) + (size_t)row * p.N + col), o);
+  }
+}
+
+template <int S>
+__global__ void __launch_bounds__(kThreads, 1)
+gemm_i8_splitk_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  uint8_t* sA = base;
+  uint8_t* sB = base + kStages * kABytes;
+  uint8_t* part = base;  // after the main loop: the int32 partial, 128 rows of kPartRowBytes
+  uint64_t* full = reinterpret_cast<uint64_t*>(base + kStages * kStageBytes);
+  uint64_t* empty = full + kStages;
+  uint64_t* tfull = empty + kStages;
+  uint64_t* drain = tfull + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int rank = (int)cluster_ctarank();
+  const int tile = blockIdx.x / S;
+  const int m_blk = tile / p.num_n, n_blk = tile % p.num_n;
+  const int kb0 = rank * p.num_kb / S, kb1 = (rank + 1) * p.num_kb / S;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(tfull, 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, kSplitTmemCols);
+  fence_before();
+  __syncthreads();
+  fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  asm volatile("griddepcontrol.wait;" ::: "memory");  // as in gemm_i8_kernel
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+
+  if (warp == 0) {
+    if (lane == 0) {
+      prefetch_tensormap(&tmA);
+      prefetch_tensormap(&tmB);
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int kb = kb0; kb < kb1; ++kb) {
+        if (!wait_bounded(&empty[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
+        mbar_expect_tx(&full[stage], (uint32_t)kStageBytes);
+        tma_load_2d(sA + stage * kABytes, &tmA, kb * kBK, m_blk * kBM, &full[stage]);
+        tma_load_2d(sB + stage * kBBytes, &tmB, kb * kBK, n_blk * kBN, &full[stage]);
+        if (++stage == kStages) { stage = 0; phase ^= 1u; }
+      }
+      if (!ok) {
+        const uint64_t t0 = globaltimer();
+        while (globaltimer() - t0 < 20000000ull) {
+        }
+      }
+    }
+    __syncwarp();
+    cluster_phase();  // partials written
+    cluster_phase();  // partials read
+  } else if (warp == 1) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int kb = kb0; kb < kb1; ++kb) {
+        if (!wait_bounded(&full[stage], phase, abort_flag)) break;
+        fence_after();
+        const uint64_t a0 = sdesc(smem_u32(sA + stage * kABytes));
+        const uint64_t b0 = sdesc(smem_u32(sB + stage * kBBytes));
+#pragma unroll
+        for (int k = 0; k < kBK / 32; ++k)
+          mma_i8(tmem_base, a0 + (uint64_t)(2 * k), b0 + (uint64_t)(2 * k), (kb > kb0 || k > 0) ? 1u : 0u);
+        umma_commit(&empty[stage]);
+        if (++stage == kStages) { stage = 0; phase ^= 1u; }
+      }
+      umma_commit(tfull);
+      umma_commit(drain);
+      const uint64_t t0 = globaltimer();
+      while (!mbar_try_wait(drain, 0) && globaltimer() - t0 < 200000000ull) {
+      }
+    }
+    __syncwarp();
+    cluster_phase();
+    cluster_phase();
+  } else {
+    // ------------------------------------------------ epilogue (warps 2..5)
+    const int quarter = warp & 3;
+    const int et = threadIdx.x - 64;  // 0 .. 127
+    if (lane == 0) wait_bounded(tfull, 0, abort_flag);
+    __syncwarp();
+    fence_after();
+    // The partial's valid rows into shared memory (on a failed wait:
+    // whatever TMEM holds; the error word is set and the handshakes below
+    // still run).  Two TMEM loads in flight per wait.
+    const int rows = min(kBM, p.M - m_blk * kBM);
+    if (quarter * 32 < rows) {
+      const int prow = quarter * 32 + lane;
+      uint8_t* dst = part + (size_t)prow * kPartRowBytes;
+      const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16);
+#pragma unroll 1
+      for (int c = 0; c < 256; c += 64) {
+        uint32_t r[64];
+        tmem_ld32_nowait(tbase + (uint32_t)c, &r[0]);
+        tmem_ld32_nowait(tbase + (uint32_t)(c + 32), &r[32]);
+        tmem_wait_ld();
+        if (prow < rows) {
+#pragma unroll
+          for (int j = 0; j < 64; j += 4)
+            *reinterpret_cast<uint4*>(dst + 4 * (c + j)) = make_uint4(r[j], r[j + 1], r[j + 2], r[j + 3]);
+        }
+      }
+    }
+    cluster_phase();  // every rank's partial is in its shared memory
+    {
+      // This rank's columns, W = 256 / S, as 4-column groups over 128 rows:
+      // 64 / S groups per thread, taken GB at a time with the S loads of each
+      // group all issued before any is used (16 remote loads in flight per
+      // thread, so the distributed-shared-memory latency is paid 4 times).
+      constexpr int W = kBN / S;
+      constexpr int GPR = W / 4;        // groups per row
+      constexpr int GB = 16 / S;        // groups per batch and thread
+      const int total = rows * GPR;     // groups of the valid rows
+      const uint32_t part_u32 = smem_u32(part);
+#pragma unroll 1
+      for (int b = 0; b < total; b += 128 * GB) {
+        uint4 u[GB][S];
+#pragma unroll
+        for (int gi = 0; gi < GB; ++gi) {
+          const int g = b + 128 * gi + et;
+          if (g < total) {
+            const uint32_t off = part_u32 + (uint32_t)((g / GPR) * kPartRowBytes + 4 * (rank * W + 4 * (g % GPR)));
+#pragma unroll
+            for (int r = 0; r < S; ++r) u[gi][r] = ld_cluster_v4(mapa_shared(off, (uint32_t)r));
+          }
+        }
+#pragma unroll
+        for (int gi = 0; gi < GB; ++gi) {
+          const int g = b + 128 * gi + et;
+          if (g >= total) continue;
+          int v[4] = {0, 0, 0, 0};
+#pragma unroll
+          for (int r = 0; r < S; ++r) {
+            v[0] += (int)u[gi][r].x;
+            v[1] += (int)u[gi][r].y;
+            v[2] += (int)u[gi][r].z;
+            v[3] += (int)u[gi][r].w;
+          }
+          const int row = m_blk * kBM + g / GPR;
+          const int col = n_blk * kBN + rank * W + 4 * (g % GPR);
+          if (row < p.M && col < p.N) {
+            const float sa = p.y_mode != 0 ? __fmul_rn(__ldg(p.scales + row), __ldg(p.alpha)) : 0.0f;
+            store_y4(p, row, col, v, sa);
+          }
+        }
+      }
+    }
+    cluster_phase();  // no rank leaves while another still reads its partial
+  }
+
+  fence_before();
+  __syncthreads();
+  fence_after();
+  if (warp == 1) tmem_dealloc(tmem_base, kSplitTmemCols);
+}
+
 // 2-D K-major int8 tensor map: rows x K bytes, box kBK x box_rows, 128-byte swizzle.
 bool make_map(CUtensorMap* map, const void* ptr, int64_t rows, int64_t K, int box_rows) {
   return sm100_host::encode_2d(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, ptr, (uint64_t)K, (uint64_t)rows, (uint64_t)K,
@@ -552,6 +780,36 @@ bool make_map(CUtensorMap* map, const void* ptr, int64_t rows, int64_t K, int bo
 }
 
 int sm_count() { return sm100_host::sm_count(); }
+
+constexpr int kSplitMaxRows = 64;
+
+// clusters of `split` CTAs of `kern` that the device holds at once (cached
+// per device and cluster size; 0 when the query fails)
+template <typename Kernel>
+int max_active_clusters(Kernel kern, int split, int idx) {
+  static int cache[3][sm100_host::kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= sm100_host::kMaxDevices) return 0;
+  if (cache[idx][dev] > 0) return cache[idx][dev];
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)split, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)split;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return 0;
+  }
+  cache[idx][dev] = n;
+  return n;
+}
 
 }  // namespace
 
@@ -586,10 +844,28 @@ cudaError_t launch_gemm_i8(const int8_t* A, const int8_t* B, int64_t M, int64_t 
     return sm100_host::launch_pdl(gemm_i8_2sm_kernel, (unsigned)(2 * nclusters), kThreads, k2SmemBytes, stream, 2,
                                   ta, tb2, p);
   }
+  // A few rows and few tiles: split K over a cluster of S CTAs per tile, the
+  // largest S whose clusters all fit on the GPU at once.  (With more rows the
+  // partials' exchange through distributed shared memory costs more than the
+  // split saves.)
+  const int nsm = sm_count();
+  if (M <= kSplitMaxRows) {
+    for (int split = kSplitMax; split >= 2; split /= 2) {
+      if (split > p.num_kb || p.num_tiles * split > nsm) continue;
+      auto kern = split == 2 ? gemm_i8_splitk_kernel<2> : split == 4 ? gemm_i8_splitk_kernel<4> : gemm_i8_splitk_kernel<8>;
+      const int idx = split == 2 ? 0 : split == 4 ? 1 : 2;
+      static bool smem_set_s[3][sm100_host::kMaxDevices] = {};
+      cudaError_t e = sm100_host::ensure_smem(kern, (int)kSmemBytes, smem_set_s[idx]);
+      if (e != cudaSuccess) return e;
+      if (p.num_tiles > max_active_clusters(kern, split, idx)) continue;
+      return sm100_host::launch_pdl(kern, (unsigned)(p.num_tiles * split), kThreads, kSmemBytes, stream,
+                                    (unsigned)split, ta, tb, p);
+    }
+  }
   static bool smem_set[sm100_host::kMaxDevices] = {false};
   cudaError_t e = sm100_host::ensure_smem(gemm_i8_kernel, (int)kSmemBytes, smem_set);
   if (e != cudaSuccess) return e;
-  const int grid = p.num_tiles < sm_count() ? p.num_tiles : sm_count();
+  const int grid = p.num_tiles < nsm ? p.num_tiles : nsm;
   return sm100_host::launch_pdl(gemm_i8_kernel, (unsigned)grid, kThreads, kSmemBytes, stream, 1, ta, tb, p);
 }
 

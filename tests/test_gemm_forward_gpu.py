@@ -62,8 +62,11 @@ def test_widen_ternary_bit_exact(H, orc, N, K):
 # ----------------------------------------------------------------- int8 GEMM
 
 @pytest.mark.parametrize("M,N,K", [(1, 16, 16), (8, 256, 256), (128, 256, 128), (300, 272, 2048),
-                                   (257, 512, 4096), (64, 48, 208), (1000, 4096, 64), (129, 1040, 1024)])
+                                   (257, 512, 4096), (64, 48, 208), (1000, 4096, 64), (129, 1040, 1024),
+                                   (40, 4096, 4096), (60, 528, 1152), (33, 1040, 1024)])
 def test_gemm_exact(H, orc, M, N, K):
+    """Exact int32 sums.  Up to 64 rows with few tiles take the split-K cluster kernel (split 2 at K = 256 and
+    at the ragged K = 208, up to 8 elsewhere; k-blocks shared unevenly at K = 1152)."""
     rng = np.random.default_rng(M * 7 + N * 3 + K)
     A = rng.integers(-128, 128, (M, K)).astype(np.int8)
     B = rng.integers(-128, 128, (N, K)).astype(np.int8)
