@@ -55,6 +55,8 @@ def parse_args(argv=None):
     ap.add_argument("--sweep", choices=["k1", "fwd", "k1_noh"], default=None,
                     help="instead of the step line: the LN+FHT+INT4 kernel alone at M=65536 for each K, "
                          "or the whole forward at K=N=4096 for each M (one JSON line per point)")
+    ap.add_argument("--shape", default=None,
+                    help="with --sweep k1 or k1_noh: one point M,K instead of the sweep (e.g. for a profiler)")
     a = ap.parse_args(argv)
     a.warmup = max(3, a.warmup)
     return a
@@ -473,9 +475,14 @@ def bench_sweep(args):
         return sorted(ts)[2]
 
     if args.sweep in ("k1", "k1_noh"):
-        M = 65536
-        for K in SWEEP_K1_KS:
-            distinct = 4096                      # 4096 seeded rows, repeated to M on the device
+        M, ks = 65536, SWEEP_K1_KS
+        if args.shape:
+            M, K1 = (int(v) for v in args.shape.split(","))
+            ks = [K1]
+        for K in ks:
+            distinct = min(4096, M)              # seeded rows, repeated to M on the device
+            if M % distinct:
+                raise SystemExit("--shape: M must be a multiple of 4096 or below it")
             x = _to_device(make_x(base.with_shape(distinct, K, 256))).repeat(M // distinct, 1)
             codes = torch.empty((M, K // 2), dtype=torch.uint8, device="cuda")
             sc = torch.empty((M,), dtype=torch.float32, device="cuda")
@@ -488,7 +495,8 @@ def bench_sweep(args):
             name = "k1_ln_fht_int4" if args.sweep == "k1" else "ln_int4_no_transform"
             print(json.dumps({"sweep": name, "M": M, "K": K, "ms": t * 1e3, "GB/s": gbs,
                               "frac_hbm": gbs / peaks["hbm_gbs"], "peak_kind": peak_kind,
-                              "bytes_per_launch": nbytes, "input": "4096 seeded rows repeated to 65536"}),
+                              "bytes_per_launch": nbytes,
+                              "input": "%d seeded rows repeated to %d" % (distinct, M)}),
                   flush=True)
             del x, codes, sc
             torch.cuda.empty_cache()
