@@ -227,6 +227,48 @@ hbl_status hbl_forward_noalloc(const void* x, hbl_dtype xt, int64_t M, int64_t K
                                const float* alpha_dev, int64_t N, int bits, void* y, hbl_dtype yt,
                                cudaStream_t stream);
 
+/* ---------------------------------------------------------------- backward pass
+ * "BitNet v2: Native 4-bit Activations with Hadamard Transformation for 1-bit
+ * LLMs", training strategy: gradients bypass the non-differentiable
+ * quantizers (straight-through estimator) and are carried through the
+ * Hadamard transform by its orthogonality.  With the forward's t, (q, s) and
+ * (w, alpha) as in hbl_forward (y = (s q) (alpha w)^T) and u = LN(x):
+ *   g_t = alpha g_y w                    (the quantizer of t passed straight through)
+ *   g_u = H g_t / sqrt(K)                (H symmetric: the same scaled transform)
+ *   g_x = (g_u - mean(g_u) - u mean(g_u u)) / sqrt(var(x) + 1e-5)   (LayerNorm backward, no affine)
+ *   g_W = g_y^T (s q)                    (the ternary quantizer passed straight through)
+ * The products run on the tensor cores in bf16 with float accumulation: w and
+ * q are exact in bf16, g_y is used as given (rounded to bf16 first when it is
+ * float), and s g_y is rounded to bf16 once for g_W. */
+
+/* Workspace bytes of hbl_backward (0 for unsupported shapes). */
+size_t hbl_backward_workspace_bytes(int64_t M, int64_t K, int64_t N, int bits);
+
+/* x, M, K, packed, alpha_dev, N, bits as in hbl_forward (the forward's codes
+ * and scales are recomputed from x).  g_y device [M][N] of dtype gyt (16-byte
+ * aligned); outputs g_x device [M][K] of x's dtype and g_W device float
+ * [N][K] (both 16-byte aligned, caller-owned).  workspace device, 256-byte
+ * aligned, >= hbl_backward_workspace_bytes(M, K, N, bits) bytes.  Shape and
+ * argument errors as in hbl_forward. */
+hbl_status hbl_backward(const void* x, hbl_dtype xt, int64_t M, int64_t K, const uint8_t* packed,
+                        const float* alpha_dev, int64_t N, int bits, const void* g_y, hbl_dtype gyt, void* g_x,
+                        float* g_W, void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* The backward's products alone: D[r][c] = scale * sum_k A[r][k] B[k][c] on
+ * the tcgen05 tensor cores (bf16 operands, float accumulation).  A device
+ * bf16: a_mn = 0 stored [R][Kc] (K-major), a_mn = 1 stored [Kc][R]; B device
+ * bf16 stored [Kc][C]; D device float [R][C]; scale_dev a device float or
+ * NULL for 1.  All 16-byte aligned; C a multiple of 8, and R (a_mn = 1) or Kc
+ * (a_mn = 0) a multiple of 8 (HBL_ERR_UNSUPPORTED otherwise). */
+hbl_status hbl_gemm_bf16_f32(const uint16_t* A, int a_mn, const uint16_t* B, int64_t R, int64_t C, int64_t Kc,
+                             float* D, const float* scale_dev, cudaStream_t stream);
+
+/* The LayerNorm backward alone: g_x from x [M][K] (dtype xt) and g_u float
+ * [M][K], as in hbl_backward; g_x of x's dtype.  K a power of two in
+ * [64, 32768]; device pointers, 16-byte aligned. */
+hbl_status hbl_ln_backward(const void* x, hbl_dtype xt, int64_t M, int64_t K, const float* g_u, void* g_x,
+                           cudaStream_t stream);
+
 /* ---------------------------------------------------------------- test hooks */
 
 /* Stages 1-2 alone: t = H LN(x) / sqrt(K) as float [M][K] (device output).

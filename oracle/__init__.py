@@ -67,6 +67,8 @@ def _L():
             lib.orc_hadamard_entry.restype = i32
             lib.orc_layernorm_row.argtypes = [p, i64, p]
             lib.orc_layernorm_row.restype = None
+            lib.orc_ln_backward_row.argtypes = [p, p, i64, p]
+            lib.orc_ln_backward_row.restype = None
             lib.orc_fht_rows.argtypes = [p, i32, i64, i64, p, p]
             lib.orc_fht_rows.restype = i32
             lib.orc_rmsnorm_row.argtypes = [p, i64, p]
@@ -117,6 +119,16 @@ def layernorm_row(x: np.ndarray) -> np.ndarray:
     u = np.empty_like(x)
     _L().orc_layernorm_row(_ptr(x), x.size, _ptr(u))
     return u
+
+
+def ln_backward_row(x: np.ndarray, g_u: np.ndarray) -> np.ndarray:
+    """Gradient of a loss through LayerNorm (no affine, eps 1e-5) of one row, double:
+    g_x = (g_u - mean g_u - u mean(g_u u)) / sigma."""
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    g_u = np.ascontiguousarray(g_u, dtype=np.float64)
+    g_x = np.empty_like(x)
+    _L().orc_ln_backward_row(_ptr(x), _ptr(g_u), x.size, _ptr(g_x))
+    return g_x
 
 
 def fht_unnormalized(v: np.ndarray) -> np.ndarray:
@@ -310,3 +322,39 @@ def forward_rows(x: np.ndarray, w: np.ndarray, alpha, bits: int, rows=None):
     if rc != 0:
         raise ValueError("orc_forward_rows failed (%d)" % rc)
     return y, codes, scales
+
+
+def input_as_float64(x: np.ndarray) -> np.ndarray:
+    """float32 data or bf16 bit patterns (uint16) as double values."""
+    x, dt = _as_input(x)
+    return (bf16_bits_to_float(x) if dt == BF16 else x).astype(np.float64)
+
+
+def backward_act_rows(x: np.ndarray, w: np.ndarray, alpha, g_y: np.ndarray, rows=None):
+    """Activation gradient of the H-BitLinear forward under the straight-through
+    estimator (training strategy: the quantizers are bypassed, the gradient goes
+    through the Hadamard transform by its orthogonality), in double:
+
+        g_t = alpha g_y w          (d y / d t with the activation quantizer passed through)
+        g_u = H g_t / sqrt(K)      (t = H u / sqrt(K), H symmetric)
+        g_x = LayerNorm backward of g_u at x
+
+    x [M][K] float32 or bf16 bits, w int8 ternary [N][K], g_y [M][N] values.
+    Returns (g_x, g_u, g_t), double [nrows][K]; numpy's matmul is the product.
+    """
+    xv = input_as_float64(x)
+    M, K = xv.shape
+    rows = np.arange(M) if rows is None else np.asarray(rows)
+    gy = np.asarray(g_y, dtype=np.float64)[rows]
+    g_t = float(alpha) * (gy @ np.asarray(w, dtype=np.float64))
+    g_u = np.stack([fht_unnormalized(r) for r in g_t]) / np.sqrt(float(K))
+    g_x = np.stack([ln_backward_row(xv[m], g_u[i]) for i, m in enumerate(rows)])
+    return g_x, g_u, g_t
+
+
+def backward_weight(g_y: np.ndarray, codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    """Weight gradient under the straight-through estimator, double:
+    g_W = g_y^T (s q), the forward's dequantized activations (the ternary
+    quantizer passed through).  g_y [M][N], codes [M][K], scales [M]."""
+    a = np.asarray(codes, dtype=np.float64) * np.asarray(scales, dtype=np.float64)[:, None]
+    return np.asarray(g_y, dtype=np.float64).T @ a

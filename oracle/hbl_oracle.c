@@ -98,6 +98,30 @@ void orc_layernorm_row(const double* x, int64_t K, double* u) {
   for (int64_t i = 0; i < K; ++i) u[i] = (x[i] - mu) * inv;
 }
 
+/* LayerNorm backward of one row in double (no affine, eps 1e-5), the chain
+ * rule through u = (x - mu) / sigma with mu and sigma functions of x:
+ *   g_x = (g_u - mean(g_u) - u mean(g_u u)) / sigma
+ * ("the straight-through estimator approximates the gradient ... the
+ * Hadamard matrix's orthogonality transforms the gradient": everything before
+ * the transform is ordinary backpropagation). */
+void orc_ln_backward_row(const double* x, const double* gu, int64_t K, double* gx) {
+  double sum = 0.0;
+  for (int64_t i = 0; i < K; ++i) sum += x[i];
+  const double mu = sum / (double)K;
+  double ss = 0.0;
+  for (int64_t i = 0; i < K; ++i) ss += (x[i] - mu) * (x[i] - mu);
+  const double var = ss / (double)K;
+  const double inv = 1.0 / sqrt(var + ORC_EPS_LN); /* 1 / sigma */
+  double mg = 0.0, mgu = 0.0;
+  for (int64_t i = 0; i < K; ++i) {
+    mg += gu[i];
+    mgu += gu[i] * (x[i] - mu) * inv;
+  }
+  mg /= (double)K;
+  mgu /= (double)K;
+  for (int64_t i = 0; i < K; ++i) gx[i] = (gu[i] - mg - (x[i] - mu) * inv * mgu) * inv;
+}
+
 /* ------------------------------------------------------- Hadamard (Sylvester) */
 
 /* In-place unnormalised fast Walsh-Hadamard transform, natural (Sylvester)

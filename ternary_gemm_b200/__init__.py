@@ -70,6 +70,14 @@ def lib():
             L.hbl_forward.restype = i32
             L.hbl_fht.argtypes = [p, i32, i64, i64, p, p]
             L.hbl_fht.restype = i32
+            L.hbl_backward_workspace_bytes.argtypes = [i64, i64, i64, i32]
+            L.hbl_backward_workspace_bytes.restype = sz
+            L.hbl_backward.argtypes = [p, i32, i64, i64, p, p, i64, i32, p, i32, p, p, p, sz, p]
+            L.hbl_backward.restype = i32
+            L.hbl_gemm_bf16_f32.argtypes = [p, i32, p, i64, i64, i64, p, p, p]
+            L.hbl_gemm_bf16_f32.restype = i32
+            L.hbl_ln_backward.argtypes = [p, i32, i64, i64, p, p, p]
+            L.hbl_ln_backward.restype = i32
             L.hbl_pack_ternary_rotated_workspace_bytes.argtypes = [i64, i64]
             L.hbl_pack_ternary_rotated_workspace_bytes.restype = sz
             L.hbl_pack_ternary_rotated.argtypes = [p, i32, i64, i64, p, p, p, sz, p]
@@ -210,6 +218,54 @@ def hbl_forward(x, packed, alpha, N: int, bits: int, y=None, y_dtype=None, works
     _check(lib().hbl_forward(_ptr(x), _dtype_code(x), M, K, _ptr(packed), _ptr(alpha), N, bits, _ptr(y),
                              _dtype_code(y), _ptr(workspace), workspace.numel(), _stream(stream)), "hbl_forward")
     return y
+
+
+def hbl_backward_workspace_bytes(M: int, K: int, N: int, bits: int) -> int:
+    return int(lib().hbl_backward_workspace_bytes(M, K, N, bits))
+
+
+def hbl_backward(x, packed, alpha, N: int, bits: int, g_y, g_x=None, g_W=None, workspace=None, stream=None):
+    """Straight-through-estimator gradients of hbl_forward: (g_x [M][K] of x's dtype, g_W float32 [N][K])."""
+    torch = _torch()
+    _need_cuda(x, packed, alpha, g_y)
+    M, K = x.shape
+    if g_x is None:
+        g_x = torch.empty((M, K), dtype=x.dtype, device=x.device)
+    if g_W is None:
+        g_W = torch.empty((N, K), dtype=torch.float32, device=x.device)
+    if workspace is None:
+        workspace = torch.empty((hbl_backward_workspace_bytes(M, K, N, bits),), dtype=torch.uint8, device=x.device)
+    _check(lib().hbl_backward(_ptr(x), _dtype_code(x), M, K, _ptr(packed), _ptr(alpha), N, bits, _ptr(g_y),
+                              _dtype_code(g_y), _ptr(g_x), _ptr(g_W), _ptr(workspace), workspace.numel(),
+                              _stream(stream)), "hbl_backward")
+    return g_x, g_W
+
+
+def hbl_gemm_bf16_f32(A, B, a_mn: bool = False, scale=None, D=None, stream=None):
+    """D = scale * A B on the tensor cores.  A bf16 [R][Kc] (a_mn False) or [Kc][R] (a_mn True),
+    B bf16 [Kc][C], D float32 [R][C]; scale a device float32 [1] or None."""
+    torch = _torch()
+    _need_cuda(A, B)
+    Kc, C = B.shape
+    R = A.shape[1] if a_mn else A.shape[0]
+    if D is None:
+        D = torch.empty((R, C), dtype=torch.float32, device=A.device)
+    _check(lib().hbl_gemm_bf16_f32(_ptr(A), 1 if a_mn else 0, _ptr(B), R, C, Kc, _ptr(D),
+                                   _ptr(scale) if scale is not None else None, _stream(stream)),
+           "hbl_gemm_bf16_f32")
+    return D
+
+
+def hbl_ln_backward(x, g_u, g_x=None, stream=None):
+    """LayerNorm backward (no affine): g_x [M][K] of x's dtype from x and float32 g_u."""
+    torch = _torch()
+    _need_cuda(x, g_u)
+    M, K = x.shape
+    if g_x is None:
+        g_x = torch.empty((M, K), dtype=x.dtype, device=x.device)
+    _check(lib().hbl_ln_backward(_ptr(x), _dtype_code(x), M, K, _ptr(g_u), _ptr(g_x), _stream(stream)),
+           "hbl_ln_backward")
+    return g_x
 
 
 def hbl_fht(x, t=None, stream=None):

@@ -85,6 +85,16 @@ cudaError_t launch_gemv_ternary(const int8_t* A, const float* scales, const uint
 // Device error word (bounded-wait timeouts) -- lives in gemm_i8.cu; kernels in
 // other translation units receive its device address.
 int* device_error_word();
+
+// backward pass (gemm_bf16.cu, backward.cu)
+cudaError_t launch_gemm_bf16(const uint16_t* A, bool a_mn, const uint16_t* B, int64_t R, int64_t C, int64_t Kc,
+                             float* d, const float* scale, cudaStream_t stream);
+cudaError_t launch_ternary_to_bf16(const uint8_t* packed, int64_t N, int64_t K, uint16_t* out, cudaStream_t stream);
+cudaError_t launch_codes_to_bf16(const int8_t* q, int64_t count, uint16_t* out, cudaStream_t stream);
+cudaError_t launch_scale_rows_bf16(const void* g, bool g_bf16, const float* s, int64_t M, int64_t N, uint16_t* out,
+                                   cudaStream_t stream);
+cudaError_t launch_ln_backward(const void* x, bool x_bf16, const float* gu, int64_t M, int log2k, void* gx,
+                               cudaStream_t stream);
 // Records e as the thread's last CUDA error (hbl_last_cuda_error) and maps it
 // to a status: HBL_OK for cudaSuccess, else HBL_ERR_CUDA.
 hbl_status note_cuda_error(cudaError_t e);

@@ -72,6 +72,27 @@ ForwardLayout forward_layout(int64_t M, int64_t K, int64_t N) {
   return L;
 }
 
+// hbl_backward's workspace: codes int8 [M][K], scales [M], bf16 copies of
+// w [N][K], g_y [M][N], s g_y [M][N] and q [M][K], g_t and g_u f32 [M][K]
+struct BackwardLayout {
+  size_t q_off, s_off, w16_off, gy16_off, gys_off, q16_off, gt_off, gu_off, total;
+};
+
+BackwardLayout backward_layout(int64_t M, int64_t K, int64_t N) {
+  const size_t m = (size_t)M, k = (size_t)K, n = (size_t)N;
+  BackwardLayout L;
+  L.q_off = 0;
+  L.s_off = L.q_off + align256(m * k);
+  L.w16_off = L.s_off + align256(m * 4);
+  L.gy16_off = L.w16_off + align256(n * k * 2);
+  L.gys_off = L.gy16_off + align256(m * n * 2);
+  L.q16_off = L.gys_off + align256(m * n * 2);
+  L.gt_off = L.q16_off + align256(m * k * 2);
+  L.gu_off = L.gt_off + align256(m * k * 4);
+  L.total = L.gu_off + align256(m * k * 4);
+  return L;
+}
+
 }  // namespace
 
 namespace hbl {
@@ -311,6 +332,81 @@ hbl_status hbl_gemm_i8_i32(const int8_t* A, const int8_t* B, int64_t M, int64_t 
   if (s != HBL_OK) return s;
   if ((s = check_n(N)) != HBL_OK) return s;
   return cuda_status(hbl::launch_gemm_i8(A, B, M, N, K, 0, acc, nullptr, nullptr, stream));
+}
+
+size_t hbl_backward_workspace_bytes(int64_t M, int64_t K, int64_t N, int bits) {
+  int l;
+  if (check_k(K, &l) != HBL_OK || check_rows(M) != HBL_OK || check_n(N) != HBL_OK || (bits != 4 && bits != 8))
+    return 0;
+  return backward_layout(M, K, N).total;
+}
+
+hbl_status hbl_backward(const void* x, hbl_dtype xt, int64_t M, int64_t K, const uint8_t* packed,
+                        const float* alpha_dev, int64_t N, int bits, const void* g_y, hbl_dtype gyt, void* g_x,
+                        float* g_W, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  if (!x || !packed || !alpha_dev || !g_y || !g_x || !g_W || !dtype_ok(xt) || !dtype_ok(gyt) ||
+      (bits != 4 && bits != 8))
+    return HBL_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(packed, 16) || !aligned(alpha_dev, 4) || !aligned(g_y, 16) || !aligned(g_x, 16) ||
+      !aligned(g_W, 16))
+    return HBL_ERR_INVALID_ARG;
+  int l;
+  hbl_status s = check_k(K, &l);
+  if (s != HBL_OK) return s;
+  if ((s = check_rows(M)) != HBL_OK) return s;
+  if ((s = check_n(N)) != HBL_OK) return s;
+  const BackwardLayout L = backward_layout(M, K, N);
+  if (!workspace || !aligned(workspace, 256) || workspace_bytes < L.total) return HBL_ERR_WORKSPACE;
+  uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
+  int8_t* q = reinterpret_cast<int8_t*>(ws + L.q_off);
+  float* scales = reinterpret_cast<float*>(ws + L.s_off);
+  uint16_t* w16 = reinterpret_cast<uint16_t*>(ws + L.w16_off);
+  uint16_t* gy16 = reinterpret_cast<uint16_t*>(ws + L.gy16_off);
+  uint16_t* gys = reinterpret_cast<uint16_t*>(ws + L.gys_off);
+  uint16_t* q16 = reinterpret_cast<uint16_t*>(ws + L.q16_off);
+  float* gt = reinterpret_cast<float*>(ws + L.gt_off);
+  float* gu = reinterpret_cast<float*>(ws + L.gu_off);
+  const bool gy_bf16 = gyt == HBL_BF16;
+  const K1Mode mode = bits == 4 ? hbl::K1_Q4_I8 : hbl::K1_Q8_I8;
+  // the forward's codes and scales, recomputed
+  cudaError_t e = hbl::launch_ln_fht_quant(x, xt == HBL_BF16, M, l, mode, q, scales, stream);
+  // activation gradient: g_t = alpha g_y w, g_u = H g_t / sqrt(K), LayerNorm backward
+  if (e == cudaSuccess) e = hbl::launch_ternary_to_bf16(packed, N, K, w16, stream);
+  const uint16_t* gyb = reinterpret_cast<const uint16_t*>(g_y);
+  if (e == cudaSuccess && !gy_bf16) {
+    e = hbl::launch_scale_rows_bf16(g_y, false, nullptr, M, N, gy16, stream);
+    gyb = gy16;
+  }
+  if (e == cudaSuccess) e = hbl::launch_gemm_bf16(gyb, false, w16, M, K, N, gt, alpha_dev, stream);
+  if (e == cudaSuccess) e = hbl::launch_ln_fht_quant(gt, false, M, l, hbl::K1_FHT_F32, gu, nullptr, stream);
+  if (e == cudaSuccess) e = hbl::launch_ln_backward(x, xt == HBL_BF16, gu, M, l, g_x, stream);
+  // weight gradient: g_W = (s g_y)^T q
+  if (e == cudaSuccess) e = hbl::launch_scale_rows_bf16(g_y, gy_bf16, scales, M, N, gys, stream);
+  if (e == cudaSuccess) e = hbl::launch_codes_to_bf16(q, M * K, q16, stream);
+  if (e == cudaSuccess) e = hbl::launch_gemm_bf16(gys, true, q16, N, K, M, g_W, nullptr, stream);
+  return cuda_status(e);
+}
+
+hbl_status hbl_gemm_bf16_f32(const uint16_t* A, int a_mn, const uint16_t* B, int64_t R, int64_t C, int64_t Kc,
+                             float* D, const float* scale_dev, cudaStream_t stream) {
+  if (!A || !B || !D) return HBL_ERR_INVALID_ARG;
+  if (!aligned(A, 16) || !aligned(B, 16) || !aligned(D, 16) || (scale_dev && !aligned(scale_dev, 4)))
+    return HBL_ERR_INVALID_ARG;
+  if (R <= 0 || C <= 0 || Kc <= 0) return HBL_ERR_INVALID_ARG;
+  if (R > kMaxRows || C > kMaxRows || Kc > kMaxRows || C % 8 != 0 || (a_mn ? R % 8 : Kc % 8) != 0)
+    return HBL_ERR_UNSUPPORTED;
+  return cuda_status(hbl::launch_gemm_bf16(A, a_mn != 0, B, R, C, Kc, D, scale_dev, stream));
+}
+
+hbl_status hbl_ln_backward(const void* x, hbl_dtype xt, int64_t M, int64_t K, const float* g_u, void* g_x,
+                           cudaStream_t stream) {
+  if (!x || !g_u || !g_x || !dtype_ok(xt)) return HBL_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(g_u, 16) || !aligned(g_x, 16)) return HBL_ERR_INVALID_ARG;
+  int l;
+  hbl_status s = check_k(K, &l);
+  if (s != HBL_OK) return s;
+  if ((s = check_rows(M)) != HBL_OK) return s;
+  return cuda_status(hbl::launch_ln_backward(x, xt == HBL_BF16, g_u, M, l, g_x, stream));
 }
 
 hbl_status hbl_last_device_error(cudaStream_t stream) {

@@ -40,6 +40,15 @@ MUTANTS = [
      "out[m * (K / 2) + j] = (uint8_t)(hi | (lo << 4));"),
     ("ternary -1 encoded as 10", "unsigned f = (v == 0) ? 0u : (v == 1 ? 1u : 3u);",
      "unsigned f = (v == 0) ? 0u : (v == 1 ? 1u : 2u);"),
+    # the backward pass (tests/test_oracle_backward_pins.py)
+    ("LayerNorm backward without the mean term", "gx[i] = (gu[i] - mg - (x[i] - mu) * inv * mgu) * inv;",
+     "gx[i] = (gu[i] - (x[i] - mu) * inv * mgu) * inv;"),
+    ("LayerNorm backward projection sign", "gx[i] = (gu[i] - mg - (x[i] - mu) * inv * mgu) * inv;",
+     "gx[i] = (gu[i] - mg + (x[i] - mu) * inv * mgu) * inv;"),
+    ("LayerNorm backward missing 1/sigma", "gx[i] = (gu[i] - mg - (x[i] - mu) * inv * mgu) * inv;",
+     "gx[i] = (gu[i] - mg - (x[i] - mu) * inv * mgu);"),
+    ("LayerNorm backward unbiased variance", "const double var = ss / (double)K;",
+     "const double var = ss / (double)(K - 1);"),
 ]
 
 
@@ -55,7 +64,8 @@ def _run_mutant(m):
                        check=True)
         env = dict(os.environ, HBL_ORACLE_LIB=so)
         p = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
-                            os.path.join(ROOT, "tests", "test_oracle_pins.py")],
+                            os.path.join(ROOT, "tests", "test_oracle_pins.py"),
+                            os.path.join(ROOT, "tests", "test_oracle_backward_pins.py")],
                            env=env, capture_output=True, text=True, timeout=600)
         return name, p.returncode, p.stdout[-400:]
 
