@@ -52,7 +52,7 @@ def parse_args(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
-    ap.add_argument("--sweep", choices=["k1", "fwd", "k1_noh"], default=None,
+    ap.add_argument("--sweep", choices=["k1", "fwd", "k1_noh", "bwd"], default=None,
                     help="instead of the step line: the LN+FHT+INT4 kernel alone at M=65536 for each K, "
                          "or the whole forward at K=N=4096 for each M (one JSON line per point)")
     ap.add_argument("--shape", default=None,
@@ -474,6 +474,8 @@ def bench_sweep(args):
         del g
         return sorted(ts)[2]
 
+    if args.sweep == "bwd":
+        return bench_backward(args, hbl, peaks, peak_kind, timed)
     if args.sweep in ("k1", "k1_noh"):
         M, ks = 65536, SWEEP_K1_KS
         if args.shape:
@@ -516,6 +518,58 @@ def bench_sweep(args):
                               "us_gpu": tg * 1e6, "tokens/s_gpu": M / tg,
                               "timing": "us: eager calls back to back (host launch cost included); "
                                         "us_gpu: 20 calls captured in one CUDA graph, replayed"}), flush=True)
+    return 0
+
+
+def bench_backward(args, hbl, peaks, peak_kind, timed):
+    """The straight-through-estimator backward at the step workload (one JSON line):
+    tokens/s of hbl_backward, and the roofline of its dominant kernel, the bf16
+    tensor-core GEMM (two per call, 2 M N K flops each), timed alone through its
+    stage entry point against the measured bf16 peak."""
+    import numpy as np
+    import torch
+    from ternary_gemm_b200.inputs import WORKLOADS, make_w, make_x
+    wl = WORKLOADS[args.workload]
+    M, K, N = wl.M, wl.K, wl.N
+    reps = max(3, min(args.steps, 20))
+    x = _to_device(make_x(wl))
+    packed, alpha = hbl.hbl_pack_ternary(_to_device(make_w(wl)))
+    rng = np.random.default_rng(17)
+    gy = _to_device((rng.standard_normal((M, N)).astype(np.float32) * 0.01).view(np.uint32).__rshift__(16)
+                    .astype(np.uint16))
+    gx = torch.empty_like(x)
+    gW = torch.empty((N, K), dtype=torch.float32, device="cuda")
+    ws = torch.empty((hbl.hbl_backward_workspace_bytes(M, K, N, args.bits),), dtype=torch.uint8, device="cuda")
+    t = timed(lambda: hbl.hbl_backward(x, packed, alpha, N, args.bits, gy, g_x=gx, g_W=gW, workspace=ws), reps)
+    # stages alone (same shapes; operand values do not change the timing)
+    w16 = torch.randint(-1, 2, (N, K), device="cuda").to(torch.bfloat16)
+    q16 = torch.randint(-8, 8, (M, K), device="cuda").to(torch.bfloat16)
+    gt = torch.empty((M, K), dtype=torch.float32, device="cuda")
+    gu = torch.empty((M, K), dtype=torch.float32, device="cuda")
+    t_gt = timed(lambda: hbl.hbl_gemm_bf16_f32(gy, w16, scale=alpha, D=gt), reps)
+    t_gw = timed(lambda: hbl.hbl_gemm_bf16_f32(gy, q16, a_mn=True, D=gW), reps)
+    t_fht = timed(lambda: hbl.hbl_fht(gt, t=gu), reps)
+    t_lnb = timed(lambda: hbl.hbl_ln_backward(x, gu, g_x=gx), reps)
+    flops = 2.0 * M * N * K
+    gemm_t = min(t_gt, t_gw)
+    achieved = flops / gemm_t / 1e12
+    peak = peaks["bf16_tflops"]
+    esz = x.element_size()
+    print(json.dumps({
+        "sweep": "bwd", "metric": "H-BitLinear backward tokens/s (straight-through estimator)",
+        "value": M / t, "unit": "tokens/s", "ms": t * 1e3, "dtype": "bf16",
+        "config": {"workload": args.workload, "M": M, "K": K, "N": N, "bits": args.bits},
+        "roofline": {"bound": "tensor", "kernel": "gemm_bf16_2sm_kernel (tcgen05 kind::f16, cta_group::2)",
+                     "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                     "traffic": None, "peak_source": "%s bf16 burst" % peak_kind,
+                     "algorithmic_flops_per_launch": flops},
+        "stages_ms": {"gemm_g_t": t_gt * 1e3, "gemm_g_W": t_gw * 1e3, "fht_g_t": t_fht * 1e3,
+                      "ln_backward": t_lnb * 1e3},
+        "stage_gbs": {"fht_g_t": 8.0 * M * K / t_fht / 1e9,
+                      "ln_backward": (2.0 * esz + 4.0) * M * K / t_lnb / 1e9},
+        "hbm_gbs_peak": peaks["hbm_gbs"],
+        "data": "synthetic", "timing": "CUDA events, %d calls after 3 warm-ups, each stage alone" % reps}),
+        flush=True)
     return 0
 
 

@@ -44,7 +44,8 @@ def _bf16_values(bits):
 
 
 @pytest.mark.parametrize("a_mn", [False, True])
-@pytest.mark.parametrize("R,C,Kc", [(128, 256, 64), (136, 264, 72), (8, 16, 8), (120, 520, 200), (1024, 4096, 2048)])
+@pytest.mark.parametrize("R,C,Kc", [(128, 256, 64), (136, 264, 72), (8, 16, 8), (120, 520, 200), (1024, 4096, 2048),
+                                    (264, 264, 72), (520, 136, 200), (256, 512, 4096)])
 def test_gemm_bf16_exact_on_integer_operands(H, a_mn, R, C, Kc):
     import torch
     rng = np.random.default_rng(R * 31 + C * 7 + Kc + int(a_mn))
