@@ -64,7 +64,23 @@ struct BParams {
   float* d;
   const float* scale;  // device scalar, or null for 1
   int* err;            // device error word (bounded waits that gave up)
+  int col_major;       // tile order: rows fastest (1) or columns fastest (0)
 };
+
+// Output tile of a linear tile index.  The CTAs in flight at once take
+// consecutive indices; with rows fastest they share one B column panel and
+// cycle through all A row panels, with columns fastest the reverse.  The host
+// picks the order whose cycled operand is the smaller one, so that it stays in
+// L2 and the other streams from DRAM once.
+__device__ __forceinline__ void tile_coords(const BParams& p, int tile, int& r_blk, int& c_blk) {
+  if (p.col_major) {
+    r_blk = tile % p.num_r;
+    c_blk = tile / p.num_r;
+  } else {
+    r_blk = tile / p.num_c;
+    c_blk = tile % p.num_c;
+  }
+}
 
 template <bool A_MN>
 __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t accumulate) {
@@ -124,7 +140,8 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       uint32_t phase = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x) {
-        const int r_blk = tile / p.num_c, c_blk = tile % p.num_c;
+        int r_blk, c_blk;
+        tile_coords(p, tile, r_blk, c_blk);
         for (int kb = 0; kb < p.num_kb; ++kb) {
           if (!wait_bounded(&empty[stage], phase ^ 1u, abort_flag, p.err)) { ok = false; break; }
           mbar_expect_tx(&full[stage], (uint32_t)kStageBytes);
@@ -197,7 +214,8 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
       fence_after();
-      const int r_blk = tile / p.num_c, c_blk = tile % p.num_c;
+      int r_blk, c_blk;
+      tile_coords(p, tile, r_blk, c_blk);
       const int row = r_blk * kBM + quarter * 32 + lane;
       const uint32_t tbase = tmem_base + (uint32_t)(acc * kBN) + ((uint32_t)(quarter * 32) << 16);
 #pragma unroll 1
@@ -319,7 +337,8 @@ gemm_bf16_2sm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
       uint32_t phase = 0;
       bool ok = true;
       for (int tile = cid; tile < p.num_tiles && ok; tile += ncl) {
-        const int r_blk = tile / p.num_c, c_blk = tile % p.num_c;
+        int r_blk, c_blk;
+        tile_coords(p, tile, r_blk, c_blk);
         const int r0 = r_blk * 256 + (int)rank * 128;
         const int c0 = c_blk * 256 + (int)rank * 128;
         for (int kb = 0; kb < p.num_kb; ++kb) {
@@ -390,7 +409,8 @@ gemm_bf16_2sm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
       fence_after();
-      const int r_blk = tile / p.num_c, c_blk = tile % p.num_c;
+      int r_blk, c_blk;
+      tile_coords(p, tile, r_blk, c_blk);
       const int row = r_blk * 256 + (int)rank * 128 + quarter * 32 + lane;
       const uint32_t tbase = tmem_base + (uint32_t)(acc * 256) + ((uint32_t)(quarter * 32) << 16);
 #pragma unroll 1
@@ -470,6 +490,7 @@ cudaError_t launch_gemm_bf16(const uint16_t* A, bool a_mn, const uint16_t* B, in
   p.num_kb = (int)((Kc + kBKe - 1) / kBKe);
   p.d = d;
   p.scale = scale;
+  p.col_major = R <= C ? 1 : 0;  // A (R x Kc) the smaller operand: cycle it, stream B
   p.err = device_error_word();
   if (!p.err) return cudaErrorInvalidValue;
   const int nsm = sm100_host::sm_count();
