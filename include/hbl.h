@@ -1,5 +1,5 @@
 /*
- * hbl.h -- C ABI of the B200 (sm_100a) H-BitLinear forward library.
+ * hbl.h -- C ABI of the B200 (sm_100a) H-BitLinear forward (and backward) library.
  *
  * The layer is the H-BitLinear module of "BitNet v2: Native 4-bit
  * Activations with Hadamard Transformation for 1-bit LLMs" (arXiv 2504.18415;
@@ -268,6 +268,13 @@ hbl_status hbl_gemm_bf16_f32(const uint16_t* A, int a_mn, const uint16_t* B, int
  * [64, 32768]; device pointers, 16-byte aligned. */
 hbl_status hbl_ln_backward(const void* x, hbl_dtype xt, int64_t M, int64_t K, const float* g_u, void* g_x,
                            cudaStream_t stream);
+
+/* The transform and the LayerNorm backward of hbl_backward in one pass:
+ * g_x = LayerNorm backward at x of H g / sqrt(K), g float [M][K], x [M][K] of
+ * dtype xt, g_x [M][K] of x's dtype (device, 16-byte aligned).  K a power of
+ * two in [64, 32768]. */
+hbl_status hbl_fht_ln_backward(const float* g, const void* x, hbl_dtype xt, int64_t M, int64_t K, void* g_x,
+                               cudaStream_t stream);
 
 /* ---------------------------------------------------------------- test hooks */
 

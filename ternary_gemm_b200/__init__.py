@@ -78,6 +78,8 @@ def lib():
             L.hbl_gemm_bf16_f32.restype = i32
             L.hbl_ln_backward.argtypes = [p, i32, i64, i64, p, p, p]
             L.hbl_ln_backward.restype = i32
+            L.hbl_fht_ln_backward.argtypes = [p, p, i32, i64, i64, p, p]
+            L.hbl_fht_ln_backward.restype = i32
             L.hbl_pack_ternary_rotated_workspace_bytes.argtypes = [i64, i64]
             L.hbl_pack_ternary_rotated_workspace_bytes.restype = sz
             L.hbl_pack_ternary_rotated.argtypes = [p, i32, i64, i64, p, p, p, sz, p]
@@ -265,6 +267,18 @@ def hbl_ln_backward(x, g_u, g_x=None, stream=None):
         g_x = torch.empty((M, K), dtype=x.dtype, device=x.device)
     _check(lib().hbl_ln_backward(_ptr(x), _dtype_code(x), M, K, _ptr(g_u), _ptr(g_x), _stream(stream)),
            "hbl_ln_backward")
+    return g_x
+
+
+def hbl_fht_ln_backward(g, x, g_x=None, stream=None):
+    """g_x [M][K] (x's dtype) = LayerNorm backward at x of H g / sqrt(K), g float32 [M][K]."""
+    torch = _torch()
+    _need_cuda(g, x)
+    M, K = x.shape
+    if g_x is None:
+        g_x = torch.empty((M, K), dtype=x.dtype, device=x.device)
+    _check(lib().hbl_fht_ln_backward(_ptr(g), _ptr(x), _dtype_code(x), M, K, _ptr(g_x), _stream(stream)),
+           "hbl_fht_ln_backward")
     return g_x
 
 

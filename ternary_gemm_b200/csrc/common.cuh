@@ -18,6 +18,7 @@ enum K1Mode : int {
   K1_Q4_I8 = 2,      // INT4 absmean codes widened to one int8 per element
   K1_Q8_I8 = 3,      // INT8 absmax codes, one int8 per element
   K1_FHT_F32 = 4,    // the plain scaled transform H x / sqrt(K) as float (no LN, no quantizer)
+  K1_LNBWD = 5,      // backward: LayerNorm backward at x of H g / sqrt(K) (g float; register kernel only)
 };
 
 constexpr int kMinLogK = 6;   // K = 64
@@ -95,6 +96,9 @@ cudaError_t launch_scale_rows_bf16(const void* g, bool g_bf16, const float* s, i
                                    cudaStream_t stream);
 cudaError_t launch_ln_backward(const void* x, bool x_bf16, const float* gu, int64_t M, int log2k, void* gx,
                                cudaStream_t stream);
+// g_x = LayerNorm backward at x of H g / sqrt(K), in one pass (fht_quant.cu)
+cudaError_t launch_fht_ln_backward(const float* g, const void* x, bool x_bf16, int64_t M, int log2k, void* gx,
+                                   cudaStream_t stream);
 // Records e as the thread's last CUDA error (hbl_last_cuda_error) and maps it
 // to a status: HBL_OK for cudaSuccess, else HBL_ERR_CUDA.
 hbl_status note_cuda_error(cudaError_t e);

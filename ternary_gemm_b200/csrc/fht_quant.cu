@@ -37,6 +37,8 @@
 // which is exactly H LN(x) / sqrt(K) with the biased variance and no affine.
 #include <cstdint>
 
+#include <cuda_bf16.h>
+
 #include "common.cuh"
 #include "sm100.cuh"
 #include "quant.cuh"
@@ -191,10 +193,38 @@ __device__ __forceinline__ void store_pass1(const float (&e)[64], float* smem, c
 }
 
 // One CTA handles one group of R rows.
+// Sum of four floats over the T threads of a row (the RowReduce pattern with a
+// float4 slot per warp; every thread of the row ends with the same totals).
+template <int T, int WPR>
+__device__ __forceinline__ float4 row_sum4(float4 v, float4* red, int rl, int t) {
+  constexpr int W = T < 32 ? T : 32;
+#pragma unroll
+  for (int o = W / 2; o >= 1; o >>= 1) {
+    v.x += __shfl_xor_sync(0xffffffffu, v.x, o);
+    v.y += __shfl_xor_sync(0xffffffffu, v.y, o);
+    v.z += __shfl_xor_sync(0xffffffffu, v.z, o);
+    v.w += __shfl_xor_sync(0xffffffffu, v.w, o);
+  }
+  if constexpr (T > 32) {
+    if ((t & 31) == 0) red[rl * WPR + (t >> 5)] = v;
+    __syncthreads();
+    float4 s = red[rl * WPR];
+#pragma unroll
+    for (int w = 1; w < WPR; ++w) {
+      s.x += red[rl * WPR + w].x;
+      s.y += red[rl * WPR + w].y;
+      s.z += red[rl * WPR + w].z;
+      s.w += red[rl * WPR + w].w;
+    }
+    v = s;
+  }
+  return v;
+}
+
 template <int LOGK, bool BF16, int MODE>
 __global__ void __launch_bounds__(Shape<LOGK>::THREADS, Shape<LOGK>::MINB)
 ln_fht_quant_kernel(const void* __restrict__ x, int64_t M, float sK, void* __restrict__ out,
-                    float* __restrict__ scales) {
+                    float* __restrict__ scales, const void* __restrict__ aux) {
   using S = Shape<LOGK>;
   constexpr int K = S::K, T = S::T, R = S::R;
   extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -207,10 +237,14 @@ ln_fht_quant_kernel(const void* __restrict__ x, int64_t M, float sK, void* __res
   const int t = tid % T;
   const int64_t row = (int64_t)blockIdx.x * R + rl;
   const bool active = row < M;
-  const size_t esz = BF16 ? 2 : 4;
+  // K1_LNBWD transforms a float gradient row; BF16 then describes the
+  // LayerNorm input x (aux) and the output
+  constexpr bool IN_BF16 = MODE == K1_LNBWD ? false : BF16;
+  const size_t esz = IN_BF16 ? 2 : 4;
   const void* xrow = reinterpret_cast<const unsigned char*>(x) + (size_t)(active ? row : 0) * K * esz;
   const int row_off = rl * S::STRIDE;
-  constexpr bool kLN = MODE != K1_FHT_F32;  // the plain transform mode has no LayerNorm
+  // the plain transform and the backward transform have no forward LayerNorm
+  constexpr bool kLN = MODE != K1_FHT_F32 && MODE != K1_LNBWD;
   // a programmatic dependent of this kernel may start now (it waits for this
   // kernel's results itself before reading them)
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -220,9 +254,9 @@ ln_fht_quant_kernel(const void* __restrict__ x, int64_t M, float sK, void* __res
   // ---- pass 1: load, remove a large row offset, stages of bits {0,1,2,k-3,k-2,k-1}
   float f8[8] = {0, 0, 0, 0, 0, 0, 0, 0};
   if (active) {
-    load8<BF16>(xrow, 0, f8);
+    load8<IN_BF16>(xrow, 0, f8);
 #pragma unroll
-    for (int jj = 0; jj < 8; ++jj) load8<BF16>(xrow, (jj * T + t) * 8, &e[jj * 8]);
+    for (int jj = 0; jj < 8; ++jj) load8<IN_BF16>(xrow, (jj * T + t) * 8, &e[jj * 8]);
   } else {
 #pragma unroll
     for (int r = 0; r < 64; ++r) e[r] = 0.0f;
@@ -286,7 +320,66 @@ ln_fht_quant_kernel(const void* __restrict__ x, int64_t M, float sK, void* __res
   for (int r = 0; r < 64; r += 2) mul2(e[r], e[r + 1], cmul);
   if (kLN && t == 0) e[0] = 0.0f;
 
-  if constexpr (MODE == K1_T_F32 || MODE == K1_FHT_F32) {
+  if constexpr (MODE == K1_LNBWD) {
+    // e = g_u[base .. base + 63]; the LayerNorm backward at the forward's x of
+    // the same elements: g_x = (g_u - mean g_u - u mean(g_u u)) / sigma.
+    // Statistics on x - x0 (x0 the row's first value, the same in every
+    // thread) so that a large row mean costs no precision; one reduction of
+    // four sums: sum d, sum d^2, sum g_u d, sum g_u.
+    const unsigned char* xl = reinterpret_cast<const unsigned char*>(aux) + (size_t)(active ? row : 0) * K * (BF16 ? 2 : 4);
+    float x0 = 0.0f;
+    float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    if (active) {
+      float f0[8];
+      load8<BF16>(xl, 0, f0);
+      x0 = f0[0];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        float xv[8];
+        load8<BF16>(xl, base + 8 * j, xv);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const float d = xv[u] - x0;
+          acc.x += d;
+          acc.y = fmaf(d, d, acc.y);
+          acc.z = fmaf(e[8 * j + u], d, acc.z);
+          acc.w += e[8 * j + u];
+        }
+      }
+    }
+    acc = row_sum4<T, S::WPR>(acc, reinterpret_cast<float4*>(red1), rl, t);
+    const float invK = 1.0f / (float)K;
+    const float mu = acc.x * invK;                            // mean of x - x0
+    const float var = fmaxf(acc.y * invK - mu * mu, 0.0f);
+    const float rs = rsqrtf(var + 1e-5f);                     // 1 / sigma
+    const float mg = acc.w * invK;                            // mean g_u
+    const float mgu = rs * (acc.z * invK - mu * mg);          // mean(g_u u)
+    if (active) {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        float xv[8], r[8];
+        load8<BF16>(xl, base + 8 * j, xv);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const float uu = (xv[u] - x0 - mu) * rs;
+          r[u] = (e[8 * j + u] - mg - uu * mgu) * rs;
+        }
+        if constexpr (BF16) {
+          uint32_t h[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+            h[u] = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(r[2 * u])) |
+                   ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(r[2 * u + 1])) << 16);
+          reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(out) + (size_t)row * K + base)[j] =
+              make_uint4(h[0], h[1], h[2], h[3]);
+        } else {
+          float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(out) + (size_t)row * K + base + 8 * j);
+          dst[0] = make_float4(r[0], r[1], r[2], r[3]);
+          dst[1] = make_float4(r[4], r[5], r[6], r[7]);
+        }
+      }
+    }
+  } else if constexpr (MODE == K1_T_F32 || MODE == K1_FHT_F32) {
     if (active) {
       float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(out) + (size_t)row * K + base);
 #pragma unroll
@@ -345,7 +438,8 @@ ln_fht_quant_kernel(const void* __restrict__ x, int64_t M, float sK, void* __res
 }
 
 template <int LOGK, bool BF16, int MODE>
-cudaError_t launch_one(const void* x, int64_t M, void* out, float* scales, cudaStream_t stream) {
+cudaError_t launch_one(const void* x, int64_t M, void* out, float* scales, cudaStream_t stream,
+                       const void* aux = nullptr) {
   using S = Shape<LOGK>;
   auto kern = ln_fht_quant_kernel<LOGK, BF16, MODE>;
   static bool smem_set[sm100_host::kMaxDevices] = {false};
@@ -353,7 +447,7 @@ cudaError_t launch_one(const void* x, int64_t M, void* out, float* scales, cudaS
   if (e != cudaSuccess) return e;
   const int64_t grid = (M + S::R - 1) / S::R;
   const float sK = (float)(1.0 / sqrt((double)S::K));
-  kern<<<(unsigned)grid, S::THREADS, S::SMEM, stream>>>(x, M, sK, out, scales);
+  kern<<<(unsigned)grid, S::THREADS, S::SMEM, stream>>>(x, M, sK, out, scales, aux);
   return cudaGetLastError();
 }
 
@@ -466,6 +560,32 @@ cudaError_t launch_ln_fht_quant(const void* x, bool in_bf16, int64_t M, int log2
     case 13: return launch_k<13>(x, in_bf16, M, mode, out, scales, stream);
     case 14: return launch_k<14>(x, in_bf16, M, mode, out, scales, stream);
     case 15: return launch_k<15>(x, in_bf16, M, mode, out, scales, stream);
+  }
+  return cudaErrorInvalidValue;
+}
+
+namespace {
+template <int LOGK>
+cudaError_t launch_lnbwd_k(const float* g, const void* x, bool x_bf16, int64_t M, void* gx, cudaStream_t s) {
+  return x_bf16 ? launch_one<LOGK, true, K1_LNBWD>(g, M, gx, nullptr, s, x)
+                : launch_one<LOGK, false, K1_LNBWD>(g, M, gx, nullptr, s, x);
+}
+}  // namespace
+
+cudaError_t launch_fht_ln_backward(const float* g, const void* x, bool x_bf16, int64_t M, int log2k, void* gx,
+                                   cudaStream_t stream) {
+  if (M <= 0) return cudaSuccess;
+  switch (log2k) {
+    case 6: return launch_lnbwd_k<6>(g, x, x_bf16, M, gx, stream);
+    case 7: return launch_lnbwd_k<7>(g, x, x_bf16, M, gx, stream);
+    case 8: return launch_lnbwd_k<8>(g, x, x_bf16, M, gx, stream);
+    case 9: return launch_lnbwd_k<9>(g, x, x_bf16, M, gx, stream);
+    case 10: return launch_lnbwd_k<10>(g, x, x_bf16, M, gx, stream);
+    case 11: return launch_lnbwd_k<11>(g, x, x_bf16, M, gx, stream);
+    case 12: return launch_lnbwd_k<12>(g, x, x_bf16, M, gx, stream);
+    case 13: return launch_lnbwd_k<13>(g, x, x_bf16, M, gx, stream);
+    case 14: return launch_lnbwd_k<14>(g, x, x_bf16, M, gx, stream);
+    case 15: return launch_lnbwd_k<15>(g, x, x_bf16, M, gx, stream);
   }
   return cudaErrorInvalidValue;
 }

@@ -1097,7 +1097,7 @@ cudaError_t launch_tc_mode(const void* x, int64_t M, K1Mode mode, void* out, flo
 }  // namespace
 
 bool ln_fht_quant_tc_supports(bool in_bf16, int log2k, K1Mode mode, const void* x, const void* out) {
-  return in_bf16 && log2k >= 7 && log2k <= 15 && mode != K1_FHT_F32 &&
+  return in_bf16 && log2k >= 7 && log2k <= 15 && mode != K1_FHT_F32 && mode != K1_LNBWD &&
          (reinterpret_cast<uintptr_t>(x) & 15u) == 0 && (reinterpret_cast<uintptr_t>(out) & 15u) == 0;
 }
 

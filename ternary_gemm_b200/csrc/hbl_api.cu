@@ -73,9 +73,9 @@ ForwardLayout forward_layout(int64_t M, int64_t K, int64_t N) {
 }
 
 // hbl_backward's workspace: codes int8 [M][K], scales [M], bf16 copies of
-// w [N][K], g_y [M][N], s g_y [M][N] and q [M][K], g_t and g_u f32 [M][K]
+// w [N][K], g_y [M][N], s g_y [M][N] and q [M][K], g_t f32 [M][K]
 struct BackwardLayout {
-  size_t q_off, s_off, w16_off, gy16_off, gys_off, q16_off, gt_off, gu_off, total;
+  size_t q_off, s_off, w16_off, gy16_off, gys_off, q16_off, gt_off, total;
 };
 
 BackwardLayout backward_layout(int64_t M, int64_t K, int64_t N) {
@@ -88,8 +88,7 @@ BackwardLayout backward_layout(int64_t M, int64_t K, int64_t N) {
   L.gys_off = L.gy16_off + align256(m * n * 2);
   L.q16_off = L.gys_off + align256(m * n * 2);
   L.gt_off = L.q16_off + align256(m * k * 2);
-  L.gu_off = L.gt_off + align256(m * k * 4);
-  L.total = L.gu_off + align256(m * k * 4);
+  L.total = L.gt_off + align256(m * k * 4);
   return L;
 }
 
@@ -365,12 +364,11 @@ hbl_status hbl_backward(const void* x, hbl_dtype xt, int64_t M, int64_t K, const
   uint16_t* gys = reinterpret_cast<uint16_t*>(ws + L.gys_off);
   uint16_t* q16 = reinterpret_cast<uint16_t*>(ws + L.q16_off);
   float* gt = reinterpret_cast<float*>(ws + L.gt_off);
-  float* gu = reinterpret_cast<float*>(ws + L.gu_off);
   const bool gy_bf16 = gyt == HBL_BF16;
   const K1Mode mode = bits == 4 ? hbl::K1_Q4_I8 : hbl::K1_Q8_I8;
   // the forward's codes and scales, recomputed
   cudaError_t e = hbl::launch_ln_fht_quant(x, xt == HBL_BF16, M, l, mode, q, scales, stream);
-  // activation gradient: g_t = alpha g_y w, g_u = H g_t / sqrt(K), LayerNorm backward
+  // activation gradient: g_t = alpha g_y w, then g_u = H g_t / sqrt(K) and the LayerNorm backward
   if (e == cudaSuccess) e = hbl::launch_ternary_to_bf16(packed, N, K, w16, stream);
   const uint16_t* gyb = reinterpret_cast<const uint16_t*>(g_y);
   if (e == cudaSuccess && !gy_bf16) {
@@ -378,8 +376,8 @@ hbl_status hbl_backward(const void* x, hbl_dtype xt, int64_t M, int64_t K, const
     gyb = gy16;
   }
   if (e == cudaSuccess) e = hbl::launch_gemm_bf16(gyb, false, w16, M, K, N, gt, alpha_dev, stream);
-  if (e == cudaSuccess) e = hbl::launch_ln_fht_quant(gt, false, M, l, hbl::K1_FHT_F32, gu, nullptr, stream);
-  if (e == cudaSuccess) e = hbl::launch_ln_backward(x, xt == HBL_BF16, gu, M, l, g_x, stream);
+  // g_u = H g_t / sqrt(K) and the LayerNorm backward in one pass over the rows
+  if (e == cudaSuccess) e = hbl::launch_fht_ln_backward(gt, x, xt == HBL_BF16, M, l, g_x, stream);
   // weight gradient: g_W = (s g_y)^T q
   if (e == cudaSuccess) e = hbl::launch_scale_rows_bf16(g_y, gy_bf16, scales, M, N, gys, stream);
   if (e == cudaSuccess) e = hbl::launch_codes_to_bf16(q, M * K, q16, stream);
@@ -407,6 +405,17 @@ hbl_status hbl_ln_backward(const void* x, hbl_dtype xt, int64_t M, int64_t K, co
   if (s != HBL_OK) return s;
   if ((s = check_rows(M)) != HBL_OK) return s;
   return cuda_status(hbl::launch_ln_backward(x, xt == HBL_BF16, g_u, M, l, g_x, stream));
+}
+
+hbl_status hbl_fht_ln_backward(const float* g, const void* x, hbl_dtype xt, int64_t M, int64_t K, void* g_x,
+                               cudaStream_t stream) {
+  if (!g || !x || !g_x || !dtype_ok(xt)) return HBL_ERR_INVALID_ARG;
+  if (!aligned(g, 16) || !aligned(x, 16) || !aligned(g_x, 16)) return HBL_ERR_INVALID_ARG;
+  int l;
+  hbl_status s = check_k(K, &l);
+  if (s != HBL_OK) return s;
+  if ((s = check_rows(M)) != HBL_OK) return s;
+  return cuda_status(hbl::launch_fht_ln_backward(g, x, xt == HBL_BF16, M, l, g_x, stream));
 }
 
 hbl_status hbl_last_device_error(cudaStream_t stream) {

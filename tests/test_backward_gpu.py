@@ -106,6 +106,33 @@ def test_ln_backward(H, orc, xdt, K):
         assert np.linalg.norm(got[m].astype(np.float64) - want[m]) <= rel * n + 1e-30, m
 
 
+@pytest.mark.parametrize("xdt", ["bf16", "f32"])
+@pytest.mark.parametrize("K", [64, 256, 2048, 16384, 32768])
+def test_fht_ln_backward(H, orc, xdt, K):
+    """The fused transform + LayerNorm backward of hbl_backward, on rows with a
+    large mean, a tiny variance and no variance at all."""
+    import torch
+    rng = np.random.default_rng(3 * K + (xdt == "bf16"))
+    M = 6
+    x = rng.standard_normal((M, K)).astype(np.float32)
+    x[1] += 40.0
+    x[2] = x[2] * 1e-3 - 7.0
+    x[3] = 2.5
+    if xdt == "bf16":
+        xb = _bf16_bits(x)
+        x_in, xv = xb, _bf16_values(xb)
+    else:
+        x_in, xv = x, x
+    g = (rng.standard_normal((M, K)) * 0.1).astype(np.float32)
+    got = to_host(H.hbl_fht_ln_backward(torch.from_numpy(g).cuda(), to_device(x_in)))
+    got = _bf16_values(got) if xdt == "bf16" else got
+    rel = 4e-3 if xdt == "bf16" else 1e-4
+    for m in range(M):
+        g_u = orc.fht_unnormalized(g[m].astype(np.float64)) / np.sqrt(K)
+        want = orc.ln_backward_row(xv[m].astype(np.float64), g_u)
+        assert np.linalg.norm(got[m].astype(np.float64) - want) <= rel * np.linalg.norm(want), m
+
+
 def _backward_case(H, orc, M, K, N, bits, x_dtype, gy_dtype, seed):
     import torch
     wl = WORKLOADS["sweep"].with_shape(M, K, N)
