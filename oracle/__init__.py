@@ -69,6 +69,8 @@ def _L():
             lib.orc_layernorm_row.restype = None
             lib.orc_ln_backward_row.argtypes = [p, p, i64, p]
             lib.orc_ln_backward_row.restype = None
+            lib.orc_kv_quant.argtypes = [p, i32, i64, i64, i32, p, p]
+            lib.orc_kv_quant.restype = i32
             lib.orc_fht_rows.argtypes = [p, i32, i64, i64, p, p]
             lib.orc_fht_rows.restype = i32
             lib.orc_rmsnorm_row.argtypes = [p, i64, p]
@@ -358,3 +360,25 @@ def backward_weight(g_y: np.ndarray, codes: np.ndarray, scales: np.ndarray) -> n
     quantizer passed through).  g_y [M][N], codes [M][K], scales [M]."""
     a = np.asarray(codes, dtype=np.float64) * np.asarray(scales, dtype=np.float64)[:, None]
     return np.asarray(g_y, dtype=np.float64).T @ a
+
+
+def kv_quant(x: np.ndarray, bits: int):
+    """Low-bit QKV-state quantizer (post-RoPE heads to unsigned integers by absmax).
+
+    x: [rows][D] float32 or bf16 bits, one head vector per row.  Per row
+    gamma = max|x|, r = (2^b - 1) / (2 (gamma + eps)), q = clip(rint(x r + (2^b - 1)/2), 0, 2^b - 1)
+    (the product and the sum rounded to float).  Returns (codes uint8 [rows][D], scales = gamma [rows]).
+    """
+    x, dt = _as_input(x)
+    rows, D = x.shape
+    codes = np.empty((rows, D), np.uint8)
+    scales = np.empty((rows,), np.float32)
+    if _L().orc_kv_quant(_ptr(x), dt, rows, D, int(bits), _ptr(codes), _ptr(scales)) != 0:
+        raise ValueError("orc_kv_quant: bits must be in [2, 8]")
+    return codes, scales
+
+
+def kv_dequant(codes: np.ndarray, scales: np.ndarray, bits: int) -> np.ndarray:
+    """x~ = (2 q - L) gamma / L in double, L = 2^b - 1."""
+    L = float((1 << bits) - 1)
+    return (2.0 * np.asarray(codes, np.float64) - L) * np.asarray(scales, np.float64)[:, None] / L

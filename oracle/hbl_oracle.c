@@ -408,3 +408,39 @@ int orc_forward_rows(const void* x, int dtype, int64_t M, int64_t K, const int64
   free(xr); free(t); free(q); free(acc);
   return rc;
 }
+
+/* ------------------------------------------------------- low-bit QKV states */
+
+/* Post-RoPE QKV-state quantizer of the low-bit attention experiments (QbitAI
+ * report / Xinzhiyuan article, "low-bit attention": the QKV heads are quantized
+ * to unsigned integers by the absmax function, with no calibration data; a
+ * 3-bit KV cache matches full precision).  Reading of the open steps: one head
+ * vector of D values (one token, one head) at a time; gamma = max|x|; the
+ * range [-gamma, gamma] maps linearly onto the 2^b unsigned levels 0 .. 2^b-1:
+ *   L = 2^b - 1,  r = L / (2 (gamma + eps))  (one float division),
+ *   q = clip(rint(fl(fl(x r) + L/2)), 0, L),  scale = gamma,
+ * so x ~ (2 q - L) gamma / L.  rint rounds half to even. */
+int orc_kv_quant(const void* x, int dtype, int64_t rows, int64_t D, int bits, uint8_t* codes, float* scales) {
+  if (rows < 0 || D <= 0 || bits < 2 || bits > 8) return -1;
+  const float L = (float)((1 << bits) - 1);
+  const float half = 0.5f * L;
+  for (int64_t m = 0; m < rows; ++m) {
+    float g = 0.0f;
+    for (int64_t i = 0; i < D; ++i) {
+      float a = fabsf((float)orc_load(x, dtype, m * D + i));
+      if (a > g) g = a;
+    }
+    volatile float den = 2.0f * (g + ORC_EPS_Q);
+    volatile float r = L / den;
+    for (int64_t i = 0; i < D; ++i) {
+      volatile float t = (float)orc_load(x, dtype, m * D + i) * r;
+      volatile float u = t + half;
+      double q = orc_rint((double)u);
+      if (q < 0.0) q = 0.0;
+      if (q > (double)L) q = (double)L;
+      codes[m * D + i] = (uint8_t)q;
+    }
+    scales[m] = g;
+  }
+  return 0;
+}

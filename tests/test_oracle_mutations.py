@@ -49,6 +49,11 @@ MUTANTS = [
      "gx[i] = (gu[i] - mg - (x[i] - mu) * inv * mgu);"),
     ("LayerNorm backward unbiased variance", "const double var = ss / (double)K;",
      "const double var = ss / (double)(K - 1);"),
+    # the QKV-state quantizer (tests/test_oracle_kv_pins.py)
+    ("KV levels without the offset", "volatile float u = t + half;", "volatile float u = t;"),
+    ("KV absmax without abs", "float a = fabsf((float)orc_load(x, dtype, m * D + i));",
+     "float a = (float)orc_load(x, dtype, m * D + i);"),
+    ("KV 2^b levels off by one", "const float L = (float)((1 << bits) - 1);", "const float L = (float)(1 << bits);"),
 ]
 
 
@@ -65,7 +70,8 @@ def _run_mutant(m):
         env = dict(os.environ, HBL_ORACLE_LIB=so)
         p = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
                             os.path.join(ROOT, "tests", "test_oracle_pins.py"),
-                            os.path.join(ROOT, "tests", "test_oracle_backward_pins.py")],
+                            os.path.join(ROOT, "tests", "test_oracle_backward_pins.py"),
+                            os.path.join(ROOT, "tests", "test_oracle_kv_pins.py")],
                            env=env, capture_output=True, text=True, timeout=600)
         return name, p.returncode, p.stdout[-400:]
 
