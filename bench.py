@@ -52,7 +52,7 @@ def parse_args(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
-    ap.add_argument("--sweep", choices=["k1", "fwd", "k1_noh", "bwd"], default=None,
+    ap.add_argument("--sweep", choices=["k1", "fwd", "k1_noh", "bwd", "kv"], default=None,
                     help="instead of the step line: the LN+FHT+INT4 kernel alone at M=65536 for each K, "
                          "or the whole forward at K=N=4096 for each M (one JSON line per point)")
     ap.add_argument("--shape", default=None,
@@ -476,6 +476,22 @@ def bench_sweep(args):
 
     if args.sweep == "bwd":
         return bench_backward(args, hbl, peaks, peak_kind, timed)
+    if args.sweep == "kv":
+        # QKV states of 8192 tokens, 32 heads of 128 (the 7B shape), three tensors, bf16
+        rows, D = 3 * 8192 * 32, 128
+        g = torch.Generator(device="cuda").manual_seed(7)
+        x = (torch.randn((rows, D), device="cuda", generator=g) * 2.0).to(torch.bfloat16)
+        codes = torch.empty((rows, D), dtype=torch.uint8, device="cuda")
+        sc = torch.empty((rows,), dtype=torch.float32, device="cuda")
+        for bits in (3, 4, 8):
+            t = timed(lambda: hbl.hbl_kv_quant(x, bits, codes=codes, scales=sc), reps)
+            nbytes = rows * D * 2 + rows * D + 4 * rows
+            gbs = nbytes / t / 1e9
+            print(json.dumps({"sweep": "kv_quant", "rows": rows, "D": D, "bits": bits, "ms": t * 1e3, "GB/s": gbs,
+                              "frac_hbm": gbs / peaks["hbm_gbs"], "peak_kind": peak_kind,
+                              "bytes_per_launch": nbytes, "input": "seeded N(0, 4) bf16 head vectors"}),
+                  flush=True)
+        return 0
     if args.sweep in ("k1", "k1_noh"):
         M, ks = 65536, SWEEP_K1_KS
         if args.shape:

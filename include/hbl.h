@@ -276,6 +276,24 @@ hbl_status hbl_ln_backward(const void* x, hbl_dtype xt, int64_t M, int64_t K, co
 hbl_status hbl_fht_ln_backward(const float* g, const void* x, hbl_dtype xt, int64_t M, int64_t K, void* g_x,
                                cudaStream_t stream);
 
+/* ---------------------------------------------------------------- low-bit QKV states
+ * The low-bit attention experiments of the pages quantize the QKV states after
+ * RoPE: the heads go to unsigned integers through the absmax function, with no
+ * calibration data (a 3-bit KV cache matches full precision).  The pages give
+ * no formula; this library reads it as a linear map of [-gamma, gamma] onto
+ * the 2^b unsigned levels, per head vector (one token, one head):
+ *   gamma = max|x|, L = 2^b - 1, r = L / (2 (gamma + eps)) (float division),
+ *   q = clip(rint(fl(fl(x r) + L/2)), 0, L),  scale = gamma,
+ * so that x ~ (2 q - L) gamma / L.  RoPE itself and the attention are the
+ * caller's.
+ *   x      device, [rows][D] of dtype xt (each row one head vector, post-RoPE)
+ *   D      head dimension: 32, 64, 128 or 256 (else HBL_ERR_UNSUPPORTED)
+ *   bits   2 .. 8
+ *   codes  device, [rows][D] bytes, one unsigned code per byte (output)
+ *   scales device, rows floats: gamma per head vector (output) */
+hbl_status hbl_kv_quant(const void* x, hbl_dtype xt, int64_t rows, int64_t D, int bits, uint8_t* codes,
+                        float* scales, cudaStream_t stream);
+
 /* ---------------------------------------------------------------- test hooks */
 
 /* Stages 1-2 alone: t = H LN(x) / sqrt(K) as float [M][K] (device output).

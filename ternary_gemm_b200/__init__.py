@@ -80,6 +80,8 @@ def lib():
             L.hbl_ln_backward.restype = i32
             L.hbl_fht_ln_backward.argtypes = [p, p, i32, i64, i64, p, p]
             L.hbl_fht_ln_backward.restype = i32
+            L.hbl_kv_quant.argtypes = [p, i32, i64, i64, i32, p, p, p]
+            L.hbl_kv_quant.restype = i32
             L.hbl_pack_ternary_rotated_workspace_bytes.argtypes = [i64, i64]
             L.hbl_pack_ternary_rotated_workspace_bytes.restype = sz
             L.hbl_pack_ternary_rotated.argtypes = [p, i32, i64, i64, p, p, p, sz, p]
@@ -280,6 +282,20 @@ def hbl_fht_ln_backward(g, x, g_x=None, stream=None):
     _check(lib().hbl_fht_ln_backward(_ptr(g), _ptr(x), _dtype_code(x), M, K, _ptr(g_x), _stream(stream)),
            "hbl_fht_ln_backward")
     return g_x
+
+
+def hbl_kv_quant(x, bits: int, codes=None, scales=None, stream=None):
+    """Post-RoPE head vectors x [rows][D] -> (unsigned codes uint8 [rows][D], gamma float32 [rows])."""
+    torch = _torch()
+    _need_cuda(x)
+    rows, D = x.shape
+    if codes is None:
+        codes = torch.empty((rows, D), dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty((rows,), dtype=torch.float32, device=x.device)
+    _check(lib().hbl_kv_quant(_ptr(x), _dtype_code(x), rows, D, bits, _ptr(codes), _ptr(scales), _stream(stream)),
+           "hbl_kv_quant")
+    return codes, scales
 
 
 def hbl_fht(x, t=None, stream=None):

@@ -96,6 +96,9 @@ cudaError_t launch_scale_rows_bf16(const void* g, bool g_bf16, const float* s, i
                                    cudaStream_t stream);
 cudaError_t launch_ln_backward(const void* x, bool x_bf16, const float* gu, int64_t M, int log2k, void* gx,
                                cudaStream_t stream);
+// low-bit QKV-state quantizer (kv_quant.cu): D in {32, 64, 128, 256}, bits in [2, 8]
+cudaError_t launch_kv_quant(const void* x, bool bf16, int64_t rows, int64_t D, int bits, uint8_t* codes,
+                            float* scales, cudaStream_t stream);
 // g_x = LayerNorm backward at x of H g / sqrt(K), in one pass (fht_quant.cu)
 cudaError_t launch_fht_ln_backward(const float* g, const void* x, bool x_bf16, int64_t M, int log2k, void* gx,
                                    cudaStream_t stream);

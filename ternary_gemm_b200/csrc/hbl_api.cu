@@ -418,6 +418,16 @@ hbl_status hbl_fht_ln_backward(const float* g, const void* x, hbl_dtype xt, int6
   return cuda_status(hbl::launch_fht_ln_backward(g, x, xt == HBL_BF16, M, l, g_x, stream));
 }
 
+hbl_status hbl_kv_quant(const void* x, hbl_dtype xt, int64_t rows, int64_t D, int bits, uint8_t* codes,
+                        float* scales, cudaStream_t stream) {
+  if (!x || !codes || !scales || !dtype_ok(xt)) return HBL_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(codes, 16) || !aligned(scales, 4)) return HBL_ERR_INVALID_ARG;
+  if (rows <= 0 || D <= 0 || bits <= 0) return HBL_ERR_INVALID_ARG;
+  if ((D != 32 && D != 64 && D != 128 && D != 256) || bits < 2 || bits > 8 || rows > kMaxRows * 64)
+    return HBL_ERR_UNSUPPORTED;
+  return cuda_status(hbl::launch_kv_quant(x, xt == HBL_BF16, rows, D, bits, codes, scales, stream));
+}
+
 hbl_status hbl_last_device_error(cudaStream_t stream) {
   int v = 0;
   cudaError_t e = hbl::read_and_clear_device_error(stream, &v);
