@@ -211,6 +211,42 @@ def oracle_rows_per_second(wl, bits: int, seconds: float, max_rows: int = 512):
     return done / dt, done, dt
 
 
+def oracle_rows_per_second_all_cores(wl, bits: int, seconds: float, max_rows: int = 2048):
+    """The same oracle forward, rows spread over every host core: one thread per
+    core, each calling the single-threaded C oracle on its own rows (ctypes
+    releases the GIL during the call).  Returns (rows/s, rows, seconds, threads)."""
+    import concurrent.futures as cf
+    import numpy as np
+    import oracle
+    from ternary_gemm_b200.inputs import make_w, make_x_rows
+    oracle.build()
+    w, a = oracle.ternary(make_w(wl))
+    threads = max(1, os.cpu_count() or 1)
+    rows = np.arange(min(max_rows, wl.M), dtype=np.int64)
+    x = make_x_rows(wl, rows)
+    deadline = time.perf_counter() + seconds
+    counter = {"next": 0}
+    lock = threading.Lock()
+
+    def work():
+        done = 0
+        while time.perf_counter() < deadline:
+            with lock:
+                i = counter["next"]
+                counter["next"] += 1
+            if i >= rows.size:
+                break
+            oracle.forward_rows(x[i:i + 1], w, a, bits)
+            done += 1
+        return done
+
+    t0 = time.perf_counter()
+    with cf.ThreadPoolExecutor(max_workers=threads) as ex:
+        done = sum(ex.map(lambda _: work(), range(threads)))
+    dt = time.perf_counter() - t0
+    return done / dt, done, dt, threads
+
+
 def run_reference(args):
     """The reference arm: the CPU oracle on bounded samples, rank 0 only."""
     rank = int(os.environ.get("RANK", "0"))
@@ -271,12 +307,16 @@ def bench_ours(args):
     peaks, peak_kind = load_peaks()
 
     # CPU baseline first, before any GPU work in this process (rank 0, N = 1 only)
-    cpu = None
+    cpu = cpu_all = None
     if ranks.rank == 0 and ranks.world == 1 and not args.no_cpu_baseline:
         v, n, dt = oracle_rows_per_second(wl, bits, args.cpu_seconds)
         cpu = {"value": v, "unit": "tokens/s", "cores": 1, "kind": "oracle",
                "sample": "%d rows of %s (K=%d, N=%d, INT%d) through LN+FHT+quant+GEMM+dequant, single-threaded C "
                          "oracle, %.1f s" % (n, wl.name, K, N, bits, dt)}
+        va, na, dta, nt = oracle_rows_per_second_all_cores(wl, bits, args.cpu_seconds / 2)
+        cpu_all = {"value": va, "unit": "tokens/s", "cores": nt, "kind": "oracle",
+                   "sample": "%d rows of %s through the same C oracle, one thread per host core, %.1f s"
+                             % (na, wl.name, dta)}
 
     x = _to_device(make_x(wl))
     W = _to_device(make_w(wl))
@@ -415,7 +455,8 @@ def bench_ours(args):
                        % (x.numel() * x.element_size() // 2 ** 20), "parallelism": "replicas"},
             "roofline": roofline, "k1": k1, "int8_tops": achieved_tops,
             "stages_ms": {"ln_fht_quant": t_k1 * 1e3, "widen_ternary": t_wd * 1e3, "gemm_dequant": t_gm * 1e3},
-            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 2 * args.steps, "clocks": clk}
+            "cpu_baseline": cpu, "cpu_baseline_all_cores": cpu_all, "e2e": e2e, "gpu_launches": 2 * args.steps,
+            "clocks": clk}
     if ranks.rank == 0:
         print(json.dumps(line), flush=True)
     ranks.barrier()
