@@ -70,9 +70,11 @@ cudaError_t launch_widen_ternary(const uint8_t* packed, int64_t N, int64_t K, in
 // tcgen05 int8 GEMM: acc[m][n] = sum_k A[m][k] B[n][k].  Epilogue: either the
 // raw int32 (y_mode 0) or y = (float)acc * (scales[m] * alpha[0]) as float
 // (y_mode 1) or bf16 (y_mode 2).
+// ab_max: a bound on |A[m][k] B[n][k]| known to the caller (8 for INT4 codes
+// times ternary weights), or 0; it lets short batches exchange int16 partials
 cudaError_t launch_gemm_i8(const int8_t* A, const int8_t* B, int64_t M, int64_t N, int64_t K,
                            int y_mode, void* y, const float* scales, const float* alpha,
-                           cudaStream_t stream);
+                           cudaStream_t stream, int ab_max = 0);
 
 // Small-M product straight from the packed 2-bit weights with the same
 // dequantisation (y_mode 1 float, 2 bf16): M <= kGemvMaxRows and

@@ -520,6 +520,7 @@ gemm_i8_2sm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
 // them, so each thread reaches both.
 constexpr int kSplitMax = 8;
 constexpr int kPartRowBytes = 256 * 4 + 16;
+constexpr int kPart16RowBytes = 256 * 2 + 16;  // int16 partials (the bound allows it)
 constexpr uint32_t kSplitTmemCols = 256;
 static_assert(128 * kPartRowBytes <= kStages * kStageBytes, "partial must fit in the stage ring");
 
@@ -560,7 +561,7 @@ __device__ __forceinline__ void store_y4(const Params& p, int row, int col, cons
   }
 }
 
-template <int S>
+template <int S, bool P16>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_i8_splitk_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, Params p) {
   extern __shared__ uint8_t smem_raw[];
@@ -659,9 +660,13 @@ gemm_i8_splitk_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
     // whatever TMEM holds; the error word is set and the handshakes below
     // still run).  Two TMEM loads in flight per wait.
     const int rows = min(kBM, p.M - m_blk * kBM);
+    // P16: every partial fits in int16 (the host's bound on |a b| times this
+    // rank's k-range), so the exchange moves half the bytes
+    constexpr int kRowBytes = P16 ? kPart16RowBytes : kPartRowBytes;
+    constexpr int kEsz = P16 ? 2 : 4;
     if (quarter * 32 < rows) {
       const int prow = quarter * 32 + lane;
-      uint8_t* dst = part + (size_t)prow * kPartRowBytes;
+      uint8_t* dst = part + (size_t)prow * kRowBytes;
       const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16);
 #pragma unroll 1
       for (int c = 0; c < 256; c += 64) {
@@ -670,9 +675,17 @@ gemm_i8_splitk_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
         tmem_ld32_nowait(tbase + (uint32_t)(c + 32), &r[32]);
         tmem_wait_ld();
         if (prow < rows) {
+          if constexpr (P16) {
 #pragma unroll
-          for (int j = 0; j < 64; j += 4)
-            *reinterpret_cast<uint4*>(dst + 4 * (c + j)) = make_uint4(r[j], r[j + 1], r[j + 2], r[j + 3]);
+            for (int j = 0; j < 64; j += 8)
+              *reinterpret_cast<uint4*>(dst + 2 * (c + j)) =
+                  make_uint4((r[j] & 0xFFFFu) | (r[j + 1] << 16), (r[j + 2] & 0xFFFFu) | (r[j + 3] << 16),
+                             (r[j + 4] & 0xFFFFu) | (r[j + 5] << 16), (r[j + 6] & 0xFFFFu) | (r[j + 7] << 16));
+          } else {
+#pragma unroll
+            for (int j = 0; j < 64; j += 4)
+              *reinterpret_cast<uint4*>(dst + 4 * (c + j)) = make_uint4(r[j], r[j + 1], r[j + 2], r[j + 3]);
+          }
         }
       }
     }
@@ -683,7 +696,8 @@ gemm_i8_splitk_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
       // group all issued before any is used (16 remote loads in flight per
       // thread, so the distributed-shared-memory latency is paid 4 times).
       constexpr int W = kBN / S;
-      constexpr int GPR = W / 4;        // groups per row
+      constexpr int GW = 16 / kEsz;     // columns per group: one 16-byte load
+      constexpr int GPR = W / GW;       // groups per row
       constexpr int GB = 16 / S;        // groups per batch and thread
       const int total = rows * GPR;     // groups of the valid rows
       const uint32_t part_u32 = smem_u32(part);
@@ -694,7 +708,7 @@ gemm_i8_splitk_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
         for (int gi = 0; gi < GB; ++gi) {
           const int g = b + 128 * gi + et;
           if (g < total) {
-            const uint32_t off = part_u32 + (uint32_t)((g / GPR) * kPartRowBytes + 4 * (rank * W + 4 * (g % GPR)));
+            const uint32_t off = part_u32 + (uint32_t)((g / GPR) * kRowBytes + kEsz * (rank * W + GW * (g % GPR)));
 #pragma unroll
             for (int r = 0; r < S; ++r) u[gi][r] = ld_cluster_v4(mapa_shared(off, (uint32_t)r));
           }
@@ -703,19 +717,33 @@ gemm_i8_splitk_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
         for (int gi = 0; gi < GB; ++gi) {
           const int g = b + 128 * gi + et;
           if (g >= total) continue;
-          int v[4] = {0, 0, 0, 0};
+          int v[GW];
+#pragma unroll
+          for (int i = 0; i < GW; ++i) v[i] = 0;
 #pragma unroll
           for (int r = 0; r < S; ++r) {
-            v[0] += (int)u[gi][r].x;
-            v[1] += (int)u[gi][r].y;
-            v[2] += (int)u[gi][r].z;
-            v[3] += (int)u[gi][r].w;
+            const uint32_t w[4] = {u[gi][r].x, u[gi][r].y, u[gi][r].z, u[gi][r].w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              if constexpr (P16) {
+                v[2 * i] += (int)(w[i] << 16) >> 16;  // sign-extended halves
+                v[2 * i + 1] += (int)w[i] >> 16;
+              } else {
+                v[i] += (int)w[i];
+              }
+            }
           }
           const int row = m_blk * kBM + g / GPR;
-          const int col = n_blk * kBN + rank * W + 4 * (g % GPR);
-          if (row < p.M && col < p.N) {
+          const int col = n_blk * kBN + rank * W + GW * (g % GPR);
+          if (row < p.M) {
             const float sa = p.y_mode != 0 ? __fmul_rn(__ldg(p.scales + row), __ldg(p.alpha)) : 0.0f;
-            store_y4(p, row, col, v, sa);
+#pragma unroll
+            for (int h = 0; h < GW; h += 4) {
+              if (col + h < p.N) {
+                const int q4[4] = {v[h], v[h + 1], v[h + 2], v[h + 3]};
+                store_y4(p, row, col + h, q4, sa);
+              }
+            }
           }
         }
       }
@@ -737,13 +765,14 @@ bool make_map(CUtensorMap* map, const void* ptr, int64_t rows, int64_t K, int bo
 
 int sm_count() { return sm100_host::sm_count(); }
 
-constexpr int kSplitMaxRows = 64;
+constexpr int kSplitMaxRows = 64;     // int32 partials: the exchange grows with the rows
+constexpr int kSplitMaxRows16 = 255;  // int16 partials: every short batch
 
 // clusters of `split` CTAs of `kern` that the device holds at once (cached
 // per device and cluster size; 0 when the query fails)
 template <typename Kernel>
 int max_active_clusters(Kernel kern, int split, int idx) {
-  static int cache[3][sm100_host::kMaxDevices] = {};
+  static int cache[6][sm100_host::kMaxDevices] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= sm100_host::kMaxDevices) return 0;
   if (cache[idx][dev] > 0) return cache[idx][dev];
@@ -770,7 +799,7 @@ int max_active_clusters(Kernel kern, int split, int idx) {
 }  // namespace
 
 cudaError_t launch_gemm_i8(const int8_t* A, const int8_t* B, int64_t M, int64_t N, int64_t K, int y_mode, void* y,
-                           const float* scales, const float* alpha, cudaStream_t stream) {
+                           const float* scales, const float* alpha, cudaStream_t stream, int ab_max) {
   CUtensorMap ta, tb;
   if (!make_map(&ta, A, M, K, kBM) || !make_map(&tb, B, N, K, kBN)) return cudaErrorInvalidValue;
   Params p;
@@ -805,18 +834,23 @@ cudaError_t launch_gemm_i8(const int8_t* A, const int8_t* B, int64_t M, int64_t 
   // partials' exchange through distributed shared memory costs more than the
   // split saves.)
   const int nsm = sm_count();
-  if (M <= kSplitMaxRows) {
-    for (int split = kSplitMax; split >= 2; split /= 2) {
-      if (split > p.num_kb || p.num_tiles * split > nsm) continue;
-      auto kern = split == 2 ? gemm_i8_splitk_kernel<2> : split == 4 ? gemm_i8_splitk_kernel<4> : gemm_i8_splitk_kernel<8>;
-      const int idx = split == 2 ? 0 : split == 4 ? 1 : 2;
-      static bool smem_set_s[3][sm100_host::kMaxDevices] = {};
-      cudaError_t e = sm100_host::ensure_smem(kern, (int)kSmemBytes, smem_set_s[idx]);
-      if (e != cudaSuccess) return e;
-      if (p.num_tiles > max_active_clusters(kern, split, idx)) continue;
-      return sm100_host::launch_pdl(kern, (unsigned)(p.num_tiles * split), kThreads, kSmemBytes, stream,
-                                    (unsigned)split, ta, tb, p);
-    }
+  for (int split = kSplitMax; split >= 2; split /= 2) {
+    if (split > p.num_kb || p.num_tiles * split > nsm) continue;
+    // int16 partials when |a b| times this split's k-range per rank stays below 2^15
+    const int64_t kb_per = (p.num_kb + split - 1) / split;
+    const bool p16 = ab_max > 0 && (int64_t)ab_max * kb_per * kBK <= 32767;
+    if (M > (p16 ? kSplitMaxRows16 : kSplitMaxRows)) continue;
+    auto kern = p16 ? (split == 2 ? gemm_i8_splitk_kernel<2, true>
+                       : split == 4 ? gemm_i8_splitk_kernel<4, true> : gemm_i8_splitk_kernel<8, true>)
+                    : (split == 2 ? gemm_i8_splitk_kernel<2, false>
+                       : split == 4 ? gemm_i8_splitk_kernel<4, false> : gemm_i8_splitk_kernel<8, false>);
+    const int idx = (split == 2 ? 0 : split == 4 ? 1 : 2) + (p16 ? 3 : 0);
+    static bool smem_set_s[6][sm100_host::kMaxDevices] = {};
+    cudaError_t e = sm100_host::ensure_smem(kern, (int)kSmemBytes, smem_set_s[idx]);
+    if (e != cudaSuccess) return e;
+    if (p.num_tiles > max_active_clusters(kern, split, idx)) continue;
+    return sm100_host::launch_pdl(kern, (unsigned)(p.num_tiles * split), kThreads, kSmemBytes, stream,
+                                  (unsigned)split, ta, tb, p);
   }
   static bool smem_set[sm100_host::kMaxDevices] = {false};
   cudaError_t e = sm100_host::ensure_smem(gemm_i8_kernel, (int)kSmemBytes, smem_set);

@@ -185,7 +185,9 @@ hbl_status hbl_forward(const void* x, hbl_dtype xt, int64_t M, int64_t K, const 
     e = hbl::launch_ln_fht_quant(x, xt == HBL_BF16, M, l, mode, A, scales, stream);
     if (e == cudaSuccess) e = hbl::launch_widen_ternary(packed, N, K, B, stream, /*overlap_previous=*/true);
   }
-  if (e == cudaSuccess) e = hbl::launch_gemm_i8(A, B, M, N, K, yt == HBL_BF16 ? 2 : 1, y, scales, alpha_dev, stream);
+  // |code x weight| <= 8 (INT4 codes, ternary weights) or 128 (INT8)
+  if (e == cudaSuccess)
+    e = hbl::launch_gemm_i8(A, B, M, N, K, yt == HBL_BF16 ? 2 : 1, y, scales, alpha_dev, stream, bits == 4 ? 8 : 128);
   return cuda_status(e);
 }
 

@@ -161,3 +161,27 @@ def test_device_error_word(H):
     assert H.hbl_last_device_error() == H.HBL_ERR_TIMEOUT
     assert H.hbl_last_device_error() == H.HBL_OK
     torch.cuda.synchronize()
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+@pytest.mark.parametrize("M,K,N", [(5, 4096, 4096), (33, 1024, 1040), (64, 4096, 256), (65, 4096, 4096),
+                                   (100, 1024, 528), (128, 4096, 4096), (200, 2048, 1040), (255, 4096, 2048)])
+def test_forward_short_batch_split_matches_stage_path(H, orc, bits, M, K, N):
+    """Short batches split K over a cluster; with INT4 codes and ternary weights
+    each rank's partial is bounded by 8 x its k-range and is exchanged as int16
+    (M up to 255).  The sums are exact, so hbl_forward equals the stage path
+    (quantizer, then the general int8 GEMM) bit for bit."""
+    import torch
+    wl = WORKLOADS["sweep"].with_shape(M, K, N)
+    x = to_device(make_x(wl))
+    packed, alpha = H.hbl_pack_ternary(to_device(make_w(wl)))
+    y = H.hbl_forward(x, packed, alpha, N, bits)
+    codes, scales = H.hbl_fht_quant_i8(x, bits)
+    y_stage = H.hbl_gemm_dequant(codes, H.hbl_widen_ternary(packed, K), scales, alpha)
+    torch.cuda.synchronize()
+    assert torch.equal(y, y_stage)
+    rows = np.unique(np.r_[0, M - 1, np.random.default_rng(M).integers(0, M, 4)])
+    w, a = orc.ternary(make_w(wl))
+    y_exact = orc.dequant(orc.gemm_i32(to_host(codes)[rows], w), to_host(scales)[rows], a)
+    assert np.array_equal(to_host(y)[rows], orc.round_to_bf16(y_exact))
+    assert H.hbl_last_device_error() == H.HBL_OK
