@@ -1132,10 +1132,12 @@ cudaError_t launch_ln_fht_quant_tc(const void* x, int64_t M, int log2k, K1Mode m
 cudaError_t launch_ln_fht_quant_tc_widen(const void* x, int64_t M, int log2k, K1Mode mode, void* out,
                                          float* scales, const uint8_t* packed, int64_t N, int64_t K, int8_t* w,
                                          cudaStream_t stream) {
-  // The widening needs every SM's idle warps: with fewer CTAs than SMs (a
-  // short batch) it runs as its own kernel instead.
+  // The widening needs every SM's idle warps, and enough quantizer work to
+  // hide behind: with fewer CTAs than SMs, or when the weights' traffic
+  // (1.25 bytes per code) is not well below the quantizer's (3 bytes per
+  // element), it runs as its own kernel beside the quantizer instead.
   const int64_t ctas = log2k >= 14 ? M : (M * ((int64_t)1 << (log2k - 6)) + 2 * kBoxRows - 1) / (2 * kBoxRows);
-  if (M <= 0 || ctas < sm100_host::sm_count()) {
+  if (M <= 0 || ctas < sm100_host::sm_count() || 3 * M < 5 * N) {
     cudaError_t e = launch_tc_any(x, M, log2k, mode, out, scales, WidenJob(), stream);
     if (e == cudaSuccess) e = launch_widen_ternary(packed, N, K, w, stream, /*overlap_previous=*/true);
     return e;
