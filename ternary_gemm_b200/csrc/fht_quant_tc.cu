@@ -683,8 +683,8 @@ ln_fht_quant_tc_kernel(const __grid_constant__ CUtensorMap tmX, TcParams p) {
 // the 6 low stages; two exchange rounds through TMEM, each behind a barrier
 // of the two warpgroups involved, bring the partners of column bit 6 and
 // then of bit 7 together.  In 32-column units u (columns 32 u ..), warpgroup
-// g starts with units {2g, 2g+1}, holds {0,2} {1,3} {4,6} {5,7} after round
-// 1 and the final outputs {g, g+4} after round 2.  Every exchange write goes
+// g starts with units {2g, 2g+1}, holds {0,2} {1,3} {4,6} {5,7} after
+// exchange 1 and the final outputs {g, g+4} after exchange 2.  Every exchange write goes
 // to a unit nobody reads again except its receiver, and unit 0 (whose first
 // column the i_hi = 0 lanes of every warpgroup read for the mean removal) is
 // never written.
@@ -845,11 +845,11 @@ ln_fht_quant_tc256_kernel(const __grid_constant__ CUtensorMap tmX, TcParams p) {
     const int quarter = warp & 3;
     const int m = quarter * 32 + lane;  // lane = i_hi
     const int wq = 4 * g + quarter;
-    const int h1 = g & 1;               // role in round 1 (pairs {0,1}, {2,3})
+    const int h1 = g & 1;               // role in exchange 1 (pairs {0,1}, {2,3})
     const int bar_r1 = 1 + (g >> 1);
-    const int bar_r2 = 3 + (g & 1);     // round 2 pairs {0,2}, {1,3}
+    const int bar_r2 = 3 + (g & 1);     // exchange 2 pairs {0,2}, {1,3}
     const int bar_row = 5;
-    // round 2: location written, location read, and whether the kept 32
+    // exchange 2: location written, location read, and whether the kept 32
     // values are y[0..31] (else y[32..63])
     const int w2 = g == 0 ? 3 : g == 1 ? 1 : g == 2 ? 4 : 7;
     const int r2 = g == 0 ? 4 : g == 1 ? 7 : g == 2 ? 3 : 1;
@@ -887,7 +887,7 @@ ln_fht_quant_tc256_kernel(const __grid_constant__ CUtensorMap tmX, TcParams p) {
       stage<3>(y);
       stage<4>(y);
       stage<5>(y);
-      // round 1 (column bit 6): units 2g, 2g+1 -> {4(g>>1) + h1, 4(g>>1) + h1 + 2}
+      // exchange 1 (column bit 6): units 2g, 2g+1 -> {4(g>>1) + h1, 4(g>>1) + h1 + 2}
       if (h1 == 0) tm_put32(tl + (uint32_t)(64 * g + 32), &y[32]);  // hand over unit 2g+1
       else tm_put32(tl + (uint32_t)(64 * g), &y[0]);                 // hand over unit 2g
       tmem_wait_st();
@@ -898,7 +898,7 @@ ln_fht_quant_tc256_kernel(const __grid_constant__ CUtensorMap tmX, TcParams p) {
       else tm_get32(tl + (uint32_t)(64 * g - 32), &y[0]);            // partner's unit 2g-1
 #pragma unroll
       for (int r = 0; r < 32; r += 2) bfly2(y[r], y[r + 1], y[32 + r], y[33 + r]);
-      // round 2 (column bit 7)
+      // exchange 2 (column bit 7)
       if (keep_lo2) tm_put32(tl + (uint32_t)(32 * w2), &y[32]);
       else tm_put32(tl + (uint32_t)(32 * w2), &y[0]);
       tmem_wait_st();
