@@ -22,7 +22,10 @@
  *    to device memory of the current CUDA device, 16-byte aligned.  The library
  *    never allocates or frees memory, never synchronises the stream (except
  *    hbl_last_device_error) and keeps no state between calls other than the
- *    device error word read by hbl_last_device_error.
+ *    device error word read by hbl_last_device_error, per-device caches of
+ *    queried values (SM count, kernel attributes, cluster occupancy, symbol
+ *    addresses; each set once, the same value by every thread), and the
+ *    fixed scratch area of hbl_forward_noalloc.
  *  - Work is enqueued on `stream` (0 = legacy default stream) and is
  *    asynchronous; outputs are valid once the stream reaches that point.
  *  - Arguments are checked on the host before any launch.  A failed check
