@@ -52,7 +52,7 @@ def parse_args(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
-    ap.add_argument("--sweep", choices=["k1", "fwd", "k1_noh", "bwd", "kv"], default=None,
+    ap.add_argument("--sweep", choices=["k1", "fwd", "k1_noh", "bwd", "kv", "lib"], default=None,
                     help="instead of the step line: the LN+FHT+INT4 kernel alone at M=65536 for each K, "
                          "or the whole forward at K=N=4096 for each M (one JSON line per point)")
     ap.add_argument("--shape", default=None,
@@ -532,6 +532,53 @@ def bench_sweep(args):
                               "frac_hbm": gbs / peaks["hbm_gbs"], "peak_kind": peak_kind,
                               "bytes_per_launch": nbytes, "input": "seeded N(0, 4) bf16 head vectors"}),
                   flush=True)
+        return 0
+    if args.sweep == "lib":
+        # the int8 GEMM beside the library's (torch._int_mm, cuBLASLt) and a bf16 GEMM of
+        # the same shape (torch.matmul, cuBLAS), on INT4-range codes and ternary weights;
+        # the arms alternate in blocks of launches so that clock drift hits them alike
+        g = torch.Generator(device="cuda").manual_seed(11)
+        for name, (M, K, N) in (("wo_1p3b", (4096, 2048, 2048)), ("wdown_3b", (8192, 8192, 2560)),
+                                ("wdown_7b", (8192, 16384, 4096))):
+            A = torch.randint(-8, 8, (M, K), device="cuda", generator=g, dtype=torch.int8)
+            w = torch.randint(-1, 2, (N, K), device="cuda", generator=g, dtype=torch.int8)
+            acc = torch.empty((M, N), dtype=torch.int32, device="cuda")
+            Ab, wb = A.to(torch.bfloat16), w.to(torch.bfloat16)
+            sc = torch.rand((M,), device="cuda", generator=g)
+            al = torch.full((1,), 0.01, device="cuda")
+            y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+            # ours: int32 sums (the library's output type) and the forward's GEMM (dequantised bf16 y)
+            arms = {"ours": lambda: hbl.hbl_gemm_i8_i32(A, w, acc=acc),
+                    "ours_dequant_bf16": lambda: hbl.hbl_gemm_dequant(A, w, sc, al, y=y),
+                    "cublas_bf16": lambda: torch.matmul(Ab, wb.t())}
+            arm_unit = {"ours": "_int8_tops", "ours_dequant_bf16": "_int8_tops", "cublaslt": "_int8_tops",
+                        "cublas_bf16": "_tflops"}
+            same = None
+            try:
+                same = bool(torch.equal(torch._int_mm(A, w.t()), hbl.hbl_gemm_i8_i32(A, w, acc=acc)))
+                arms["cublaslt"] = lambda: torch._int_mm(A, w.t())
+            except RuntimeError as e:     # no int8 library GEMM for this device or shape
+                same = str(e).splitlines()[0]
+            n = 10 if K >= 8192 else 40
+            ts = {k: [] for k in arms}
+            clocks = ClockSampler("GPU-" + str(torch.cuda.get_device_properties(0).uuid))
+            clocks.start()
+            for r in range(16):
+                for k in (list(arms) if r % 2 == 0 else list(arms)[::-1]):
+                    ts[k].append(timed(arms[k], n))
+            clk = clocks.stop()
+            ops = 2.0 * M * N * K
+            out = {"sweep": "gemm_vs_library", "workload": name, "M": M, "K": K, "N": N}
+            for k, v in ts.items():
+                t = sorted(v)[len(v) // 2]
+                out[k + "_us"] = t * 1e6
+                out[k + arm_unit[k]] = ops / t / 1e12
+            out["int32_results_identical"] = same
+            out["clocks"] = clk
+            out["timing"] = "CUDA events; median of 16 blocks of %d launches, the arms alternating" % n
+            print(json.dumps(out), flush=True)
+            del A, w, acc, Ab, wb, arms, y
+            torch.cuda.empty_cache()
         return 0
     if args.sweep in ("k1", "k1_noh"):
         M, ks = 65536, SWEEP_K1_KS

@@ -74,6 +74,22 @@ def test_gemm_exact(H, orc, M, N, K):
     assert np.array_equal(acc, orc.gemm_i32(A, B))
 
 
+@pytest.mark.parametrize("M,N,K", [(2000, 2544, 1024), (2048, 1536, 512), (3072, 1344, 384), (8192, 2560, 1024),
+                                   (4096, 2048, 2048), (256, 512, 256)])
+def test_gemm_exact_2sm_shapes(H, orc, M, N, K):
+    """The 2-SM kernel at shapes whose last round of tiles is partly empty (the
+    3B and 1.3B shapes among them), with ragged rows and columns at the first:
+    every column, rows sampled from every 256-row tile and the ragged tail."""
+    rng = np.random.default_rng(M + 3 * N + 5 * K)
+    A = rng.integers(-128, 128, (M, K)).astype(np.int8)
+    B = rng.integers(-128, 128, (N, K)).astype(np.int8)
+    acc = to_host(H.hbl_gemm_i8_i32(to_device(A), to_device(B)))
+    rows = np.unique(np.r_[np.arange(0, M, 256), np.arange(255, M, 256), M - 1,
+                           rng.integers(0, M, 24)])
+    rows = rows[rows < M]
+    assert np.array_equal(acc[rows], orc.gemm_i32(A[rows], B))
+
+
 @pytest.mark.slow
 def test_gemm_exact_7b_shape_sampled(H, orc):
     M, N, K = 8192, 4096, 16384
