@@ -56,7 +56,8 @@ def parse_args(argv=None):
                     help="instead of the step line: the LN+FHT+INT4 kernel alone at M=65536 for each K, "
                          "or the whole forward at K=N=4096 for each M (one JSON line per point)")
     ap.add_argument("--shape", default=None,
-                    help="with --sweep k1 or k1_noh: one point M,K instead of the sweep (e.g. for a profiler)")
+                    help="with --sweep k1 or k1_noh: one point M,K instead of the sweep (e.g. for a profiler); "
+                         "with --sweep lib: one shape M,K,N")
     a = ap.parse_args(argv)
     a.warmup = max(3, a.warmup)
     return a
@@ -538,8 +539,13 @@ def bench_sweep(args):
         # the same shape (torch.matmul, cuBLAS), on INT4-range codes and ternary weights;
         # the arms alternate in blocks of launches so that clock drift hits them alike
         g = torch.Generator(device="cuda").manual_seed(11)
-        for name, (M, K, N) in (("wo_1p3b", (4096, 2048, 2048)), ("wdown_3b", (8192, 8192, 2560)),
-                                ("wdown_7b", (8192, 16384, 4096))):
+        shapes = (("wo_1p3b", (4096, 2048, 2048)), ("wdown_3b", (8192, 8192, 2560)), ("wdown_7b", (8192, 16384, 4096)))
+        if args.shape:
+            shape = tuple(int(v) for v in args.shape.split(","))
+            if len(shape) != 3:
+                raise SystemExit("--shape with --sweep lib: M,K,N")
+            shapes = (("%dx%dx%d" % shape, shape),)
+        for name, (M, K, N) in shapes:
             A = torch.randint(-8, 8, (M, K), device="cuda", generator=g, dtype=torch.int8)
             w = torch.randint(-1, 2, (N, K), device="cuda", generator=g, dtype=torch.int8)
             acc = torch.empty((M, N), dtype=torch.int32, device="cuda")

@@ -249,7 +249,8 @@ gemm_i8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           int32_t* yrow = reinterpret_cast<int32_t*>(p.y) + (size_t)row * p.N;
 #pragma unroll
           for (int j = 0; j < 32; j += 4)
-            if (col0 + j < p.N) *reinterpret_cast<uint4*>(yrow + col0 + j) = make_uint4(r[j], r[j + 1], r[j + 2], r[j + 3]);
+            if (col0 + j < p.N)
+              __stcs(reinterpret_cast<uint4*>(yrow + col0 + j), make_uint4(r[j], r[j + 1], r[j + 2], r[j + 3]));
         } else if (p.y_mode == 1) {
           float* yrow = reinterpret_cast<float*>(p.y) + (size_t)row * p.N;
 #pragma unroll
@@ -336,7 +337,8 @@ __device__ __forceinline__ void epilogue_tile(const Params& p, uint32_t tbase, i
       int32_t* yrow = reinterpret_cast<int32_t*>(p.y) + (size_t)row * p.N;
 #pragma unroll
       for (int j = 0; j < 32; j += 4)
-        if (col0 + j < p.N) *reinterpret_cast<uint4*>(yrow + col0 + j) = make_uint4(r[j], r[j + 1], r[j + 2], r[j + 3]);
+        if (col0 + j < p.N)
+          __stcs(reinterpret_cast<uint4*>(yrow + col0 + j), make_uint4(r[j], r[j + 1], r[j + 2], r[j + 3]));
     } else if (p.y_mode == 1) {
       float* yrow = reinterpret_cast<float*>(p.y) + (size_t)row * p.N;
 #pragma unroll
@@ -564,8 +566,8 @@ __device__ __forceinline__ uint4 ld_cluster_v4(uint32_t addr) {
 // y[row][col .. col + 3] from four int32 sums (col + 3 < N, 16-byte-aligned rows)
 __device__ __forceinline__ void store_y4(const Params& p, int row, int col, const int (&v)[4], float sa) {
   if (p.y_mode == 0) {
-    *reinterpret_cast<int4*>(reinterpret_cast<int32_t*>(p.y) + (size_t)row * p.N + col) =
-        make_int4(v[0], v[1], v[2], v[3]);
+    __stcs(reinterpret_cast<int4*>(reinterpret_cast<int32_t*>(p.y) + (size_t)row * p.N + col),
+           make_int4(v[0], v[1], v[2], v[3]));
   } else if (p.y_mode == 1) {
     float4 o;
     o.x = __fmul_rn(__int2float_rn(v[0]), sa);
