@@ -10,8 +10,12 @@ numpy arrays into it.  Each wrapper names the step of the method it follows
 ("BitNet v2: Native 4-bit Activations with Hadamard Transformation for 1-bit
 LLMs", arXiv 2504.18415, section "H-BitLinear").
 
-Parity pins: every function here is pinned by ``tests/test_oracle_pins.py``
-against closed forms, hand-worked examples, library routines and brute force.
+Parity pins: every function here is pinned against closed forms, hand-worked
+examples, library routines, finite differences and brute force
+(``tests/test_oracle_pins.py`` for the forward, ``tests/test_oracle_backward_pins.py``
+for the backward pass, ``tests/test_oracle_kv_pins.py`` for the QKV-state
+quantizer), and ``tests/test_oracle_mutations.py`` checks that a planted slip in
+the C arithmetic or in the Python steps fails those pins.
 The model-level claims of the pages (perplexity, zero-shot accuracy) are
 "parity unpinned": they need trained weights and evaluation datasets.
 """

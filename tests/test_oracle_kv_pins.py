@@ -61,3 +61,22 @@ def test_kv_mirror_symmetry(orc, bits):
     np.testing.assert_array_equal(s1, s2)
     # exact ties (x r + L/2 on a half-integer) could break the mirror; random data has none
     np.testing.assert_array_equal(c1.astype(int) + c2.astype(int), L)
+
+
+@pytest.mark.parametrize("bits", [2, 3, 8])
+def test_kv_dequant_error_bound_and_end_levels(orc, bits):
+    """x~ = (2 q - L) gamma / L: every value within half a step of x (the step
+    of the grid the codes were chosen on, 2 (gamma + eps) / L, plus the eps that
+    separates that grid from the one x~ lies on), and the absmax element comes
+    back exactly."""
+    rng = np.random.default_rng(7 + bits)
+    x = (rng.standard_normal((48, 64)) * rng.uniform(0.05, 20.0, (48, 1))).astype(np.float32)
+    codes, scales = orc.kv_quant(x, bits)
+    xr = orc.kv_dequant(codes, scales, bits)
+    L = (1 << bits) - 1
+    g = scales.astype(np.float64)
+    bound = (g + 1e-5) / L + 1e-5
+    assert np.all(np.abs(x.astype(np.float64) - xr) <= bound[:, None] * (1 + 1e-6))
+    for m in range(x.shape[0]):
+        i = int(np.argmax(np.abs(x[m])))
+        assert xr[m, i] == np.float64(x[m, i])

@@ -1,9 +1,11 @@
 """The pins catch plausible mistakes: each mutant below is a copy of the oracle
-with one planted slip, compiled on the CPU; the pin suite must fail on every
-one of them (and pass on the unmodified oracle, which test_oracle_pins checks).
+with one planted slip (in the C arithmetic, compiled on the CPU, or in the
+Python steps of the oracle package); the pin suite must fail on every one of
+them (and pass on the unmodified oracle, which the pin files check).
 """
 import concurrent.futures as cf
 import os
+import shutil
 import subprocess
 import sys
 import tempfile
@@ -12,6 +14,9 @@ import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 SRC = os.path.join(ROOT, "oracle", "hbl_oracle.c")
+PY_SRC = os.path.join(ROOT, "oracle", "__init__.py")
+PIN_FILES = [os.path.join(ROOT, "tests", f)
+             for f in ("test_oracle_pins.py", "test_oracle_backward_pins.py", "test_oracle_kv_pins.py")]
 
 # (name, text in hbl_oracle.c, replacement)
 MUTANTS = [
@@ -57,6 +62,34 @@ MUTANTS = [
 ]
 
 
+# slips in the Python steps of the oracle package: (name, text in oracle/__init__.py, replacement)
+PY_MUTANTS = [
+    ("backward g_t without alpha", "g_t = float(alpha) * (gy @ np.asarray(w, dtype=np.float64))",
+     "g_t = gy @ np.asarray(w, dtype=np.float64)"),
+    ("backward g_u without 1/sqrt(K)", "g_u = np.stack([fht_unnormalized(r) for r in g_t]) / np.sqrt(float(K))",
+     "g_u = np.stack([fht_unnormalized(r) for r in g_t])"),
+    ("backward weight columns reversed", "g_t = float(alpha) * (gy @ np.asarray(w, dtype=np.float64))",
+     "g_t = float(alpha) * (gy @ np.asarray(w, dtype=np.float64)[:, ::-1])"),
+    ("weight gradient without the scales",
+     "a = np.asarray(codes, dtype=np.float64) * np.asarray(scales, dtype=np.float64)[:, None]",
+     "a = np.asarray(codes, dtype=np.float64)"),
+    ("KV dequant without the doubling", "return (2.0 * np.asarray(codes, np.float64) - L)",
+     "return (np.asarray(codes, np.float64) - L)"),
+    ("KV dequant over 2^b", "L = float((1 << bits) - 1)\n    return", "L = float(1 << bits)\n    return"),
+]
+
+
+def _pytest(env, pre_import=None):
+    if pre_import is None:
+        cmd = [sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider"] + PIN_FILES
+    else:
+        # import the mutated package first, so the tests' own import finds it in sys.modules
+        code = ("import sys, pytest; sys.path.insert(0, %r); import oracle; "
+                "sys.exit(pytest.main(['-x', '-q', '-p', 'no:cacheprovider'] + %r))" % (pre_import, PIN_FILES))
+        cmd = [sys.executable, "-c", code]
+    return subprocess.run(cmd, env=env, capture_output=True, text=True, timeout=600, cwd=ROOT)
+
+
 def _run_mutant(m):
     name, old, new = m
     src = open(SRC).read()
@@ -67,17 +100,37 @@ def _run_mutant(m):
         open(c, "w").write(src.replace(old, new))
         subprocess.run(["gcc", "-O2", "-ffp-contract=off", "-std=c11", "-fPIC", "-shared", "-o", so, c, "-lm"],
                        check=True)
-        env = dict(os.environ, HBL_ORACLE_LIB=so)
-        p = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
-                            os.path.join(ROOT, "tests", "test_oracle_pins.py"),
-                            os.path.join(ROOT, "tests", "test_oracle_backward_pins.py"),
-                            os.path.join(ROOT, "tests", "test_oracle_kv_pins.py")],
-                           env=env, capture_output=True, text=True, timeout=600)
+        p = _pytest(dict(os.environ, HBL_ORACLE_LIB=so))
         return name, p.returncode, p.stdout[-400:]
+
+
+def _run_py_mutant(m):
+    name, old, new = m
+    src = open(PY_SRC).read()
+    assert src.count(old) == 1, name
+    with tempfile.TemporaryDirectory() as d:
+        pkg = os.path.join(d, "oracle")
+        os.makedirs(pkg)
+        shutil.copy2(SRC, os.path.join(pkg, "hbl_oracle.c"))
+        open(os.path.join(pkg, "__init__.py"), "w").write(src.replace(old, new))
+        p = _pytest(dict(os.environ), pre_import=d)
+        return name, p.returncode, p.stdout[-400:]
+
+
+def test_python_mutants_load_the_mutated_package():
+    """The harness really runs the pins against the copy: an unmodified copy passes."""
+    with tempfile.TemporaryDirectory() as d:
+        pkg = os.path.join(d, "oracle")
+        os.makedirs(pkg)
+        shutil.copy2(SRC, os.path.join(pkg, "hbl_oracle.c"))
+        open(os.path.join(pkg, "__init__.py"), "w").write(open(PY_SRC).read() + "\nMUTATED_COPY = True\n")
+        code = ("import sys; sys.path.insert(0, %r); import oracle; "
+                "sys.path.insert(0, %r); import oracle as o2; assert o2.MUTATED_COPY" % (d, ROOT))
+        subprocess.run([sys.executable, "-c", code], check=True, cwd=ROOT)
 
 
 def test_every_planted_mistake_fails_a_pin():
     with cf.ThreadPoolExecutor(max_workers=min(8, os.cpu_count() or 1)) as ex:
-        results = list(ex.map(_run_mutant, MUTANTS))
+        results = list(ex.map(_run_mutant, MUTANTS)) + list(ex.map(_run_py_mutant, PY_MUTANTS))
     survivors = [(n, out) for n, rc, out in results if rc == 0]
     assert not survivors, "mutants not caught by any pin: %s" % [n for n, _ in survivors]
