@@ -103,6 +103,101 @@ def test_norm_quant_validation(L):
     assert L.hbl_debug_norm(FAKE, 1, 0, 1024, 1, FAKE, S0) == hbl.HBL_ERR_INVALID_ARG
 
 
+def test_stage_validation(L):
+    E_ARG, E_UNS = hbl.HBL_ERR_INVALID_ARG, hbl.HBL_ERR_UNSUPPORTED
+    # activation path with int8 codes
+    assert L.hbl_fht_quant_i8(FAKE, 1, 8, 256, 6, FAKE, FAKE, S0) == E_ARG
+    assert L.hbl_fht_quant_i8(FAKE, 1, 8, 96, 4, FAKE, FAKE, S0) == E_UNS
+    assert L.hbl_fht_quant_i8(FAKE, 1, 0, 256, 4, FAKE, FAKE, S0) == E_ARG
+    assert L.hbl_fht_quant_i8(FAKE, 1, 8, 256, 4, FAKE_ODD, FAKE, S0) == E_ARG
+    # weight widening
+    assert L.hbl_widen_ternary(NULL, 256, 256, FAKE, S0) == E_ARG
+    assert L.hbl_widen_ternary(FAKE, 256, 24, FAKE, S0) == E_UNS
+    assert L.hbl_widen_ternary(FAKE, 200, 256, FAKE, S0) == E_UNS
+    # GEMM + dequantisation
+    assert L.hbl_gemm_dequant(FAKE, FAKE, 8, 256, 256, FAKE, NULL, FAKE, 1, S0) == E_ARG
+    assert L.hbl_gemm_dequant(FAKE, FAKE, 8, 256, 256, FAKE, FAKE, FAKE, 3, S0) == E_ARG
+    assert L.hbl_gemm_dequant(FAKE, FAKE, 8, 256, 72, FAKE, FAKE, FAKE, 1, S0) == E_UNS
+    assert L.hbl_gemm_dequant(FAKE, FAKE, 8, 40, 256, FAKE, FAKE, FAKE, 1, S0) == E_UNS
+    assert L.hbl_gemm_dequant(FAKE, FAKE, 8, 256, 1 << 17, FAKE, FAKE, FAKE, 1, S0) == E_UNS
+    # the packed-weight product is for decode-sized batches only
+    assert L.hbl_gemv_ternary_dequant(FAKE, FAKE, 5, 256, 4096, FAKE, FAKE, FAKE, 1, S0) == E_UNS
+    assert L.hbl_gemv_ternary_dequant(FAKE, FAKE, 4, 256, 32768, FAKE, FAKE, FAKE, 1, S0) == E_UNS
+    assert L.hbl_gemv_ternary_dequant(FAKE, FAKE, 1, 24, 4096, FAKE, FAKE, FAKE, 1, S0) == E_UNS
+    assert L.hbl_gemv_ternary_dequant(FAKE, NULL, 1, 256, 4096, FAKE, FAKE, FAKE, 1, S0) == E_ARG
+    # transform alone and the rotated packing
+    assert L.hbl_fht(FAKE, 1, 8, 100, FAKE, S0) == E_UNS
+    assert L.hbl_fht(FAKE, 2, 8, 256, FAKE, S0) == E_ARG
+    assert hbl.hbl_pack_ternary_rotated_workspace_bytes(256, 256) >= 256 * 256 * 4
+    assert hbl.hbl_pack_ternary_rotated_workspace_bytes(100, 256) == 0
+    need = hbl.hbl_pack_ternary_rotated_workspace_bytes(256, 256)
+    assert L.hbl_pack_ternary_rotated(FAKE, 1, 256, 256, FAKE, FAKE, FAKE, need - 1, S0) == hbl.HBL_ERR_WORKSPACE
+    assert L.hbl_pack_ternary_rotated(FAKE, 1, 256, 24, FAKE, FAKE, FAKE, need, S0) == E_UNS
+
+
+def test_forward_noalloc_validation(L):
+    f = L.hbl_forward_noalloc
+    assert f(NULL, 1, 8, 256, FAKE, FAKE, 256, 4, FAKE, 1, S0) == hbl.HBL_ERR_INVALID_ARG
+    assert f(FAKE, 1, 8, 256, FAKE, FAKE, 24, 4, FAKE, 1, S0) == hbl.HBL_ERR_UNSUPPORTED
+    # the 7B Wdown forward needs more than the library's 32 MiB area: refused before any CUDA call
+    assert hbl.hbl_forward_workspace_bytes(8192, 16384, 4096, 4) > (32 << 20)
+    assert f(FAKE, 1, 8192, 16384, FAKE, FAKE, 4096, 4, FAKE, 1, S0) == hbl.HBL_ERR_WORKSPACE
+    assert L.hbl_last_cuda_error() == 0
+
+
+def test_backward_validation(L):
+    E_ARG, E_UNS, E_WS = hbl.HBL_ERR_INVALID_ARG, hbl.HBL_ERR_UNSUPPORTED, hbl.HBL_ERR_WORKSPACE
+    ws = hbl.hbl_backward_workspace_bytes(64, 1024, 256, 4)
+    # the forward's codes (int8) and the bf16 copies of w, q and g_y live in the workspace
+    assert ws >= 64 * 1024 + 256 * 1024 * 2 + 64 * 1024 * 2 + 64 * 256 * 2
+    assert hbl.hbl_backward_workspace_bytes(64, 1000, 256, 4) == 0
+    assert hbl.hbl_backward_workspace_bytes(64, 1024, 24, 4) == 0
+    assert hbl.hbl_backward_workspace_bytes(64, 1024, 256, 5) == 0
+    assert hbl.hbl_backward_workspace_bytes(0, 1024, 256, 4) == 0
+    f = L.hbl_backward
+    args = [FAKE, 1, 64, 1024, FAKE, FAKE, 256, 4, FAKE, 1, FAKE, FAKE, FAKE, ws, S0]
+
+    def call(**kw):
+        a = list(args)
+        for i, v in kw.items():
+            a[int(i[1:])] = v
+        return f(*a)
+
+    assert call(a0=NULL) == E_ARG              # x
+    assert call(a7=6) == E_ARG                 # bits
+    assert call(a9=5) == E_ARG                 # g_y dtype
+    assert call(a11=FAKE_ODD) == E_ARG         # g_W alignment
+    assert call(a3=96) == E_UNS                # K not a power of two
+    assert call(a6=40) == E_UNS                # N not a multiple of 16
+    assert call(a12=NULL) == E_WS
+    assert call(a13=ws - 1) == E_WS
+    assert call(a12=ctypes.c_void_p(0x10010)) == E_WS   # 256-byte alignment
+    # the products and the LayerNorm backward alone
+    g = L.hbl_gemm_bf16_f32
+    assert g(FAKE, 0, FAKE, 128, 256, 12, FAKE, NULL, S0) == E_UNS    # K-major A: Kc % 8
+    assert g(FAKE, 1, FAKE, 12, 256, 64, FAKE, NULL, S0) == E_UNS     # MN-major A: R % 8
+    assert g(FAKE, 0, FAKE, 128, 20, 64, FAKE, NULL, S0) == E_UNS     # C % 8
+    assert g(FAKE, 0, FAKE, 0, 256, 64, FAKE, NULL, S0) == E_ARG
+    assert g(FAKE, 0, FAKE, 128, 256, 64, FAKE, FAKE_ODD, S0) == E_ARG
+    assert L.hbl_ln_backward(FAKE, 1, 8, 48, FAKE, FAKE, S0) == E_UNS
+    assert L.hbl_ln_backward(FAKE, 1, 8, 1024, NULL, FAKE, S0) == E_ARG
+    assert L.hbl_fht_ln_backward(FAKE, FAKE, 1, 8, 65536, FAKE, S0) == E_UNS
+    assert L.hbl_fht_ln_backward(FAKE, FAKE, 3, 8, 1024, FAKE, S0) == E_ARG
+
+
+def test_kv_quant_validation(L):
+    f = L.hbl_kv_quant
+    E_ARG, E_UNS = hbl.HBL_ERR_INVALID_ARG, hbl.HBL_ERR_UNSUPPORTED
+    assert f(FAKE, 1, 64, 96, 3, FAKE, FAKE, S0) == E_UNS      # head dimension
+    assert f(FAKE, 1, 64, 128, 1, FAKE, FAKE, S0) == E_UNS     # one bit
+    assert f(FAKE, 1, 64, 128, 9, FAKE, FAKE, S0) == E_UNS
+    assert f(FAKE, 1, 64, 128, 0, FAKE, FAKE, S0) == E_ARG
+    assert f(FAKE, 1, 0, 128, 3, FAKE, FAKE, S0) == E_ARG
+    assert f(FAKE, 1, 64, 128, 3, FAKE_ODD, FAKE, S0) == E_ARG
+    assert f(NULL, 1, 64, 128, 3, FAKE, FAKE, S0) == E_ARG
+    assert L.hbl_last_cuda_error() == 0
+
+
 def test_status_strings(L):
     assert hbl.status_string(hbl.HBL_OK) == "HBL_OK"
     assert hbl.status_string(hbl.HBL_ERR_TIMEOUT) == "HBL_ERR_TIMEOUT"
