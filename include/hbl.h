@@ -262,7 +262,8 @@ hbl_status hbl_backward(const void* x, hbl_dtype xt, int64_t M, int64_t K, const
  * bf16: a_mn = 0 stored [R][Kc] (K-major), a_mn = 1 stored [Kc][R]; B device
  * bf16 stored [Kc][C]; D device float [R][C]; scale_dev a device float or
  * NULL for 1.  All 16-byte aligned; C a multiple of 8, and R (a_mn = 1) or Kc
- * (a_mn = 0) a multiple of 8 (HBL_ERR_UNSUPPORTED otherwise). */
+ * (a_mn = 0) a multiple of 8, R * C at most 2^40 (HBL_ERR_UNSUPPORTED
+ * otherwise). */
 hbl_status hbl_gemm_bf16_f32(const uint16_t* A, int a_mn, const uint16_t* B, int64_t R, int64_t C, int64_t Kc,
                              float* D, const float* scale_dev, cudaStream_t stream);
 

@@ -179,7 +179,8 @@ hbl_status hbl_forward(const void* x, hbl_dtype xt, int64_t M, int64_t K, const 
     return cuda_status(e);
   }
   if (hbl::ln_fht_quant_tc_supports(xt == HBL_BF16, l, mode, x, A)) {
-    // the weight widening runs inside the quantizer kernel (its idle warps)
+    // the quantizer, with the weight widening in its idle warps when the
+    // quantizer's traffic dominates, else in a kernel that overlaps it
     e = hbl::launch_ln_fht_quant_tc_widen(x, M, l, mode, A, scales, packed, N, K, B, stream);
   } else {
     e = hbl::launch_ln_fht_quant(x, xt == HBL_BF16, M, l, mode, A, scales, stream);
@@ -395,6 +396,7 @@ hbl_status hbl_gemm_bf16_f32(const uint16_t* A, int a_mn, const uint16_t* B, int
   if (R <= 0 || C <= 0 || Kc <= 0) return HBL_ERR_INVALID_ARG;
   if (R > kMaxRows || C > kMaxRows || Kc > kMaxRows || C % 8 != 0 || (a_mn ? R % 8 : Kc % 8) != 0)
     return HBL_ERR_UNSUPPORTED;
+  if (R * C > (int64_t(1) << 40)) return HBL_ERR_UNSUPPORTED;  // keeps the tile count within int
   return cuda_status(hbl::launch_gemm_bf16(A, a_mn != 0, B, R, C, Kc, D, scale_dev, stream));
 }
 

@@ -178,6 +178,7 @@ def test_backward_validation(L):
     assert g(FAKE, 1, FAKE, 12, 256, 64, FAKE, NULL, S0) == E_UNS     # MN-major A: R % 8
     assert g(FAKE, 0, FAKE, 128, 20, 64, FAKE, NULL, S0) == E_UNS     # C % 8
     assert g(FAKE, 0, FAKE, 0, 256, 64, FAKE, NULL, S0) == E_ARG
+    assert g(FAKE, 0, FAKE, 1 << 26, 1 << 26, 64, FAKE, NULL, S0) == E_UNS   # tile count beyond int
     assert g(FAKE, 0, FAKE, 128, 256, 64, FAKE, FAKE_ODD, S0) == E_ARG
     assert L.hbl_ln_backward(FAKE, 1, 8, 48, FAKE, FAKE, S0) == E_UNS
     assert L.hbl_ln_backward(FAKE, 1, 8, 1024, NULL, FAKE, S0) == E_ARG
