@@ -22,17 +22,20 @@
  *    to device memory of the current CUDA device, 16-byte aligned.  The library
  *    never allocates or frees memory, never synchronises the stream (except
  *    hbl_last_device_error) and keeps no state between calls other than the
- *    device error word read by hbl_last_device_error, per-device caches of
- *    queried values (SM count, kernel attributes, cluster occupancy, symbol
- *    addresses; each set once, the same value by every thread), and the
- *    fixed scratch area of hbl_forward_noalloc.
+ *    device error word read by hbl_last_device_error, each host thread's
+ *    last CUDA error code (hbl_last_cuda_error), per-device caches of queried
+ *    values (SM count, kernel attributes, cluster occupancy, symbol addresses;
+ *    each filled on first use with the same value whichever thread fills it,
+ *    so concurrent first calls only repeat the query), and the fixed scratch
+ *    area of hbl_forward_noalloc.
  *  - Work is enqueued on `stream` (0 = legacy default stream) and is
  *    asynchronous; outputs are valid once the stream reaches that point.
  *  - Arguments are checked on the host before any launch.  A failed check
  *    returns an error status and enqueues nothing.  Launch failures return
  *    HBL_ERR_CUDA.  Nothing traps, asserts or exits.
- *  - Supported sizes: K a power of two with 64 <= K <= 32768; M >= 1;
- *    N >= 16 and a multiple of 16 (forward, ternary packing).
+ *  - Supported sizes: K a power of two with 64 <= K <= 32768; 1 <= M <= 2^26;
+ *    N a multiple of 16 with 16 <= N <= 2^20 (forward, ternary packing).
+ *    Entry points that differ say so below.
  *  - Row-major layouts throughout.  x is [M][K]; W is [N][K] (out x in, the
  *    layout of a PyTorch Linear weight); y is [M][N].
  */
