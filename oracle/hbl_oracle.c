@@ -28,6 +28,15 @@
  *   dequant : y[m][n] = (float)acc[m][n] * (scale[m] * alpha).
  * eps = 1e-5 for every quantizer; rint rounds half to even.
  *
+ * Beside the forward (the next steps the pages describe):
+ *   LN backward : g_x = (g_u - mean g_u - u mean(g_u u)) / sqrt(var + eps_ln),
+ *                 the LayerNorm gradient the straight-through estimator needs
+ *                 (training strategy: gradients bypass the quantizers);
+ *   QKV states  : gamma = max|x| per head vector, L = 2^b - 1,
+ *                 q = clip(rint(x L / (2 (gamma+eps)) + L/2), 0, L), scale = gamma
+ *                 (low-bit attention: heads to unsigned integers by absmax);
+ *   RMSNorm     : x / sqrt(mean x^2 + eps_ln), for the layers without the transform.
+ *
  * Precision: LN and the Hadamard transform run in double (the reference
  * precision).  The quantizers take the single-precision FHT output and make
  * their integer decisions in single precision, as the GPU does: the mean of
