@@ -22,12 +22,13 @@
  *    to device memory of the current CUDA device, 16-byte aligned.  The library
  *    never allocates or frees memory, never synchronises the stream (except
  *    hbl_last_device_error) and keeps no state between calls other than the
- *    device error word read by hbl_last_device_error, each host thread's
+ *    device status (the error word read by hbl_last_device_error and the
+ *    kernels' wait limit, hbl_debug_set_wait_limit_ns), each host thread's
  *    last CUDA error code (hbl_last_cuda_error), per-device caches of queried
  *    values (SM count, kernel attributes, cluster occupancy, symbol addresses;
- *    each filled on first use with the same value whichever thread fills it,
- *    so concurrent first calls only repeat the query), and the fixed scratch
- *    area of hbl_forward_noalloc.
+ *    atomics filled on first use with the same value whichever thread fills
+ *    them, so concurrent first calls only repeat the query), and the fixed
+ *    scratch area of hbl_forward_noalloc.
  *  - Work is enqueued on `stream` (0 = legacy default stream) and is
  *    asynchronous; outputs are valid once the stream reaches that point.
  *  - Arguments are checked on the host before any launch.  A failed check
@@ -223,9 +224,12 @@ hbl_status hbl_gemv_ternary_dequant(const int8_t* A, const uint8_t* packed, int6
  * hbl_forward_workspace_bytes(M, K, N, bits) exceeds 32 MiB are rejected with
  * HBL_ERR_WORKSPACE before anything is launched; other argument errors are
  * those of hbl_forward.  It calls no allocator.
- *  - The first call on a device (with that device current) looks up the
- *    area's device address once (cudaGetSymbolAddress, a query); make that
- *    first call before any stream capture.
+ *  - Each call made outside stream capture (with the device current) looks
+ *    up the area's device address (cudaGetSymbolAddress, a query) and
+ *    remembers it; a call made during capture uses the remembered address,
+ *    so make the first call on a device before any stream capture (a
+ *    captured first call returns HBL_ERR_CUDA).  The lookup on every
+ *    uncaptured call keeps the address valid after cudaDeviceReset.
  *  - All calls share the area, which keeps the last call's contents; nothing
  *    in it needs to start at zero.  Calls whose kernels overlap on the GPU
  *    (other streams, unordered host threads) race on it: serialise them. */
@@ -329,6 +333,15 @@ hbl_status hbl_last_device_error(cudaStream_t stream);
 /* Sets the device error word as a kernel would on a bounded-wait timeout
  * (used by the tests of the error path; enqueued on `stream`). */
 hbl_status hbl_debug_raise_device_error(cudaStream_t stream);
+
+/* Limit, in nanoseconds, of the kernels' pipeline waits on the current device
+ * (each mbarrier wait of a producer, MMA issuer or epilogue gives up after it,
+ * sets the device error word and leaves; its CTA then waits, for at most 2 s,
+ * for the copies it issued before it exits).  0 restores the default of 2 s.
+ * A test hook: a limit shorter than a kernel's run makes a wait run out so
+ * that the error path can be tested without a fault.  Synchronises the device
+ * before it changes the limit. */
+hbl_status hbl_debug_set_wait_limit_ns(uint64_t ns);
 
 /* Static string for a status code. */
 const char* hbl_status_string(hbl_status status);

@@ -110,6 +110,8 @@ def lib():
             L.hbl_last_device_error.restype = i32
             L.hbl_debug_raise_device_error.argtypes = [p]
             L.hbl_debug_raise_device_error.restype = i32
+            L.hbl_debug_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
+            L.hbl_debug_set_wait_limit_ns.restype = i32
             L.hbl_status_string.argtypes = [i32]
             L.hbl_status_string.restype = ctypes.c_char_p
             L.hbl_last_cuda_error.argtypes = []
@@ -463,3 +465,8 @@ def hbl_last_device_error(stream=None) -> int:
 
 def hbl_debug_raise_device_error(stream=None):
     _check(lib().hbl_debug_raise_device_error(_stream(stream)), "hbl_debug_raise_device_error")
+
+
+def hbl_debug_set_wait_limit_ns(ns: int):
+    """Limit of the kernels' pipeline waits on the current device (0: 2 s)."""
+    _check(lib().hbl_debug_set_wait_limit_ns(int(ns)), "hbl_debug_set_wait_limit_ns")

@@ -109,5 +109,8 @@ cudaError_t launch_fht_ln_backward(const float* g, const void* x, bool x_bf16, i
 hbl_status note_cuda_error(cudaError_t e);
 cudaError_t read_and_clear_device_error(cudaStream_t stream, int* value);
 cudaError_t raise_device_error(cudaStream_t stream);
+// Limit of the kernels' pipeline waits on the current device (0: the 2 s
+// default); synchronizes the device first.
+cudaError_t set_wait_limit(unsigned long long ns);
 
 }  // namespace hbl

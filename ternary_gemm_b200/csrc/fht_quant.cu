@@ -442,7 +442,7 @@ cudaError_t launch_one(const void* x, int64_t M, void* out, float* scales, cudaS
                        const void* aux = nullptr) {
   using S = Shape<LOGK>;
   auto kern = ln_fht_quant_kernel<LOGK, BF16, MODE>;
-  static bool smem_set[sm100_host::kMaxDevices] = {false};
+  static std::atomic<bool> smem_set[sm100_host::kMaxDevices];
   cudaError_t e = sm100_host::ensure_smem(kern, (int)S::SMEM, smem_set);
   if (e != cudaSuccess) return e;
   const int64_t grid = (M + S::R - 1) / S::R;

@@ -58,26 +58,27 @@
 //              statistics, quantizer, codes stored straight to global memory
 //              (each warp writes whole consecutive chunk rows).
 // Row statistics reduce over the threads of a token row: warp shuffles, then
-// per-warp slots behind a named barrier of the row's warpgroup (pair), one
-// round for both statistics: sum Y^2, and sum |y| (INT4) or max |y| (INT8)
-// of the transformed but unscaled y, since t = cmul y.  INT8 then stays
-// exact: gamma = fl(cmul max|y|) = max|t| (rounding is monotone) and the
-// codes are rint(fl(cmul y) r).  INT4 takes beta = fl(cmul sum|y|) / K with
-// the sum in float (trees of depth <= 22), r a fast division, the scale
-// beta * fl(1/sqrt 7), and codes rint(y fl(cmul r)): beta within ~24 units
-// in the last place (1.5e-6) of the double sum over t, and y fl(cmul r)
-// within ~30 units of t r, so a code can differ from the quantizer-on-t
-// value only where t r is within ~1.5e-5 of a half-integer
-// (a double per-element sum and a second reduction round cost about a
-// quarter of the kernel's time).  INT4 codes widened to int8 are clipped on
-// packed 16-bit halves when the row bound ||t|| r keeps every code below
-// 2^15, else on 32-bit values.
+// per-warp slots behind a named barrier of the row's warpgroup (pair).  Round
+// 1 gives sum Y^2 (and for INT8 max |y| of the transformed but unscaled y),
+// hence cmul; every mode then forms t = fl(cmul y), the value the debug mode
+// writes out.  INT8 is exact from round 1: gamma = fl(cmul max|y|) = max|t|
+// (rounding is monotone).  INT4 needs sum |t| itself: round 2 sums |t| in
+// double (each |t| made exactly from its bits, scaled by a power of two) and
+// rounds the mean once to float, as the quantizer-only kernel does.  Both then take r = c / (stat + eps) and
+// the scale stat / c as correctly rounded divisions and the codes as
+// rint(t r) of the exact product, so the codes and scales are those of the
+// quantizer applied to t.  INT4 codes widened to int8 are clipped on packed
+// 16-bit halves when the row bound ||t|| r keeps every code below 2^15, else
+// on 32-bit values.
 // The block is launched with at most 96 registers per thread and rebalanced
-// with setmaxnreg: the first warpgroup gives its share down to 40, the
-// epilogue warpgroups take 104 each (the host checks that the launch count
-// covers this split before launching).  Every mbarrier wait is bounded (2 s,
-// then the CTA abort flag and the device error word are set and every role
-// leaves its loop).
+// with setmaxnreg: the first warpgroup gives its share down to 64, the
+// epilogue warpgroups take 104 each, which uses the launch's 640 x 96
+// registers exactly (the host checks that the launch count covers this split
+// before launching).  At 40 the producer, MMA and widening loops spilled.
+// Every mbarrier wait is bounded (by the device status's limit, 2 s unless a
+// test shortens it; then the CTA abort flag and the device error word are set
+// and every role leaves its loop), and the producer waits (bounded by 2 s)
+// for the loads it issued before the CTA exits.
 #include <cstdint>
 
 #include "common.cuh"
@@ -99,7 +100,7 @@ constexpr int kSlots = 4;                            // ring slots of two boxes 
 constexpr int kSlotBytes = 2 * kBoxBytes;
 constexpr int kEpiGroups = 4;                        // epilogue warpgroups
 constexpr int kThreads = 128 + 128 * kEpiGroups;
-constexpr int kCtrlRegs = 40;  // registers per thread of the first warpgroup after setmaxnreg
+constexpr int kCtrlRegs = 64;  // registers per thread of the first warpgroup after setmaxnreg
 constexpr int kEpiRegs = 104;  // registers per thread of an epilogue warpgroup after setmaxnreg
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kAcol = 448;  // TMEM column of A (64 columns: 128 bf16 per lane)
@@ -198,6 +199,45 @@ __device__ __forceinline__ float2 group_reduce2(float2 v, float2* slots, int wq,
   return v;
 }
 
+// The same all-reduce for one float sum.
+template <int RT>
+__device__ __forceinline__ float group_reduce1(float v, float* slots, int wq, int lane, int bar_id, int bar_n,
+                                               bool& failed) {
+  constexpr int W = RT < 32 ? RT : 32;
+#pragma unroll
+  for (int o = W / 2; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  if constexpr (RT > 32) {
+    constexpr int NW = RT / 32;
+    if (lane == 0) slots[wq] = v;
+    failed = named_bar_any(bar_id, bar_n, failed);
+    const int w0 = wq & ~(NW - 1);
+    v = slots[w0];
+#pragma unroll
+    for (int i = 1; i < NW; ++i) v += slots[w0 + i];
+  }
+  return v;
+}
+
+// The same all-reduce for one double sum (the INT4 absmean's second round).
+// Additions commute exactly, so the butterfly leaves every lane with the
+// identical value, and every thread reads the slots in the same order.
+template <int RT>
+__device__ __forceinline__ double group_reduce_d(double v, double* slots, int wq, int lane, int bar_id, int bar_n) {
+  constexpr int W = RT < 32 ? RT : 32;
+#pragma unroll
+  for (int o = W / 2; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  if constexpr (RT > 32) {
+    constexpr int NW = RT / 32;
+    if (lane == 0) slots[wq] = v;
+    named_bar_sync(bar_id, bar_n);
+    const int w0 = wq & ~(NW - 1);
+    v = slots[w0];
+#pragma unroll
+    for (int i = 1; i < NW; ++i) v += slots[w0 + i];
+  }
+  return v;
+}
+
 // Per-thread reductions over y[0..63] with 8 independent accumulators (8
 // short dependency chains) and a final tree, so they do not serialize on
 // the add latency.
@@ -214,13 +254,15 @@ __device__ __forceinline__ float sum_sq64(const float (&y)[64]) {
   return s[0];
 }
 
-// sum |y| in float (the |.| is an operand modifier of the adds)
-__device__ __forceinline__ float sum_abs64(const float (&y)[64]) {
-  float v[8];
+// sum |t| over t[0..63] in double, scaled by 2^-896 (q::abs_scaled_f64: each
+// |t| exact, no conversion instruction); eight independent accumulators keep
+// the dependency chains short
+__device__ __forceinline__ double sum_abs64_scaled(const float (&t)[64]) {
+  double v[8];
 #pragma unroll
-  for (int a = 0; a < 8; ++a) v[a] = fabsf(y[a]);
+  for (int a = 0; a < 8; ++a) v[a] = q::abs_scaled_f64(t[a]);
 #pragma unroll
-  for (int r = 8; r < 64; ++r) v[r & 7] += fabsf(y[r]);
+  for (int r = 8; r < 64; ++r) v[r & 7] += q::abs_scaled_f64(t[r]);
 #pragma unroll
   for (int w = 4; w >= 1; w >>= 1)
 #pragma unroll
@@ -350,7 +392,8 @@ ln_fht_quant_tc_kernel(const __grid_constant__ CUtensorMap tmX, TcParams p) {
   // with no barrier between one group's reduction and the next group's, a
   // fast warp writes the other set while a slow one still reads this one.
   float2* red2 = reinterpret_cast<float2*>(drain + 1);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(red2 + 32);
+  double* redd = reinterpret_cast<double*>(red2 + 32);  // the same layout for the INT4 double sums
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(redd + 32);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -397,15 +440,12 @@ ln_fht_quant_tc_kernel(const __grid_constant__ CUtensorMap tmX, TcParams p) {
       // ---------------------------------------------- TMA producer
       if (lane == 0) {
         prefetch_tensormap(&tmX);
-        bool ok = true;
-        for (int j = 0;; ++j) {
+        int j = 0;  // groups issued
+        for (;; ++j) {
           const int q = blockIdx.x + j * gridDim.x;
           if (q >= p.num_groups) break;
           const int slot = j % kSlots;
-          if (!wait_bounded(&empty[slot], ((uint32_t)(j / kSlots) & 1u) ^ 1u, abort_flag, p.err)) {
-            ok = false;
-            break;
-          }
+          if (!wait_bounded(&empty[slot], ((uint32_t)(j / kSlots) & 1u) ^ 1u, abort_flag, p.err)) break;
           mbar_expect_tx(&full[slot], (uint32_t)kSlotBytes);
           uint8_t* dst = sB + slot * kSlotBytes;
 #pragma unroll
@@ -416,12 +456,8 @@ ln_fht_quant_tc_kernel(const __grid_constant__ CUtensorMap tmX, TcParams p) {
               tma_load_2d(dst + u * kBoxBytes, &tmX, 0, (2 * q + u) * kBoxRows, &full[slot]);
           }
         }
-        if (!ok) {
-          // give the copies already issued time to land before the CTA exits
-          const uint64_t t0 = globaltimer();
-          while (globaltimer() - t0 < 20000000ull) {
-          }
-        }
+        // the copies issued have landed before the CTA may exit
+        drain_loads(full, kSlots, j, p.err);
       }
     } else if (warp == 1) {
       // ---------------------------------------------- MMA issuer
@@ -579,18 +615,22 @@ ln_fht_quant_tc_kernel(const __grid_constant__ CUtensorMap tmX, TcParams p) {
         if (m == 0 && h == 0) y[0] = 0.0f;  // t_0 = 0
       }
 
-      // Row statistics in one reduction round: K^2 var = sum_{i>=1} Y_i^2,
-      // and the quantizer's statistic of y (t = cmul y): sum |y| for INT4
-      // (sum |t| = cmul sum |y| up to the roundings of t), max |y| for INT8
-      // (max |t| = fl(cmul max |y|) exactly, rounding being monotone).
-      float stat_part = 0.0f;
-      if constexpr (MODE == K1_Q8_I8) stat_part = max_abs64(y);
-      if constexpr (MODE == K1_Q4_PACKED || MODE == K1_Q4_I8) stat_part = sum_abs64(y);
-      float2* slot2 = red2 + 16 * pr + 8 * ((j >> 1) & 1) + (PAIR ? 0 : 4 * h);
-      const float2 red = group_reduce2<RT, MODE == K1_Q8_I8>(make_float2(sum_sq64(y), stat_part), slot2, wq, lane,
-                                                              bar_row, bar_row_n, failed);
+      // Row statistics.  Round 1: K^2 var = sum_{i>=1} Y_i^2, and for INT8
+      // max |y| (max |t| = fl(cmul max |y|) exactly, rounding being
+      // monotone).  INT4 needs sum |t| over t = fl(cmul y) itself, which
+      // exists only once cmul is known: round 2 sums it in double.
+      const int rset = 16 * pr + 8 * ((j >> 1) & 1) + (PAIR ? 0 : 4 * h);
+      float ss, gmax = 0.0f;
+      if constexpr (MODE == K1_Q8_I8) {
+        const float2 red = group_reduce2<RT, true>(make_float2(sum_sq64(y), max_abs64(y)), red2 + rset, wq, lane,
+                                                   bar_row, bar_row_n, failed);
+        ss = red.x;
+        gmax = red.y;
+      } else {
+        ss = group_reduce1<RT>(sum_sq64(y), reinterpret_cast<float*>(red2) + rset, wq, lane, bar_row, bar_row_n,
+                               failed);
+      }
       if (failed) break;
-      const float ss = red.x;
       const float var = ss * (1.0f / ((float)K * (float)K));
       // 1 / sqrt(K (var + eps)): a correctly rounded reciprocal square root
       // (one rounding) times 1/sqrt(K); the debug and quantizing modes share it
@@ -598,10 +638,11 @@ ln_fht_quant_tc_kernel(const __grid_constant__ CUtensorMap tmX, TcParams p) {
       const bool row_ok = row < p.M;
       // this thread's chunk row: C = 64, unit row m; C = 128, tile row m
       const int64_t crow = (PAIR ? (int64_t)q * kBoxRows : unit0) + m;
+      // t = fl(cmul y) in place: the transform output every mode starts from
+#pragma unroll
+      for (int r = 0; r < 64; r += 2) mul2(y[r], y[r + 1], cmul);
 
       if constexpr (MODE == K1_T_F32) {
-#pragma unroll
-        for (int r = 0; r < 64; r += 2) mul2(y[r], y[r + 1], cmul);
         if (row_ok) {
           float* trow = p.t_out + (size_t)row * K;
 #pragma unroll
@@ -618,18 +659,15 @@ ln_fht_quant_tc_kernel(const __grid_constant__ CUtensorMap tmX, TcParams p) {
         }
       } else {
         q::RowParams qp;
-        float cq;  // multiplier from y to the value rounded to a code
         if constexpr (MODE == K1_Q8_I8) {
-          qp = q::params_int8(__fmul_rn(cmul, red.y));
-          // INT8 keeps the exact order: t = fl(cmul y), then rint(t r)
-#pragma unroll
-          for (int r = 0; r < 64; r += 2) mul2(y[r], y[r + 1], cmul);
-          cq = qp.r;
+          qp = q::params_int8(__fmul_rn(cmul, gmax));
         } else {
-          // INT4: beta from cmul sum|y| (float), codes rint(y * fl(cmul r))
-          qp = q::params_int4_f32(__fmul_rn(cmul, red.y), K);
-          cq = __fmul_rn(cmul, qp.r);
+          // round 2: beta = (float)(sum |t| / K) from a double sum, as the
+          // quantizer-only kernel computes it
+          const double sa = group_reduce_d<RT>(sum_abs64_scaled(y), redd + rset, wq, lane, bar_row, bar_row_n);
+          qp = q::params_int4(sa * q::kUnscaleAbs, K);
         }
+        const float cq = qp.r;  // codes are rint(t r)
         if (row_ok && i_hi == 0 && (!PAIR || h == 0)) p.scales[row] = qp.scale;
         if (row_ok) {
           uint8_t* crow_out = p.codes + crow * (MODE == K1_Q4_PACKED ? C / 2 : C);
@@ -643,7 +681,10 @@ ln_fht_quant_tc_kernel(const __grid_constant__ CUtensorMap tmX, TcParams p) {
           } else {
             // 16 codes per 16 bytes: C = 64 at 0, 16, 32, 48; C = 128 at
             // 32h, 32h + 16, 64 + 32h, 80 + 32h
-            const bool s16 = MODE == K1_Q4_I8 && ss * cq * cq < 9.0e8f;
+            // ||t||^2 = cmul^2 ss (up to the roundings of t), so every
+            // |t r| < 3e4 when cmul^2 r^2 ss < 9e8
+            const float cr = cmul * cq;
+            const bool s16 = MODE == K1_Q4_I8 && ss * cr * cr < 9.0e8f;
             if (PAIR && p.codes_al32) {
               // two whole 32-byte sectors per thread, not four half sectors
 #pragma unroll
@@ -754,7 +795,8 @@ ln_fht_quant_tc256_kernel(const __grid_constant__ CUtensorMap tmX, TcParams p) {
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
   float2* red2 = reinterpret_cast<float2*>(drain + 1);  // [tile parity][16 warps]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(red2 + 32);
+  double* redd = reinterpret_cast<double*>(red2 + 32);  // the same for the INT4 double sums
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(redd + 32);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -790,25 +832,18 @@ ln_fht_quant_tc256_kernel(const __grid_constant__ CUtensorMap tmX, TcParams p) {
     if (warp == 0) {
       if (lane == 0) {
         prefetch_tensormap(&tmX);
-        bool ok = true;
-        for (int j = 0;; ++j) {
+        int j = 0;  // tiles issued
+        for (;; ++j) {
           const int q = blockIdx.x + j * gridDim.x;
           if (q >= p.num_groups) break;
           const int slot = j % k256Slots;
-          if (!wait_bounded(&empty[slot], ((uint32_t)(j / k256Slots) & 1u) ^ 1u, abort_flag, p.err)) {
-            ok = false;
-            break;
-          }
+          if (!wait_bounded(&empty[slot], ((uint32_t)(j / k256Slots) & 1u) ^ 1u, abort_flag, p.err)) break;
           mbar_expect_tx(&full[slot], (uint32_t)k256TileBytes);
 #pragma unroll
           for (int u = 0; u < 4; ++u)
             tma_load_2d(sB + slot * k256TileBytes + u * kBoxBytes, &tmX, kBoxCols * u, q * kBoxRows, &full[slot]);
         }
-        if (!ok) {
-          const uint64_t t0 = globaltimer();
-          while (globaltimer() - t0 < 20000000ull) {
-          }
-        }
+        drain_loads(full, k256Slots, j, p.err);
       }
     } else if (warp == 1) {
       if (lane == 0) {
@@ -915,22 +950,27 @@ ln_fht_quant_tc256_kernel(const __grid_constant__ CUtensorMap tmX, TcParams p) {
       // now y[r] = column 32 g + r, y[32 + r] = column 128 + 32 g + r
       if (m == 0 && g == 0) y[0] = 0.0f;  // t_0 = 0
 
-      float stat_part = 0.0f;
-      if constexpr (MODE == K1_Q8_I8) stat_part = max_abs64(y);
-      if constexpr (MODE == K1_Q4_PACKED || MODE == K1_Q4_I8) stat_part = sum_abs64(y);
-      float2* slot2 = red2 + 16 * (j & 1);
-      const float2 red = group_reduce2<512, MODE == K1_Q8_I8>(make_float2(sum_sq64(y), stat_part), slot2, wq, lane,
-                                                               bar_row, 512, failed);
+      // the two statistic rounds of ln_fht_quant_tc_kernel, over all 512
+      // epilogue threads
+      const int rset = 16 * (j & 1);
+      float ss, gmax = 0.0f;
+      if constexpr (MODE == K1_Q8_I8) {
+        const float2 red = group_reduce2<512, true>(make_float2(sum_sq64(y), max_abs64(y)), red2 + rset, wq, lane,
+                                                    bar_row, 512, failed);
+        ss = red.x;
+        gmax = red.y;
+      } else {
+        ss = group_reduce1<512>(sum_sq64(y), reinterpret_cast<float*>(red2) + rset, wq, lane, bar_row, 512, failed);
+      }
       if (failed) break;
-      const float ss = red.x;
       const float var = ss * (1.0f / ((float)K * (float)K));
       const float cmul = __fmul_rn(__frsqrt_rn(__fadd_rn(var, 1e-5f)), p.sK);
       const int64_t row = q;
       const int64_t crow = (int64_t)q * kBoxRows + m;
+#pragma unroll
+      for (int r = 0; r < 64; r += 2) mul2(y[r], y[r + 1], cmul);  // t = fl(cmul y)
 
       if constexpr (MODE == K1_T_F32) {
-#pragma unroll
-        for (int r = 0; r < 64; r += 2) mul2(y[r], y[r + 1], cmul);
         float* trow = p.t_out + (size_t)row * K + (size_t)m * k256Cols;
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
@@ -943,16 +983,13 @@ ln_fht_quant_tc256_kernel(const __grid_constant__ CUtensorMap tmX, TcParams p) {
         }
       } else {
         q::RowParams qp;
-        float cq;
-        if constexpr (MODE == K1_Q8_I8) {
-          qp = q::params_int8(__fmul_rn(cmul, red.y));
-#pragma unroll
-          for (int r = 0; r < 64; r += 2) mul2(y[r], y[r + 1], cmul);
-          cq = qp.r;
-        } else {
-          qp = q::params_int4_f32(__fmul_rn(cmul, red.y), K);
-          cq = __fmul_rn(cmul, qp.r);
-        }
+        if constexpr (MODE == K1_Q8_I8)
+          qp = q::params_int8(__fmul_rn(cmul, gmax));
+        else
+          qp = q::params_int4(group_reduce_d<512>(sum_abs64_scaled(y), redd + rset, wq, lane, bar_row, 512) *
+                                  q::kUnscaleAbs,
+                              K);
+        const float cq = qp.r;
         if (m == 0 && g == 0) p.scales[row] = qp.scale;
         uint8_t* crow_out = p.codes + crow * (MODE == K1_Q4_PACKED ? k256Cols / 2 : k256Cols);
         if constexpr (MODE == K1_Q4_PACKED) {
@@ -960,7 +997,8 @@ ln_fht_quant_tc256_kernel(const __grid_constant__ CUtensorMap tmX, TcParams p) {
           *reinterpret_cast<uint4*>(crow_out + 16 * g) = codes32_s4(&y[0], cq);
           *reinterpret_cast<uint4*>(crow_out + 64 + 16 * g) = codes32_s4(&y[32], cq);
         } else {
-          const bool s16 = MODE == K1_Q4_I8 && ss * cq * cq < 9.0e8f;
+          const float cr = cmul * cq;
+          const bool s16 = MODE == K1_Q4_I8 && ss * cr * cr < 9.0e8f;
 #pragma unroll
           for (int half = 0; half < 2; ++half) {
             const uint4 v0 = s16 ? codes16_i8<MODE, true>(&y[32 * half], cq) : codes16_i8<MODE>(&y[32 * half], cq);
@@ -1026,7 +1064,7 @@ cudaError_t launch_tc(const void* x, int64_t M, void* out, float* scales, int* e
     return (int64_t)fa.numRegs * kThreads >= (int64_t)128 * kCtrlRegs + (int64_t)128 * kEpiGroups * kEpiRegs;
   }();
   if (!split_ok) return cudaErrorInvalidConfiguration;
-  static bool smem_set[sm100_host::kMaxDevices] = {false};
+  static std::atomic<bool> smem_set[sm100_host::kMaxDevices];
   cudaError_t e = sm100_host::ensure_smem(kern, (int)kSmemBytes, smem_set);
   if (e != cudaSuccess) return e;
   const int nsm = sm100_host::sm_count();
@@ -1063,7 +1101,7 @@ cudaError_t launch_tc256(const void* x, int64_t M, void* out, float* scales, int
     return (int64_t)fa.numRegs * kThreads >= (int64_t)128 * kCtrlRegs + (int64_t)128 * kEpiGroups * kEpiRegs;
   }();
   if (!split_ok) return cudaErrorInvalidConfiguration;
-  static bool smem_set[sm100_host::kMaxDevices] = {false};
+  static std::atomic<bool> smem_set[sm100_host::kMaxDevices];
   cudaError_t e = sm100_host::ensure_smem(kern, (int)k256SmemBytes, smem_set);
   if (e != cudaSuccess) return e;
   const int nsm = sm100_host::sm_count();

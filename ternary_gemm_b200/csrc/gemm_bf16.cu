@@ -139,6 +139,7 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
+      int issued = 0;
       for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x) {
         int r_blk, c_blk;
         tile_coords(p, tile, r_blk, c_blk);
@@ -155,14 +156,12 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
           }
 #pragma unroll
           for (int j = 0; j < 4; ++j) tma_load_2d(b + j * kAtomBytes, &tmB, c_blk * kBN + 64 * j, kb * kBKe, &full[stage]);
+          ++issued;
           if (++stage == kStages) { stage = 0; phase ^= 1u; }
         }
       }
-      if (!ok) {
-        const uint64_t t0 = globaltimer();
-        while (globaltimer() - t0 < 20000000ull) {
-        }
-      }
+      // the copies issued have landed before the CTA may exit
+      drain_loads(full, kStages, issued, p.err);
     }
   } else if (warp == 1) {
     // ------------------------------------------------ MMA issuer
@@ -291,13 +290,16 @@ gemm_bf16_2sm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
   uint64_t* exitb = drain + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(exitb + 1);
+  uint64_t* drainb = exitb + 1;
+  int* peer_issued = reinterpret_cast<int*>(drainb + 1);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(peer_issued + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
   const bool leader = rank == 0;
+  int issued = 0;  // stages this CTA's producer (thread 0) loaded
   const int cid = blockIdx.x >> 1;
   const int ncl = gridDim.x >> 1;
 
@@ -312,6 +314,8 @@ gemm_bf16_2sm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
     }
     mbar_init(drain, 1);
     mbar_init(exitb, 1);
+    mbar_init(drainb, 1);
+    *peer_issued = 0;
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -355,14 +359,11 @@ gemm_bf16_2sm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
           }
           tma_load_2d_pair(b, &tmB, c0, kb * kBKe, fbar);
           tma_load_2d_pair(b + kAtomBytes, &tmB, c0 + 64, kb * kBKe, fbar);
+          ++issued;
           if (++stage == k2Stages) { stage = 0; phase ^= 1u; }
         }
       }
-      if (!ok) {
-        const uint64_t t0 = globaltimer();
-        while (globaltimer() - t0 < 20000000ull) {
-        }
-      }
+      // the loads are drained at the pair's exit (pair_exit_drain)
     }
   } else if (warp == 1) {
     if (lane == 0 && leader) {
@@ -444,19 +445,13 @@ gemm_bf16_2sm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
   }
 
   // neither CTA frees its shared memory or TMEM while the pair still uses
-  // them: a bounded handshake through each other's exit barrier
+  // them, nor exits with loads into its shared memory in flight (the exit
+  // handshake and the leader's drain of the stage ring, pair_exit_drain;
+  // thread 0 is each CTA's producer)
   fence_before();
   __syncthreads();
-  if (threadIdx.x == 0) {
-    mbar_arrive_cluster(mapa_shared(smem_u32(exitb), rank ^ 1u));
-    const uint64_t t0 = globaltimer();
-    while (!mbar_try_wait(exitb, 0)) {
-      if (globaltimer() - t0 > kWaitLimitNs) {
-        atomicExch(p.err, 1);
-        break;
-      }
-    }
-  }
+  if (threadIdx.x == 0)
+    pair_exit_drain(leader, rank, full, k2Stages, (uint32_t)k2StageBytes, issued, peer_issued, exitb, drainb, p.err);
   __syncthreads();
   fence_after();
   if (warp == 1) {
@@ -501,24 +496,24 @@ cudaError_t launch_gemm_bf16(const uint16_t* A, bool a_mn, const uint16_t* B, in
     const int pairs = nsm / 2;
     const unsigned grid2 = 2u * (unsigned)(p.num_tiles < pairs ? p.num_tiles : pairs);
     if (a_mn) {
-      static bool set2[sm100_host::kMaxDevices] = {false};
+      static std::atomic<bool> set2[sm100_host::kMaxDevices];
       cudaError_t e = sm100_host::ensure_smem(gemm_bf16_2sm_kernel<true>, (int)k2SmemBytes, set2);
       if (e != cudaSuccess) return e;
       return sm100_host::launch_pdl(gemm_bf16_2sm_kernel<true>, grid2, kThreads, k2SmemBytes, stream, 2, ta, tb, p);
     }
-    static bool set2[sm100_host::kMaxDevices] = {false};
+    static std::atomic<bool> set2[sm100_host::kMaxDevices];
     cudaError_t e = sm100_host::ensure_smem(gemm_bf16_2sm_kernel<false>, (int)k2SmemBytes, set2);
     if (e != cudaSuccess) return e;
     return sm100_host::launch_pdl(gemm_bf16_2sm_kernel<false>, grid2, kThreads, k2SmemBytes, stream, 2, ta, tb, p);
   }
   const int grid = p.num_tiles < nsm ? p.num_tiles : nsm;
   if (a_mn) {
-    static bool set[sm100_host::kMaxDevices] = {false};
+    static std::atomic<bool> set[sm100_host::kMaxDevices];
     cudaError_t e = sm100_host::ensure_smem(gemm_bf16_kernel<true>, (int)kSmemBytes, set);
     if (e != cudaSuccess) return e;
     return sm100_host::launch_pdl(gemm_bf16_kernel<true>, (unsigned)grid, kThreads, kSmemBytes, stream, 1, ta, tb, p);
   }
-  static bool set[sm100_host::kMaxDevices] = {false};
+  static std::atomic<bool> set[sm100_host::kMaxDevices];
   cudaError_t e = sm100_host::ensure_smem(gemm_bf16_kernel<false>, (int)kSmemBytes, set);
   if (e != cudaSuccess) return e;
   return sm100_host::launch_pdl(gemm_bf16_kernel<false>, (unsigned)grid, kThreads, kSmemBytes, stream, 1, ta, tb, p);

@@ -45,7 +45,7 @@
 
 namespace hbl {
 
-__device__ int g_device_error = 0;
+__device__ sm100::DeviceStatus g_status = {0, 0, sm100::kWaitLimitNs};
 
 namespace {
 
@@ -92,7 +92,7 @@ __device__ __forceinline__ void tile_mn(const Params& p, int tile, int& m_blk, i
 }
 
 __device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
-  return sm100::wait_bounded(bar, parity, abort_flag, &g_device_error);
+  return sm100::wait_bounded(bar, parity, abort_flag, &g_status.error);
 }
 
 __device__ __forceinline__ uint64_t sdesc(uint32_t saddr) { return sm100::sdesc_k_sw128(saddr); }
@@ -167,6 +167,7 @@ gemm_i8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
+      int issued = 0;
       for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x) {
         int m_blk, n_blk;
         tile_mn(p, tile, m_blk, n_blk);
@@ -175,15 +176,12 @@ gemm_i8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           mbar_expect_tx(&full[stage], (uint32_t)kStageBytes);
           tma_load_2d(sA + stage * kABytes, &tmA, kb * kBK, m_blk * kBM, &full[stage]);
           tma_load_2d(sB + stage * kBBytes, &tmB, kb * kBK, n_blk * kBN, &full[stage]);
+          ++issued;
           if (++stage == kStages) { stage = 0; phase ^= 1u; }
         }
       }
-      if (!ok) {
-        // give the copies already issued time to land before the CTA exits
-        const uint64_t t0 = globaltimer();
-        while (globaltimer() - t0 < 20000000ull) {
-        }
-      }
+      // the copies issued have landed before the CTA may exit
+      drain_loads(full, kStages, issued, &g_status.error);
     }
   } else if (warp == 1) {
     // ------------------------------------------------ MMA issuer
@@ -381,7 +379,9 @@ gemm_i8_2sm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
   uint64_t* exitb = drain + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(exitb + 1);
+  uint64_t* drainb = exitb + 1;
+  int* peer_issued = reinterpret_cast<int*>(drainb + 1);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(peer_issued + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -390,6 +390,7 @@ gemm_i8_2sm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
   const bool leader = rank == 0;
   const int cid = blockIdx.x >> 1;
   const int ncl = gridDim.x >> 1;
+  int issued = 0;  // stages this CTA's producer (thread 0) loaded
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < k2Stages; ++s) {
@@ -402,6 +403,8 @@ gemm_i8_2sm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
     }
     mbar_init(drain, 1);
     mbar_init(exitb, 1);
+    mbar_init(drainb, 1);
+    *peer_issued = 0;
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -435,14 +438,11 @@ gemm_i8_2sm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
           if (leader) mbar_expect_tx(&full[stage], (uint32_t)(2 * k2StageBytes));
           tma_load_2d_pair(sA + stage * k2ABytes, &tmA, kb * kBK, m_blk * 256 + (int)rank * 128, fbar);
           tma_load_2d_pair(sB + stage * k2BBytes, &tmB, kb * kBK, n_blk * 256 + (int)rank * 128, fbar);
+          ++issued;
           if (++stage == k2Stages) { stage = 0; phase ^= 1u; }
         }
       }
-      if (!ok) {
-        const uint64_t t0 = globaltimer();
-        while (globaltimer() - t0 < 20000000ull) {
-        }
-      }
+      // the loads are drained at the pair's exit (pair_exit_drain)
     }
   } else if (warp == 1) {
     if (lane == 0 && leader) {
@@ -504,19 +504,14 @@ gemm_i8_2sm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
   }
 
   // neither CTA may free its shared memory or TMEM while the pair still uses
-  // them: a bounded handshake through each other's exit barrier
+  // them, nor exit with loads into its shared memory in flight: a bounded
+  // handshake through each other's exit barrier, then the leader drains the
+  // stage ring for both (thread 0 is each CTA's producer)
   fence_before();
   __syncthreads();
-  if (threadIdx.x == 0) {
-    mbar_arrive_cluster(mapa_shared(smem_u32(exitb), rank ^ 1u));
-    const uint64_t t0 = globaltimer();
-    while (!mbar_try_wait(exitb, 0)) {
-      if (globaltimer() - t0 > kWaitLimitNs) {
-        atomicExch(&g_device_error, 1);
-        break;
-      }
-    }
-  }
+  if (threadIdx.x == 0)
+    pair_exit_drain(leader, rank, full, k2Stages, (uint32_t)k2StageBytes, issued, peer_issued, exitb, drainb,
+                    &g_status.error);
   __syncthreads();
   fence_after();
   if (warp == 1) {
@@ -631,19 +626,17 @@ gemm_i8_splitk_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
       prefetch_tensormap(&tmB);
       int stage = 0;
       uint32_t phase = 0;
-      bool ok = true;
+      int issued = 0;
       for (int kb = kb0; kb < kb1; ++kb) {
-        if (!wait_bounded(&empty[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
+        if (!wait_bounded(&empty[stage], phase ^ 1u, abort_flag)) break;
         mbar_expect_tx(&full[stage], (uint32_t)kStageBytes);
         tma_load_2d(sA + stage * kABytes, &tmA, kb * kBK, m_blk * kBM, &full[stage]);
         tma_load_2d(sB + stage * kBBytes, &tmB, kb * kBK, n_blk * kBN, &full[stage]);
+        ++issued;
         if (++stage == kStages) { stage = 0; phase ^= 1u; }
       }
-      if (!ok) {
-        const uint64_t t0 = globaltimer();
-        while (globaltimer() - t0 < 20000000ull) {
-        }
-      }
+      // the loads have landed before the stage ring holds the partials
+      drain_loads(full, kStages, issued, &g_status.error);
     }
     __syncwarp();
     cluster_phase();  // partials written
@@ -795,10 +788,11 @@ constexpr int kSplitMaxRows16 = 255;  // int16 partials: every short batch
 // per device and cluster size; 0 when the query fails)
 template <typename Kernel>
 int max_active_clusters(Kernel kern, int split, int idx) {
-  static int cache[6][sm100_host::kMaxDevices] = {};
+  static std::atomic<int> cache[6][sm100_host::kMaxDevices];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= sm100_host::kMaxDevices) return 0;
-  if (cache[idx][dev] > 0) return cache[idx][dev];
+  const int c = cache[idx][dev].load(std::memory_order_acquire);
+  if (c > 0) return c;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)split, 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
@@ -815,7 +809,7 @@ int max_active_clusters(Kernel kern, int split, int idx) {
     (void)cudaGetLastError();
     return 0;
   }
-  cache[idx][dev] = n;
+  cache[idx][dev].store(n, std::memory_order_release);
   return n;
 }
 
@@ -852,7 +846,7 @@ cudaError_t launch_gemm_i8(const int8_t* A, const int8_t* B, int64_t M, int64_t 
     const int64_t panel = (int64_t)256 * K;
     const int64_t groups = (p.num_n * panel + (int64_t(40) << 20) - 1) / (int64_t(40) << 20);
     p.group_n = groups > 1 ? (int)((p.num_n + groups - 1) / groups) : 0;
-    static bool smem_set2[sm100_host::kMaxDevices] = {false};
+    static std::atomic<bool> smem_set2[sm100_host::kMaxDevices];
     cudaError_t e = sm100_host::ensure_smem(gemm_i8_2sm_kernel, (int)k2SmemBytes, smem_set2);
     if (e != cudaSuccess) return e;
     const int pairs = sm_count() / 2;
@@ -876,14 +870,14 @@ cudaError_t launch_gemm_i8(const int8_t* A, const int8_t* B, int64_t M, int64_t 
                     : (split == 2 ? gemm_i8_splitk_kernel<2, false>
                        : split == 4 ? gemm_i8_splitk_kernel<4, false> : gemm_i8_splitk_kernel<8, false>);
     const int idx = (split == 2 ? 0 : split == 4 ? 1 : 2) + (p16 ? 3 : 0);
-    static bool smem_set_s[6][sm100_host::kMaxDevices] = {};
+    static std::atomic<bool> smem_set_s[6][sm100_host::kMaxDevices];
     cudaError_t e = sm100_host::ensure_smem(kern, (int)kSmemBytes, smem_set_s[idx]);
     if (e != cudaSuccess) return e;
     if (p.num_tiles > max_active_clusters(kern, split, idx)) continue;
     return sm100_host::launch_pdl(kern, (unsigned)(p.num_tiles * split), kThreads, kSmemBytes, stream,
                                   (unsigned)split, ta, tb, p);
   }
-  static bool smem_set[sm100_host::kMaxDevices] = {false};
+  static std::atomic<bool> smem_set[sm100_host::kMaxDevices];
   cudaError_t e = sm100_host::ensure_smem(gemm_i8_kernel, (int)kSmemBytes, smem_set);
   if (e != cudaSuccess) return e;
   const int grid = p.num_tiles < nsm ? p.num_tiles : nsm;
@@ -893,28 +887,38 @@ cudaError_t launch_gemm_i8(const int8_t* A, const int8_t* B, int64_t M, int64_t 
 int* device_error_word() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  static int* cache[64] = {nullptr};
-  if (!cache[dev]) {
+  static std::atomic<int*> cache[64];
+  int* c = cache[dev].load(std::memory_order_acquire);
+  if (!c) {
     void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return nullptr;
-    cache[dev] = reinterpret_cast<int*>(p);
+    if (cudaGetSymbolAddress(&p, g_status) != cudaSuccess) return nullptr;
+    c = &reinterpret_cast<sm100::DeviceStatus*>(p)->error;
+    cache[dev].store(c, std::memory_order_release);
   }
-  return cache[dev];
+  return c;
 }
 
 cudaError_t read_and_clear_device_error(cudaStream_t stream, int* value) {
   cudaError_t e = cudaStreamSynchronize(stream);
   if (e != cudaSuccess) return e;
   int v = 0, zero = 0;
-  e = cudaMemcpyFromSymbol(&v, g_device_error, sizeof(int));
+  e = cudaMemcpyFromSymbol(&v, g_status, sizeof(int), offsetof(sm100::DeviceStatus, error));
   if (e != cudaSuccess) return e;
-  e = cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int));
+  e = cudaMemcpyToSymbol(g_status, &zero, sizeof(int), offsetof(sm100::DeviceStatus, error));
   *value = v;
   return e;
 }
 
+cudaError_t set_wait_limit(unsigned long long ns) {
+  // no kernel of the device may be running while the limit changes
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return e;
+  const unsigned long long v = ns ? ns : sm100::kWaitLimitNs;
+  return cudaMemcpyToSymbol(g_status, &v, sizeof(v), offsetof(sm100::DeviceStatus, wait_limit_ns));
+}
+
 namespace {
-__global__ void raise_error_kernel() { atomicExch(&g_device_error, 1); }
+__global__ void raise_error_kernel() { atomicExch(&g_status.error, 1); }
 }  // namespace
 
 cudaError_t raise_device_error(cudaStream_t stream) {

@@ -124,7 +124,7 @@ gemv_ternary_kernel(const int8_t* __restrict__ A, const float* __restrict__ scal
 template <int MT>
 cudaError_t launch_mt(const int8_t* A, const float* scales, const uint8_t* packed, const float* alpha, void* y,
                       int y_mode, int M, int N, int K, cudaStream_t stream) {
-  static bool smem_set1[sm100_host::kMaxDevices] = {false}, smem_set2[sm100_host::kMaxDevices] = {false};
+  static std::atomic<bool> smem_set1[sm100_host::kMaxDevices], smem_set2[sm100_host::kMaxDevices];
   cudaError_t e = y_mode == 2
                       ? sm100_host::ensure_smem(gemv_ternary_kernel<MT, 2>, (int)kGemvMaxCodeBytes, smem_set2)
                       : sm100_host::ensure_smem(gemv_ternary_kernel<MT, 1>, (int)kGemvMaxCodeBytes, smem_set1);

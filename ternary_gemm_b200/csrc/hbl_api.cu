@@ -443,6 +443,8 @@ hbl_status hbl_debug_raise_device_error(cudaStream_t stream) {
   return cuda_status(hbl::raise_device_error(stream));
 }
 
+hbl_status hbl_debug_set_wait_limit_ns(uint64_t ns) { return cuda_status(hbl::set_wait_limit(ns)); }
+
 const char* hbl_status_string(hbl_status status) {
   switch (status) {
     case HBL_OK: return "HBL_OK";

@@ -1,5 +1,5 @@
-// Per-token activation quantizer shared by the fused LN+FHT+quant kernel and
-// the quantizer-only kernel, so both make bit-identical decisions.
+// Per-token activation quantizer shared by the fused LN+FHT+quant kernels and
+// the quantizer-only kernel, so all of them make bit-identical decisions.
 //
 // "BitNet v2: Native 4-bit Activations with Hadamard Transformation for 1-bit
 // LLMs", section "H-BitLinear", activation-quantization formula:
@@ -29,6 +29,21 @@ constexpr int kMagicBits = 0x4B400000;
 // takes as an operand modifier.
 __device__ __forceinline__ double abs_f64(float t) { return fabs((double)t); }
 
+// |t| * 2^-896 as a double, built from the float's bits with integer shifts
+// instead of a conversion (whose pipe is narrow): the float's exponent and
+// mantissa fields, shifted right by 3, are a double's fields of the same
+// value scaled by 2^(127 - 1023).  Exact for every finite float: a normal
+// float gives a normal double, a subnormal float a subnormal double with the
+// same scaling, zero gives zero.  Sums of these values round exactly as sums
+// of |t| would (every partial sum below 2^-1022 is exact either way), so
+// multiplying the sum by kUnscaleAbs (a power of two) gives the double sum of
+// |t| itself.
+__device__ __forceinline__ double abs_scaled_f64(float t) {
+  const uint32_t b = __float_as_uint(t);
+  return __hiloint2double((int)((b & 0x7FFFFFFFu) >> 3), (int)(b << 29));
+}
+constexpr double kUnscaleAbs = 0x1p896;
+
 struct RowParams {
   float r;      // multiplier applied to t before rounding
   float scale;  // dequantisation factor of the row
@@ -40,21 +55,6 @@ __device__ __forceinline__ RowParams params_int4(double abs_sum, int64_t K) {
   RowParams p;
   p.r = __fdiv_rn(kSqrt7, __fadd_rn(beta, kEps));
   p.scale = __fdiv_rn(beta, kSqrt7);
-  return p;
-}
-
-// beta from a float sum of |t| over K elements (K a power of two, so the
-// division is exact).  Used by the fused tensor-core kernel, whose sum is a
-// float tree (relative error at most ~24 float units in the last place);
-// the quantizer-only kernel keeps the double sum above.  With that tolerance
-// the row's divisions need not be correctly rounded: r is one fast division
-// (within 2 ulp) and the scale a product with fl(1/sqrt(7)) (within 1.5 ulp).
-constexpr float kInvSqrt7 = 0.37796447300922722f;  // 1/sqrt(7) rounded to float
-__device__ __forceinline__ RowParams params_int4_f32(float abs_sum, int64_t K) {
-  const float beta = abs_sum * (1.0f / (float)K);
-  RowParams p;
-  p.r = __fdividef(kSqrt7, __fadd_rn(beta, kEps));
-  p.scale = __fmul_rn(beta, kInvSqrt7);
   return p;
 }
 

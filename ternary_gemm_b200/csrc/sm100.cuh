@@ -5,6 +5,7 @@
 // loads anywhere.
 #pragma once
 
+#include <atomic>
 #include <cstdint>
 
 #include <cuda.h>
@@ -14,7 +15,18 @@
 namespace hbl {
 namespace sm100 {
 
-constexpr uint64_t kWaitLimitNs = 2000000000ull;  // bounded waits give up after 2 s
+constexpr uint64_t kWaitLimitNs = 2000000000ull;   // default limit of the pipeline waits (2 s)
+constexpr uint64_t kDrainLimitNs = 2000000000ull;  // limit of the exit-path drains (never shortened)
+
+// The library's device status, one per device: the error flag that a bounded
+// wait sets when it gives up, and the limit of the pipeline waits (kernels
+// receive the address of `error`).  The limit is kWaitLimitNs unless a test
+// shortens it through the host API to make a wait run out.
+struct DeviceStatus {
+  int error;
+  int reserved;
+  unsigned long long wait_limit_ns;
+};
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
 
@@ -52,22 +64,49 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Bounded wait for the phase with the given parity.  Returns false if the
-// CTA already aborted or the limit ran out; then the CTA abort flag and the
-// device error word are set.
+// CTA already aborted or the limit (the device status's wait_limit_ns) ran
+// out; then the CTA abort flag and the device error word are set.  `err`
+// points at DeviceStatus::error.
 __device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int* err) {
   if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t limit = reinterpret_cast<const volatile DeviceStatus*>(err)->wait_limit_ns;
   const uint64_t t0 = globaltimer();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((i & 63u) == 0) {
       if (*abort_flag) return false;
-      if (globaltimer() - t0 > kWaitLimitNs) {
+      if (globaltimer() - t0 > limit) {
         *abort_flag = 1;
         atomicExch(err, 1);
         return false;
       }
     }
   }
+}
+
+// Exit-path wait for a phase that copies or commits already issued will
+// complete, bounded by kDrainLimitNs whatever the pipeline limit is, so that
+// a CTA that gave up still lets its copies land before it exits.
+__device__ __forceinline__ bool drain_wait(uint64_t* bar, uint32_t parity, int* err) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer() - t0 > kDrainLimitNs) {
+      atomicExch(err, 1);
+      return false;
+    }
+  }
+  return true;
+}
+
+// A producer's exit drain: issue i of a ring of `stages` stages used stage
+// i % stages in phase i / stages; the loads of the last min(issued, stages)
+// issues are waited for (every earlier phase was consumed before a later
+// issue reused its stage).  On the normal path these phases are complete or
+// about to be, so the drain costs at most the last loads' latency.
+__device__ __forceinline__ void drain_loads(uint64_t* full, int stages, int issued, int* err) {
+  for (int i = issued > stages ? issued - stages : 0; i < issued; ++i)
+    drain_wait(&full[i % stages], (uint32_t)(i / stages) & 1u, err);
 }
 
 // ---------------------------------------------------------------- named barriers
@@ -201,6 +240,81 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
+// try_wait with cluster-scope acquire: writes that another CTA of the cluster
+// made before its release-arrive on this barrier are visible afterwards
+__device__ __forceinline__ bool mbar_try_wait_acq_cluster(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// complete-tx of `bytes` on a local barrier without a copy: stands in for
+// bytes a copy that was never issued would have delivered
+__device__ __forceinline__ void mbar_complete_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.complete_tx.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ void st_shared_cluster_u32(uint32_t cluster_addr, uint32_t v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
+}
+
+// Exit of a CTA pair (cta_group::2 kernels), run by thread 0 of each CTA after
+// every role has left its loop.  Both CTAs' loads complete on the leader's
+// `full` barriers (the leader arms each phase with both CTAs' bytes), so the
+// leader drains for both, after learning how many stages the peer issued:
+//   * a phase both issued: wait for it;
+//   * a phase the leader armed that the peer never loaded: complete the
+//     peer's bytes by hand, then wait for the leader's own;
+//   * a phase the peer loaded that the leader never armed: arm it for the
+//     peer's bytes (arrive + expect-tx), then wait.
+// Each CTA issues at most `stages` stages beyond the other (a stage is reused
+// only after the MMA consumed it, which needed both halves), so the last
+// `stages` issues of the further one cover every phase that can be open.
+// The peer leaves only when the leader reports the drain done, so neither
+// CTA frees its shared memory while a copy into it is in flight.  Every wait
+// is bounded by kDrainLimitNs.
+__device__ __forceinline__ void pair_exit_drain(bool leader, uint32_t rank, uint64_t* full, int stages,
+                                                uint32_t peer_stage_bytes, int issued, int* peer_issued,
+                                                uint64_t* exitb, uint64_t* drainb, int* err) {
+  if (!leader) st_shared_cluster_u32(mapa_shared(smem_u32(peer_issued), 0), (uint32_t)issued);
+  mbar_arrive_cluster(mapa_shared(smem_u32(exitb), rank ^ 1u));
+  bool met = true;
+  const uint64_t t0 = globaltimer();
+  while (!mbar_try_wait_acq_cluster(exitb, 0)) {
+    if (globaltimer() - t0 > kDrainLimitNs) {
+      atomicExch(err, 1);
+      met = false;
+      break;
+    }
+  }
+  if (leader) {
+    const int ip = met ? *reinterpret_cast<volatile int*>(peer_issued) : issued;
+    const int last = issued > ip ? issued : ip;
+    for (int i = last > stages ? last - stages : 0; i < last; ++i) {
+      uint64_t* bar = &full[i % stages];
+      const bool armed = i < issued, loaded = i < ip;
+      if (armed && !loaded) mbar_complete_tx(bar, peer_stage_bytes);
+      if (!armed && loaded) mbar_expect_tx(bar, peer_stage_bytes);
+      drain_wait(bar, (uint32_t)(i / stages) & 1u, err);
+    }
+    mbar_arrive_cluster(mapa_shared(smem_u32(drainb), 1));
+  } else if (met) {
+    const uint64_t t1 = globaltimer();
+    while (!mbar_try_wait_acq_cluster(drainb, 0)) {
+      if (globaltimer() - t1 > kDrainLimitNs) {
+        atomicExch(err, 1);
+        break;
+      }
+    }
+  }
+}
+
 __device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* map, int x, int y, uint32_t leader_bar) {
   asm volatile(
       "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
@@ -287,27 +401,33 @@ inline bool encode_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* p
 
 constexpr int kMaxDevices = 64;
 
+// The per-device caches below are arrays of atomics: several host threads
+// may make their first calls at once, and each stores the same value.
+
 // SM count of the current device, queried once per device.
 inline int sm_count() {
-  static int cache[kMaxDevices] = {0};
+  static std::atomic<int> cache[kMaxDevices];
   int dev = 0, n = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 148;
-  if (dev >= 0 && dev < kMaxDevices && cache[dev] > 0) return cache[dev];
+  if (dev >= 0 && dev < kMaxDevices) {
+    const int c = cache[dev].load(std::memory_order_acquire);
+    if (c > 0) return c;
+  }
   if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
-  if (dev >= 0 && dev < kMaxDevices) cache[dev] = n;
+  if (dev >= 0 && dev < kMaxDevices) cache[dev].store(n, std::memory_order_release);
   return n;
 }
 
 // Dynamic shared memory limit of a kernel, set once per device: `done` is the
 // call site's own per-device flag array (one per kernel instantiation).
 template <typename Kernel>
-inline cudaError_t ensure_smem(Kernel kern, int bytes, bool (&done)[kMaxDevices]) {
+inline cudaError_t ensure_smem(Kernel kern, int bytes, std::atomic<bool> (&done)[kMaxDevices]) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (dev >= 0 && dev < kMaxDevices && done[dev]) return cudaSuccess;
+  if (dev >= 0 && dev < kMaxDevices && done[dev].load(std::memory_order_acquire)) return cudaSuccess;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-  if (e == cudaSuccess && dev >= 0 && dev < kMaxDevices) done[dev] = true;
+  if (e == cudaSuccess && dev >= 0 && dev < kMaxDevices) done[dev].store(true, std::memory_order_release);
   return e;
 }
 

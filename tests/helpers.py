@@ -76,25 +76,19 @@ def check_codes_near(q_gpu, q_orc, t_orc32, scale_orc, bits, min_agree=0.9999, h
     return agree
 
 
-# The fused tensor-core kernel (bf16 input, K in [128, 16384]) quantizes INT4
-# from the transformed, unscaled y (t = cmul y): beta = fl(cmul * S) / K with S
-# a float tree sum of |y| of depth <= 22 (10 levels inside a thread, 5 shuffle
-# levels, 7 slot additions), so beta is within 22 + 2 units in the last place
-# (1.5e-6) of the double sum over t, and the scale (beta times fl(1/sqrt 7))
-# within 1.5 more; codes are rint(y * fl(cmul r)) with r a fast division
-# (2 ulp), within 30 units of t r.  A code can then change only where the
-# exact t*r (|t*r| <= 8.5 for an unclipped code) lies within 8.5 * 30 units
-# (1.5e-5) of a half-integer.
-FUSED_BETA_REL = 2e-6
-FUSED_HALF_TOL = 3e-5
-
-
-def check_fused_int4(q_gpu, scales_gpu, q_orc, scales_orc, t32):
-    """Fused INT4 codes and scales against the oracle's quantizer on the same t."""
-    s = np.asarray(scales_gpu, np.float64)
-    so = np.asarray(scales_orc, np.float64)
-    assert np.all(np.abs(s - so) <= FUSED_BETA_REL * np.abs(so)), np.max(np.abs(s - so) / np.maximum(so, 1e-30))
-    return check_codes_near(q_gpu, q_orc, t32, scales_orc, 4, min_agree=0.9999, half_tol=FUSED_HALF_TOL)
+def check_codes_exact(q_gpu, scales_gpu, q_orc, scales_orc):
+    """Codes and scales of a kernel against the oracle's quantizer applied to
+    the same float t: bit for bit (the path's definition makes every decision
+    from t alone: the absmean a double sum rounded once, r and the scale
+    correctly rounded divisions, each code rint of the exact product t r)."""
+    q_gpu = np.asarray(q_gpu)
+    q_orc = np.asarray(q_orc)
+    s = np.asarray(scales_gpu, np.float32)
+    so = np.asarray(scales_orc, np.float32)
+    bad_s = np.nonzero(s.view(np.uint32) != so.view(np.uint32))[0]
+    assert bad_s.size == 0, "scales differ in rows %s: %s vs %s" % (bad_s[:8], s[bad_s[:8]], so[bad_s[:8]])
+    bad = q_gpu.astype(np.int32) != q_orc.astype(np.int32)
+    assert not bad.any(), "%d codes differ, first at %s" % (bad.sum(), np.argwhere(bad)[:4].tolist())
 
 
 def rel_fro(a, b):

@@ -10,7 +10,7 @@ Tolerances (stated by the path's definition):
 import numpy as np
 import pytest
 
-from helpers import check_fused_int4, check_codes_near, check_t, to_device, to_host, unpack_nibbles
+from helpers import check_codes_exact, check_codes_near, check_t, to_device, to_host, unpack_nibbles
 from ternary_gemm_b200.inputs import WORKLOADS, f32_to_bf16_bits, make_x, make_x_rows, sample_rows
 
 pytestmark = pytest.mark.gpu
@@ -116,20 +116,18 @@ def test_quant_hook_any_length(H, orc, K, bits):
 @pytest.mark.parametrize("bits", [4, 8])
 @pytest.mark.parametrize("K", KS)
 def test_fused_equals_quant_of_hook_t(H, orc, K, bits):
-    """The fused kernel quantizes its own t: bit for bit, except INT4 on the
-    tensor-core kernel (bf16, K in [128, 32768]), whose absmean is a float
-    sum (scales within 2e-6, codes off by one only at rounding boundaries)."""
+    """The fused kernel quantizes its own t bit for bit, both kernels (the
+    register one for K = 64, the tensor-core one from K = 128) and both
+    quantizers, packed and int8-widened."""
     x = x_for(K, "bf16")
     xd = to_device(x)
     t = to_host(H.hbl_debug_ln_fht(xd))
     codes, scales = H.hbl_fht_quant(xd, bits)
     q = unpack_nibbles(to_host(codes), K) if bits == 4 else to_host(codes)
     qo, so = orc.quant(t, bits)
-    if bits == 4 and 128 <= K <= 32768:
-        check_fused_int4(q, to_host(scales), qo, so, t)
-    else:
-        assert np.array_equal(q, qo)
-        assert np.array_equal(to_host(scales), so)
+    check_codes_exact(q, to_host(scales), qo, so)
+    codes_i8, scales_i8 = H.hbl_fht_quant_i8(xd, bits)
+    check_codes_exact(to_host(codes_i8), to_host(scales_i8), qo, so)
 
 
 @pytest.mark.parametrize("bits", [4, 8])
@@ -159,6 +157,16 @@ def test_fused_full_size_sampled_rows(H, orc, name, bits):
     check_codes_near(q, qo, t32, so, bits)
     s = to_host(scales)[rows].astype(np.float64)
     assert np.all(np.abs(s - so) <= 1e-5 * np.abs(so))
+    # bit for bit against the oracle's quantizer on the kernel's own t, in
+    # both output forms (the int8-widened one is what hbl_forward runs)
+    import torch
+    xd = to_device(x)
+    ridx = torch.from_numpy(rows).cuda()
+    t = to_host(H.hbl_debug_ln_fht(xd)[ridx])
+    qt, st = orc.quant(t, bits)
+    check_codes_exact(q, to_host(scales)[rows], qt, st)
+    codes_i8, scales_i8 = H.hbl_fht_quant_i8(xd, bits)
+    check_codes_exact(to_host(codes_i8[ridx]), to_host(scales_i8)[rows], qt, st)
 
 
 @pytest.mark.slow
