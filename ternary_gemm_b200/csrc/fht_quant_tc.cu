@@ -185,7 +185,7 @@ __device__ __forceinline__ float2 group_reduce2(float2 v, float2* slots, int wq,
   }
   if constexpr (RT > 32) {
     constexpr int NW = RT / 32;
-    if (lane == 0) slots[wq] = v;
+    slots[wq] = v;  // every lane holds the same value
     failed = named_bar_any(bar_id, bar_n, failed);
     const int w0 = wq & ~(NW - 1);
     v = slots[w0];
@@ -208,7 +208,7 @@ __device__ __forceinline__ float group_reduce1(float v, float* slots, int wq, in
   for (int o = W / 2; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
   if constexpr (RT > 32) {
     constexpr int NW = RT / 32;
-    if (lane == 0) slots[wq] = v;
+    slots[wq] = v;  // every lane holds the same value
     failed = named_bar_any(bar_id, bar_n, failed);
     const int w0 = wq & ~(NW - 1);
     v = slots[w0];
@@ -228,7 +228,7 @@ __device__ __forceinline__ double group_reduce_d(double v, double* slots, int wq
   for (int o = W / 2; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
   if constexpr (RT > 32) {
     constexpr int NW = RT / 32;
-    if (lane == 0) slots[wq] = v;
+    slots[wq] = v;  // every lane holds the same value
     named_bar_sync(bar_id, bar_n);
     const int w0 = wq & ~(NW - 1);
     v = slots[w0];
@@ -512,10 +512,7 @@ ln_fht_quant_tc_kernel(const __grid_constant__ CUtensorMap tmX, TcParams p) {
       // stale TMEM contents, same addresses, bounded waits) to the row
       // reduction, whose barrier ors the failure over every thread that
       // shares a barrier with this one, and all of them leave there.
-      int ok = 1;
-      if (lane == 0) ok = wait_bounded(&tfull[region], (uint32_t)(j / kRegions) & 1u, abort_flag, p.err) ? 1 : 0;
-      ok = __shfl_sync(0xffffffffu, ok, 0);
-      bool failed = ok == 0;
+      bool failed = !wait_bounded_warp(&tfull[region], (uint32_t)(j / kRegions) & 1u, abort_flag, p.err);
       fence_after();
       const uint32_t tl = tmem_base + (uint32_t)(region * 128) + ((uint32_t)(quarter * 32) << 16);
 
@@ -549,7 +546,7 @@ ln_fht_quant_tc_kernel(const __grid_constant__ CUtensorMap tmX, TcParams p) {
         stage<3>(y);
         stage<4>(y);
         stage<5>(y);
-        if (i_hi == 0) y[0] = 0.0f;  // t_0 = 0 (the mean's coefficient)
+        y[0] = i_hi == 0 ? 0.0f : y[0];  // t_0 = 0 (the mean's coefficient)
       } else {
         unit0 = 0;
         row = q;
@@ -612,7 +609,7 @@ ln_fht_quant_tc_kernel(const __grid_constant__ CUtensorMap tmX, TcParams p) {
         // column bit 6: y[r] = column 32h + r, y[32 + r] = column 64 + 32h + r
 #pragma unroll
         for (int r = 0; r < 32; r += 2) bfly2(y[r], y[r + 1], y[32 + r], y[33 + r]);
-        if (m == 0 && h == 0) y[0] = 0.0f;  // t_0 = 0
+        y[0] = (m == 0 && h == 0) ? 0.0f : y[0];  // t_0 = 0
       }
 
       // Row statistics.  Round 1: K^2 var = sum_{i>=1} Y_i^2, and for INT8
@@ -893,10 +890,7 @@ ln_fht_quant_tc256_kernel(const __grid_constant__ CUtensorMap tmX, TcParams p) {
       const int q = blockIdx.x + j * gridDim.x;
       if (q >= p.num_groups) break;
       const int region = j & 1;
-      int ok = 1;
-      if (lane == 0) ok = wait_bounded(&tfull[region], (uint32_t)(j >> 1) & 1u, abort_flag, p.err) ? 1 : 0;
-      ok = __shfl_sync(0xffffffffu, ok, 0);
-      bool failed = ok == 0;
+      bool failed = !wait_bounded_warp(&tfull[region], (uint32_t)(j >> 1) & 1u, abort_flag, p.err);
       fence_after();
       const uint32_t tl = tmem_base + (uint32_t)(region * k256Cols) + ((uint32_t)(quarter * 32) << 16);
 
@@ -948,7 +942,7 @@ ln_fht_quant_tc256_kernel(const __grid_constant__ CUtensorMap tmX, TcParams p) {
 #pragma unroll
       for (int r = 0; r < 32; r += 2) bfly2(y[r], y[r + 1], y[32 + r], y[33 + r]);
       // now y[r] = column 32 g + r, y[32 + r] = column 128 + 32 g + r
-      if (m == 0 && g == 0) y[0] = 0.0f;  // t_0 = 0
+      y[0] = (m == 0 && g == 0) ? 0.0f : y[0];  // t_0 = 0
 
       // the two statistic rounds of ln_fht_quant_tc_kernel, over all 512
       // epilogue threads

@@ -63,6 +63,40 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// try_wait that may suspend the thread for up to `hint_ns` (it returns as
+// soon as the phase completes): long waits cost a few issue slots instead of
+// a spin loop's.
+__device__ __forceinline__ bool mbar_try_wait_hint(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
+// wait_bounded for a whole warp (every lane executes it and gets the same
+// answer), suspending between polls: for consumers whose wait covers a whole
+// pipeline step.
+__device__ __forceinline__ bool wait_bounded_warp(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                                  int* err) {
+  if (mbar_try_wait_hint(bar, parity, 20000u)) return true;
+  const uint64_t limit = reinterpret_cast<const volatile DeviceStatus*>(err)->wait_limit_ns;
+  const uint64_t t0 = globaltimer();
+  for (;;) {
+    if (mbar_try_wait_hint(bar, parity, 20000u)) return true;
+    if (*abort_flag) return false;
+    if (globaltimer() - t0 > limit) {
+      *abort_flag = 1;
+      atomicExch(err, 1);
+      return false;
+    }
+  }
+}
+
 // Bounded wait for the phase with the given parity.  Returns false if the
 // CTA already aborted or the limit (the device status's wait_limit_ns) ran
 // out; then the CTA abort flag and the device error word are set.  `err`
@@ -72,7 +106,10 @@ __device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, vol
   const uint64_t limit = reinterpret_cast<const volatile DeviceStatus*>(err)->wait_limit_ns;
   const uint64_t t0 = globaltimer();
   for (uint32_t i = 1;; ++i) {
-    if (mbar_try_wait(bar, parity)) return true;
+    // suspend (up to 2 us, woken when the phase completes) instead of
+    // spinning: the polling thread shares its SM sub-partition with the
+    // consumers' warps
+    if (mbar_try_wait_hint(bar, parity, 2000u)) return true;
     if ((i & 63u) == 0) {
       if (*abort_flag) return false;
       if (globaltimer() - t0 > limit) {
