@@ -419,34 +419,53 @@ def measure_int8_peak(torch, dev, reps=10):
                    % (M, K, N, reps)}
 
 
+def packed_route(M, bits):
+    """hbl_forward's route through packed codes and the packed-operand GEMM: not taken
+    (measured slower than the int8-operand GEMM at every size)."""
+    return False
+
+
 def stage_times(torch, hbl, x, packed, alpha, N, bits, y, stream, n):
     """Mean seconds per launch of the forward's stages, through the stage entry points
-    (the same kernels hbl_forward runs): quantizer with int8 codes, weight widening, GEMM."""
+    (the same kernels hbl_forward runs): the quantizer, the weight widening (zero on the
+    packed route, which has none) and the GEMM."""
     M, K = x.shape
     dev = x.device
-    A = torch.empty((M, K), dtype=torch.int8, device=dev)
     sc = torch.empty((M,), dtype=torch.float32, device=dev)
-    Wi = torch.empty((N, K), dtype=torch.int8, device=dev)
+    if packed_route(M, bits):
+        q = torch.empty((M, K // 2), dtype=torch.uint8, device=dev)
+        stages = [lambda: hbl.hbl_fht_quant(x, 4, codes=q, scales=sc), None,
+                  lambda: hbl.hbl_gemm_tern_dequant(q, packed, sc, alpha, y=y)]
+    else:
+        q = torch.empty((M, K), dtype=torch.int8, device=dev)
+        Wi = torch.empty((N, K), dtype=torch.int8, device=dev)
+        stages = [lambda: hbl.hbl_fht_quant_i8(x, bits, codes=q, scales=sc),
+                  lambda: hbl.hbl_widen_ternary(packed, K, w=Wi),
+                  lambda: hbl.hbl_gemm_dequant(q, Wi, sc, alpha, y=y)]
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(n)]
     for _ in range(3):
-        hbl.hbl_fht_quant_i8(x, bits, codes=A, scales=sc)
-        hbl.hbl_widen_ternary(packed, K, w=Wi)
-        hbl.hbl_gemm_dequant(A, Wi, sc, alpha, y=y)
+        for f in stages:
+            if f is not None:
+                f()
     torch.cuda.synchronize()
     for i in range(n):
-        evs[i][0].record(stream)
-        hbl.hbl_fht_quant_i8(x, bits, codes=A, scales=sc)
-        evs[i][1].record(stream)
-        hbl.hbl_widen_ternary(packed, K, w=Wi)
-        evs[i][2].record(stream)
-        hbl.hbl_gemm_dequant(A, Wi, sc, alpha, y=y)
+        for j, f in enumerate(stages):
+            evs[i][j].record(stream)
+            if f is not None:
+                f()
         evs[i][3].record(stream)
     torch.cuda.synchronize()
     t_k1 = statistics.mean(e[0].elapsed_time(e[1]) for e in evs) / 1e3
     t_wd = statistics.mean(e[1].elapsed_time(e[2]) for e in evs) / 1e3
     t_gm = statistics.mean(e[2].elapsed_time(e[3]) for e in evs) / 1e3
-    del A, sc, Wi
     return t_k1, t_wd, t_gm
+
+
+def k1_bytes_of(M, K, x_bytes, bits):
+    """Algorithmic bytes of the forward's quantizer launch: x read, codes and scales written
+    (packed INT4 nibbles on the packed route, one byte per code otherwise)."""
+    codes = M * K // 2 if packed_route(M, bits) else M * K
+    return M * K * x_bytes + codes + 4 * M
 
 
 def config_numbers(torch, hbl, wl, bits, peaks, int8_peak, stream, x=None, packed=None, alpha=None):
@@ -465,7 +484,7 @@ def config_numbers(torch, hbl, wl, bits, peaks, int8_peak, stream, x=None, packe
     t = _events_timed(torch, lambda: hbl.hbl_forward(x, packed, alpha, N, bits, y=y, workspace=ws), n, stream)
     t_k1, t_wd, t_gm = stage_times(torch, hbl, x, packed, alpha, N, bits, y, stream, n)
     ops = 2.0 * M * N * K
-    k1_bytes = M * K * x.element_size() + M * K + 4 * M
+    k1_bytes = k1_bytes_of(M, K, x.element_size(), bits)
     out = {"workload": wl.name, "M": M, "K": K, "N": N, "bits": bits, "x_dtype": wl.dtype,
            "tokens_per_s": M / t, "ms_per_forward": t * 1e3,
            "gemm_tops": ops / t_gm / 1e12, "gemm_frac": ops / t_gm / 1e12 / int8_peak, "gemm_ms": t_gm * 1e3,
@@ -592,9 +611,12 @@ def bench_ours(args):
     int8_peak = max(i8["tops"] or 0.0, INT8_NOMINAL_TOPS)
     ops = 2.0 * M * N * K
     achieved_tops = ops / t_gm / 1e12
-    k1_bytes = M * K * (2 if wl.dtype == "bf16" else 4) + M * K + 4 * M
+    k1_bytes = k1_bytes_of(M, K, 2 if wl.dtype == "bf16" else 4, bits)
     k1_gbs = k1_bytes / t_k1 / 1e9
-    roofline = {"bound": "tensor", "kernel": "gemm_i8_2sm_kernel (tcgen05 kind::i8, cta_group::2, dequant epilogue)",
+    gemm_kernel = ("gemm_tern_pair_kernel (packed INT4 codes and 2-bit weights widened in shared memory; tcgen05 "
+                   "kind::i8, cta_group::2, dequant epilogue)" if packed_route(M, bits) else
+                   "gemm_i8_2sm_kernel (tcgen05 kind::i8, cta_group::2, dequant epilogue)")
+    roofline = {"bound": "tensor", "kernel": gemm_kernel,
                 "achieved": achieved_tops, "peak": int8_peak, "unit": "TFLOP/s", "frac": achieved_tops / int8_peak,
                 "traffic": measured_traffic("gemm_7b_wdown"),
                 "peak_source": "larger of the library int8 GEMM measured in this run (%s TOPS) and the nominal "
@@ -606,8 +628,8 @@ def bench_ours(args):
                 "algorithmic_ops_per_launch": ops, "launch_ms": t_gm * 1e3}
     if roofline["frac"] > 1.0:
         roofline["peak_suspect"] = "achieved above the peak: the denominator does not bound this kernel"
-    k1 = {"bound": "hbm", "kernel": "ln_fht_quant_tc_kernel (tcgen05 high Hadamard factor; INT%d, int8 codes out)"
-          % bits, "achieved": k1_gbs,
+    k1 = {"bound": "hbm", "kernel": "ln_fht_quant_tc_kernel (tcgen05 high Hadamard factor; INT%d, %s out)"
+          % (bits, "packed nibbles" if packed_route(M, bits) else "int8 codes"), "achieved": k1_gbs,
           "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": k1_gbs / peaks["hbm_gbs"],
           "traffic": measured_traffic("k1_7b_wdown"),
           "algorithmic_bytes_per_launch": k1_bytes, "launch_ms": t_k1 * 1e3}

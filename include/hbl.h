@@ -174,11 +174,26 @@ hbl_status hbl_debug_norm(const void* x, hbl_dtype xt, int64_t M, int64_t K, hbl
                           cudaStream_t stream);
 
 /* ---------------------------------------------------------------- forward stages
- * hbl_forward is exactly these three calls on slices of its workspace (for
- * decode-sized batches, M <= 4 and M * K <= 65536, the first call and then
- * hbl_gemv_ternary_dequant, whose y is identical); they are public so that
- * callers can keep the widened weight resident, overlap stages, or time each
- * kernel on their own stream. */
+ * hbl_forward is made of these calls on slices of its workspace: for
+ * decode-sized batches (M <= 4 and M * K <= 65536) hbl_fht_quant_i8 then
+ * hbl_gemv_ternary_dequant; otherwise hbl_fht_quant_i8, hbl_widen_ternary and
+ * hbl_gemm_dequant.  hbl_fht_quant then hbl_gemm_tern_dequant is another
+ * route to the identical y that needs no int8 buffers (it measured slower, so
+ * hbl_forward does not take it).  They are public so that callers can overlap
+ * stages or time each kernel on their own stream. */
+
+/* The integer GEMM and its dequantisation straight from the packed operands:
+ * y[m][n] = (float)(sum_k q[m][k] w[n][k]) * (scales[m] * alpha_dev[0]),
+ * stored as yt, with q the INT4 codes of hbl_fht_quant (device, [M][K/2],
+ * two per byte, element 2j in the low nibble) and w the 2-bit codes of
+ * hbl_pack_ternary (device, [N][K/4]).  Converter warps widen both to int8 in
+ * shared memory for the tcgen05 tensor cores (kind::i8); y is bit-identical
+ * to hbl_gemm_dequant on the widened codes.  Requires M >= 256 and K a
+ * multiple of 64 up to 32768 (else HBL_ERR_UNSUPPORTED), N a multiple of 16;
+ * scales, alpha_dev, y as in hbl_gemm_dequant. */
+hbl_status hbl_gemm_tern_dequant(const uint8_t* A, const uint8_t* packed, int64_t M, int64_t N, int64_t K,
+                                 const float* scales, const float* alpha_dev, void* y, hbl_dtype yt,
+                                 cudaStream_t stream);
 
 /* Activation path with one int8 per code (the layout the tensor cores read):
  * the same LN -> H -> quantizer as hbl_fht_quant, codes device int8 [M][K]

@@ -98,6 +98,8 @@ def lib():
             L.hbl_widen_ternary.restype = i32
             L.hbl_gemm_dequant.argtypes = [p, p, i64, i64, i64, p, p, p, i32, p]
             L.hbl_gemm_dequant.restype = i32
+            L.hbl_gemm_tern_dequant.argtypes = [p, p, i64, i64, i64, p, p, p, i32, p]
+            L.hbl_gemm_tern_dequant.restype = i32
             L.hbl_gemv_ternary_dequant.argtypes = [p, p, i64, i64, i64, p, p, p, i32, p]
             L.hbl_gemv_ternary_dequant.restype = i32
             L.hbl_debug_ln_fht.argtypes = [p, i32, i64, i64, p, p]
@@ -395,6 +397,20 @@ def hbl_widen_ternary(packed, K: int, w=None, stream=None):
         w = torch.empty((N, K), dtype=torch.int8, device=packed.device)
     _check(lib().hbl_widen_ternary(_ptr(packed), K, N, _ptr(w), _stream(stream)), "hbl_widen_ternary")
     return w
+
+
+def hbl_gemm_tern_dequant(codes, packed, scales, alpha, y=None, y_dtype=None, stream=None):
+    """Packed INT4 codes [M][K/2] (uint8), packed ternary [N][K/4] ->
+    y = (q w^T) * (scales[m] * alpha) [M][N] (M >= 256)."""
+    torch = _torch()
+    _need_cuda(codes, packed, scales, alpha)
+    M, K = codes.shape[0], codes.shape[1] * 2
+    N = packed.shape[0]
+    if y is None:
+        y = torch.empty((M, N), dtype=y_dtype or torch.bfloat16, device=codes.device)
+    _check(lib().hbl_gemm_tern_dequant(_ptr(codes), _ptr(packed), M, N, K, _ptr(scales), _ptr(alpha), _ptr(y),
+                                       _dtype_code(y), _stream(stream)), "hbl_gemm_tern_dequant")
+    return y
 
 
 def hbl_gemm_dequant(A, w, scales, alpha, y=None, y_dtype=None, stream=None):

@@ -76,6 +76,14 @@ cudaError_t launch_gemm_i8(const int8_t* A, const int8_t* B, int64_t M, int64_t 
                            int y_mode, void* y, const float* scales, const float* alpha,
                            cudaStream_t stream, int ab_max = 0);
 
+// The same product straight from packed INT4 codes A [M][K/2] and packed
+// ternary weights W [N][K/4] (gemm_packed.cu): M >= 256, K % 64 == 0;
+// y_mode 1 float, 2 bf16.  y is bit for bit that of launch_gemm_i8 on the
+// widened codes.
+bool gemm_tern_supports(int64_t M, int64_t K);
+cudaError_t launch_gemm_tern(const uint8_t* A, const uint8_t* W, int64_t M, int64_t N, int64_t K, int y_mode,
+                             void* y, const float* scales, const float* alpha, cudaStream_t stream);
+
 // Small-M product straight from the packed 2-bit weights with the same
 // dequantisation (y_mode 1 float, 2 bf16): M <= kGemvMaxRows and
 // M * K <= kGemvMaxCodeBytes (the code rows stay in L1), K % 64 == 0.

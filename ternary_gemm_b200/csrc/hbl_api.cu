@@ -59,11 +59,16 @@ hbl_status check_norm_k(int64_t K) {
   return HBL_OK;
 }
 
+// hbl_forward's workspace: int8 codes [M][K], scales [M], int8 weight codes
+// [N][K].  (The GEMM that reads packed codes, hbl_gemm_tern_dequant, needs
+// neither int8 buffer but measured slower at every size, so the forward keeps
+// the int8 operands.)
 struct ForwardLayout {
   size_t a_off, s_off, b_off, total;
 };
 
-ForwardLayout forward_layout(int64_t M, int64_t K, int64_t N) {
+ForwardLayout forward_layout(int64_t M, int64_t K, int64_t N, int bits) {
+  (void)bits;
   ForwardLayout L;
   L.a_off = 0;
   L.s_off = align256((size_t)M * (size_t)K);
@@ -122,7 +127,7 @@ size_t hbl_forward_workspace_bytes(int64_t M, int64_t K, int64_t N, int bits) {
   int l;
   if (check_k(K, &l) != HBL_OK || check_rows(M) != HBL_OK || check_n(N) != HBL_OK || (bits != 4 && bits != 8))
     return 0;
-  return forward_layout(M, K, N).total;
+  return forward_layout(M, K, N, bits).total;
 }
 
 hbl_status hbl_pack_ternary(const void* W, hbl_dtype wt, int64_t K, int64_t N, uint8_t* packed, float* alpha_dev,
@@ -163,14 +168,14 @@ hbl_status hbl_forward(const void* x, hbl_dtype xt, int64_t M, int64_t K, const 
   if (s != HBL_OK) return s;
   if ((s = check_rows(M)) != HBL_OK) return s;
   if ((s = check_n(N)) != HBL_OK) return s;
-  const ForwardLayout L = forward_layout(M, K, N);
+  const ForwardLayout L = forward_layout(M, K, N, bits);
   if (!workspace || !aligned(workspace, 256) || workspace_bytes < L.total) return HBL_ERR_WORKSPACE;
   uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
   int8_t* A = reinterpret_cast<int8_t*>(ws + L.a_off);
   float* scales = reinterpret_cast<float*>(ws + L.s_off);
   int8_t* B = reinterpret_cast<int8_t*>(ws + L.b_off);
-  const K1Mode mode = bits == 4 ? hbl::K1_Q4_I8 : hbl::K1_Q8_I8;
   cudaError_t e;
+  const K1Mode mode = bits == 4 ? hbl::K1_Q4_I8 : hbl::K1_Q8_I8;
   if (hbl::gemv_ternary_supports(M, K)) {
     // decode-sized batch: the product straight from the packed weights
     e = hbl::launch_ln_fht_quant(x, xt == HBL_BF16, M, l, mode, A, scales, stream);
@@ -225,6 +230,22 @@ hbl_status hbl_gemm_dequant(const int8_t* A, const int8_t* w, int64_t M, int64_t
   if (s != HBL_OK) return s;
   if ((s = check_n(N)) != HBL_OK) return s;
   return cuda_status(hbl::launch_gemm_i8(A, w, M, N, K, yt == HBL_BF16 ? 2 : 1, y, scales, alpha_dev, stream));
+}
+
+hbl_status hbl_gemm_tern_dequant(const uint8_t* A, const uint8_t* packed, int64_t M, int64_t N, int64_t K,
+                                 const float* scales, const float* alpha_dev, void* y, hbl_dtype yt,
+                                 cudaStream_t stream) {
+  if (!A || !packed || !scales || !alpha_dev || !y || !dtype_ok(yt)) return HBL_ERR_INVALID_ARG;
+  if (!aligned(A, 16) || !aligned(packed, 16) || !aligned(scales, 4) || !aligned(alpha_dev, 4) || !aligned(y, 16))
+    return HBL_ERR_INVALID_ARG;
+  if (K <= 0) return HBL_ERR_INVALID_ARG;
+  if (K % 64 != 0 || K > 32768) return HBL_ERR_UNSUPPORTED;
+  hbl_status s = check_rows(M);
+  if (s != HBL_OK) return s;
+  if ((s = check_n(N)) != HBL_OK) return s;
+  if (!hbl::gemm_tern_supports(M, K)) return HBL_ERR_UNSUPPORTED;
+  return cuda_status(hbl::launch_gemm_tern(A, packed, M, N, K, yt == HBL_BF16 ? 2 : 1, y, scales, alpha_dev,
+                                           stream));
 }
 
 hbl_status hbl_gemv_ternary_dequant(const int8_t* A, const uint8_t* packed, int64_t M, int64_t N, int64_t K,

@@ -291,6 +291,26 @@ __device__ __forceinline__ bool mbar_try_wait_acq_cluster(uint64_t* bar, uint32_
   return ok != 0;
 }
 
+// wait_bounded with cluster-scope acquire, for a barrier that threads of the
+// other CTA of the cluster arrive on after their own shared-memory stores
+__device__ __forceinline__ bool wait_bounded_cluster(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                                     int* err) {
+  if (mbar_try_wait_acq_cluster(bar, parity)) return true;
+  const uint64_t limit = reinterpret_cast<const volatile DeviceStatus*>(err)->wait_limit_ns;
+  const uint64_t t0 = globaltimer();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try_wait_acq_cluster(bar, parity)) return true;
+    if ((i & 63u) == 0) {
+      if (*abort_flag) return false;
+      if (globaltimer() - t0 > limit) {
+        *abort_flag = 1;
+        atomicExch(err, 1);
+        return false;
+      }
+    }
+  }
+}
+
 // complete-tx of `bytes` on a local barrier without a copy: stands in for
 // bytes a copy that was never issued would have delivered
 __device__ __forceinline__ void mbar_complete_tx(uint64_t* bar, uint32_t bytes) {

@@ -36,8 +36,13 @@ def test_size_queries(L):
     assert hbl.hbl_codes_bytes(8192, 16384, 4) == 8192 * 8192
     assert hbl.hbl_codes_bytes(8192, 16384, 8) == 8192 * 16384
     assert hbl.hbl_pack_ternary_workspace_bytes(256, 256) > 0
+    # int8 codes, scales and the widened weights
     ws = hbl.hbl_forward_workspace_bytes(8192, 16384, 4096, 4)
     assert ws >= 8192 * 16384 + 8192 * 4 + 4096 * 16384
+    ws = hbl.hbl_forward_workspace_bytes(8192, 16384, 4096, 8)
+    assert ws >= 8192 * 16384 + 8192 * 4 + 4096 * 16384
+    ws = hbl.hbl_forward_workspace_bytes(255, 16384, 4096, 4)
+    assert ws >= 255 * 16384 + 255 * 4 + 4096 * 16384
     # invalid sizes give 0
     assert hbl.hbl_packed_ternary_bytes(100, 256) == 0
     assert hbl.hbl_codes_bytes(8, 256, 5) == 0
@@ -120,6 +125,13 @@ def test_stage_validation(L):
     assert L.hbl_gemm_dequant(FAKE, FAKE, 8, 256, 72, FAKE, FAKE, FAKE, 1, S0) == E_UNS
     assert L.hbl_gemm_dequant(FAKE, FAKE, 8, 40, 256, FAKE, FAKE, FAKE, 1, S0) == E_UNS
     assert L.hbl_gemm_dequant(FAKE, FAKE, 8, 256, 1 << 17, FAKE, FAKE, FAKE, 1, S0) == E_UNS
+    # the GEMM from packed codes: M >= 256, K a multiple of 64 up to 32768
+    assert L.hbl_gemm_tern_dequant(FAKE, FAKE, 255, 256, 4096, FAKE, FAKE, FAKE, 1, S0) == E_UNS
+    assert L.hbl_gemm_tern_dequant(FAKE, FAKE, 256, 256, 96, FAKE, FAKE, FAKE, 1, S0) == E_UNS
+    assert L.hbl_gemm_tern_dequant(FAKE, FAKE, 256, 24, 4096, FAKE, FAKE, FAKE, 1, S0) == E_UNS
+    assert L.hbl_gemm_tern_dequant(FAKE, FAKE, 256, 256, 65536, FAKE, FAKE, FAKE, 1, S0) == E_UNS
+    assert L.hbl_gemm_tern_dequant(FAKE, NULL, 256, 256, 4096, FAKE, FAKE, FAKE, 1, S0) == E_ARG
+    assert L.hbl_gemm_tern_dequant(FAKE, FAKE, 256, 256, 4096, FAKE, FAKE, FAKE_ODD, 1, S0) == E_ARG
     # the packed-weight product is for decode-sized batches only
     assert L.hbl_gemv_ternary_dequant(FAKE, FAKE, 5, 256, 4096, FAKE, FAKE, FAKE, 1, S0) == E_UNS
     assert L.hbl_gemv_ternary_dequant(FAKE, FAKE, 4, 256, 32768, FAKE, FAKE, FAKE, 1, S0) == E_UNS

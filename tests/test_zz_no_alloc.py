@@ -58,7 +58,7 @@ def test_noalloc_forward_equals_forward_twice(bits):
 def test_noalloc_rejects_oversized_shapes():
     import torch
     L, hbl = _lib_and_hbl()
-    M, K, N = 4096, 8192, 4096                 # workspace 32 MiB + 32 MiB + scales > 32 MiB
+    M, K, N = 8192, 16384, 4096                # workspace: 64 MiB of packed codes + scales > 32 MiB
     assert hbl.hbl_forward_workspace_bytes(M, K, N, 4) > (32 << 20)
     x = torch.zeros((M, K), dtype=torch.bfloat16, device="cuda")
     packed = torch.zeros((N, K // 4), dtype=torch.uint8, device="cuda")
