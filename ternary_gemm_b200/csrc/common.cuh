@@ -31,8 +31,10 @@ cudaError_t launch_ln_fht_quant(const void* x, bool in_bf16, int64_t M, int log2
                                 void* out, float* scales, cudaStream_t stream);
 
 // The same operation with the high Hadamard factor on the tensor cores
-// (bf16 input, K in [128, 16384], 16-byte aligned x and out, not
-// K1_FHT_F32); launch_ln_fht_quant dispatches to it when supported.
+// (bf16 input, K in [128, 32768], 16-byte aligned x and out, not
+// K1_FHT_F32); launch_ln_fht_quant dispatches to it when supported and M is
+// above kRegisterKernelMaxRows.
+constexpr int64_t kRegisterKernelMaxRows = 4;
 bool ln_fht_quant_tc_supports(bool in_bf16, int log2k, K1Mode mode, const void* x, const void* out);
 cudaError_t launch_ln_fht_quant_tc(const void* x, int64_t M, int log2k, K1Mode mode, void* out, float* scales,
                                    cudaStream_t stream);

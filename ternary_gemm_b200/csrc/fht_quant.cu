@@ -547,7 +547,10 @@ quant_rows_kernel(const float* __restrict__ t, int64_t K, int bits, int packed, 
 
 cudaError_t launch_ln_fht_quant(const void* x, bool in_bf16, int64_t M, int log2k, K1Mode mode, void* out,
                                 float* scales, cudaStream_t stream) {
-  if (ln_fht_quant_tc_supports(in_bf16, log2k, mode, x, out))
+  // A few rows (decode-sized batches) go to the register kernel: the
+  // tensor-core kernel's setup (TMEM, barriers, the Hadamard operand) and one
+  // CTA's TMA/MMA round trips cost ~1 us more than the whole register kernel.
+  if (M > kRegisterKernelMaxRows && ln_fht_quant_tc_supports(in_bf16, log2k, mode, x, out))
     return launch_ln_fht_quant_tc(x, M, log2k, mode, out, scales, stream);
   switch (log2k) {
     case 6: return launch_k<6>(x, in_bf16, M, mode, out, scales, stream);

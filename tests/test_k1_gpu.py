@@ -29,8 +29,9 @@ def H():
 
 
 def rows_for(K):
-    # ragged against the rows-per-CTA of every shape (1..128 rows per CTA)
-    return {64: 131, 128: 67, 256: 35, 512: 19, 1024: 11, 2048: 7, 4096: 5}.get(K, 3)
+    # ragged against the rows-per-CTA of every shape (1..128 rows per CTA), and
+    # above the 4 rows that go to the register kernel for bf16 input
+    return {64: 131, 128: 67, 256: 35, 512: 19, 1024: 11, 2048: 7, 4096: 5}.get(K, 5)
 
 
 def x_for(K, dtype, dist="normal", M=None):

@@ -98,8 +98,10 @@ def test_tc_constant_and_zero_rows_bf16(H, orc, K, bits):
 
 
 def test_tc_single_row_and_partial_tile(H, orc):
-    """M * K / 128 below one tile (1 row of K = 4096 is 32 of 128 chunk rows)."""
-    for M, K in [(1, 4096), (3, 128), (1, 16384), (2, 8192), (1, 32768), (3, 32768)]:
+    """Fewer chunk rows than one MMA group (5 rows of K = 4096 are 160 of 256
+    chunk rows); up to 4 rows go to the register kernel, checked the same way."""
+    for M, K in [(5, 4096), (7, 128), (5, 16384), (6, 8192), (5, 32768), (1, 4096), (3, 128), (1, 16384),
+                 (2, 8192), (1, 32768), (3, 32768)]:
         wl = WORKLOADS["sweep"].with_shape(M, K, 256)
         x = make_x(wl)
         xd = to_device(x)
