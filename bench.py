@@ -529,7 +529,7 @@ def fwd_sweep(torch, hbl, stream):
         tg = _graph_timed(torch, lambda st: hbl.hbl_forward(x, packed, alpha, N, 4, y=y, workspace=ws, stream=st),
                           20)
         out.append({"M": M, "us_gpu": tg * 1e6, "tokens_per_s_gpu": M / tg, "us_eager": te * 1e6,
-                    "path": "quantizer + packed-weight kernel" if M <= 4 else "quantizer + tcgen05 GEMM"})
+                    "path": "one kernel: quantizer + packed-weight product" if M <= 4 else "quantizer + tcgen05 GEMM"})
         del x, y, ws
     return out
 

@@ -174,10 +174,12 @@ hbl_status hbl_debug_norm(const void* x, hbl_dtype xt, int64_t M, int64_t K, hbl
                           cudaStream_t stream);
 
 /* ---------------------------------------------------------------- forward stages
- * hbl_forward is made of these calls on slices of its workspace: for
- * decode-sized batches (M <= 4 and M * K <= 65536) hbl_fht_quant_i8 then
- * hbl_gemv_ternary_dequant; otherwise hbl_fht_quant_i8, hbl_widen_ternary and
- * hbl_gemm_dequant.  hbl_fht_quant then hbl_gemm_tern_dequant is another
+ * hbl_forward is made of these calls on slices of its workspace:
+ * hbl_fht_quant_i8, hbl_widen_ternary and hbl_gemm_dequant.  For
+ * decode-sized batches (M <= 4 and M * K <= 65536) it runs instead one kernel
+ * that does what hbl_fht_quant_i8 then hbl_gemv_ternary_dequant do, with the
+ * same arithmetic (y bit-identical), keeping the codes in shared memory and
+ * leaving the workspace untouched.  hbl_fht_quant then hbl_gemm_tern_dequant is another
  * route to the identical y that needs no int8 buffers (it measured slower, so
  * hbl_forward does not take it).  They are public so that callers can overlap
  * stages or time each kernel on their own stream. */

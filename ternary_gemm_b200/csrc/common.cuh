@@ -87,13 +87,26 @@ cudaError_t launch_gemm_tern(const uint8_t* A, const uint8_t* W, int64_t M, int6
                              void* y, const float* scales, const float* alpha, cudaStream_t stream);
 
 // Small-M product straight from the packed 2-bit weights with the same
-// dequantisation (y_mode 1 float, 2 bf16): M <= kGemvMaxRows and
-// M * K <= kGemvMaxCodeBytes (the code rows stay in L1), K % 64 == 0.
+// dequantisation (y_mode 1 float, 2 bf16): M <= kGemvMaxRows,
+// M * K <= kGemvMaxCodeBytes (the code rows live in shared memory), K a power
+// of two in 64 .. 32768.  `early`: the codes come from the stream's previous
+// kernel, which started after all earlier work, so the weight copies may
+// begin before the programmatic dependency wait.
 constexpr int64_t kGemvMaxRows = 4;
 constexpr int64_t kGemvMaxCodeBytes = 65536;
 bool gemv_ternary_supports(int64_t M, int64_t K);
 cudaError_t launch_gemv_ternary(const int8_t* A, const float* scales, const uint8_t* packed, const float* alpha,
-                                int64_t M, int64_t N, int64_t K, int y_mode, void* y, cudaStream_t stream);
+                                int64_t M, int64_t N, int64_t K, int y_mode, void* y, cudaStream_t stream,
+                                bool early = false);
+// The decode-sized forward in one launch (x -> LN -> transform -> quantize ->
+// product -> y), every CTA quantizing the rows itself: gemv_ternary_supports
+// and M * K <= kDecodeFusedMaxCodes (beyond that the redundant transforms cost
+// more than a second launch); x bf16 or float, bits 4 or 8, y_mode 1 float /
+// 2 bf16.
+constexpr int64_t kDecodeFusedMaxCodes = 16384;
+bool decode_forward_supports(int64_t M, int64_t K);
+cudaError_t launch_decode_forward(const void* x, bool x_bf16, int64_t M, int log2k, int bits, const uint8_t* packed,
+                                  const float* alpha, int64_t N, int y_mode, void* y, cudaStream_t stream);
 
 // Device error word (bounded-wait timeouts) -- lives in gemm_i8.cu; kernels in
 // other translation units receive its device address.

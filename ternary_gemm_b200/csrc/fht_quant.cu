@@ -43,154 +43,13 @@
 #include "sm100.cuh"
 #include "quant.cuh"
 #include "rowkit.cuh"
+#include "fht_rows.cuh"
 
 namespace hbl {
 namespace {
 
 using namespace rowkit;
-
-template <int LOGK>
-struct Shape {
-  static constexpr int K = 1 << LOGK;
-  static constexpr int E = 64;                          // elements per thread
-  static constexpr int T = K / E;                       // threads per row
-  static constexpr int R = T >= 128 ? 1 : 128 / T;      // rows per CTA
-  static constexpr int THREADS = T * R;
-  // CTAs per SM the register budget is tuned for: 512 threads -> 128 regs,
-  // 256 -> 80 regs (3 CTAs), 128 -> 96 regs (5 CTAs)
-  static constexpr int MINB = THREADS >= 512 ? 1 : (THREADS >= 256 ? 3 : 5);
-  static constexpr int PAD = T < 32 ? 16 : 0;           // floats of padding per row
-  static constexpr int STRIDE = K + PAD;                // floats per row in smem
-  static constexpr int WPR = T > 32 ? T / 32 : 1;       // warps per row
-  static constexpr size_t XCH = (size_t)R * STRIDE * 4;   // exchange buffer (floats)
-  static constexpr size_t RED = (size_t)R * WPR * 8;       // one row-reduction scratch
-  static constexpr size_t SMEM = XCH + 2 * RED;            // two reductions, separate slots
-  static constexpr int NPB = LOGK >= 10 ? LOGK - 9 : 0;  // pass-2 processed bits {6 .. 5+NPB}
-  static constexpr int PB = 6 - NPB;                      // pass-2 vector bits {0 .. PB-1}
-  static_assert(NPB >= 0 && NPB <= 6 && PB >= 0 && PB <= 6, "pass-2 split");
-};
-
-// The swizzle: index bits 5..8 XORed into bits 2..4 (linear over GF(2)).
-__host__ __device__ constexpr int swz(int i) {
-  return i ^ (((((i >> 5) ^ (i >> 6)) & 1) << 2) | (((i >> 7) & 1) << 3) | (((i >> 8) & 1) << 4));
-}
-
-// Shared-memory addresses of index (tb | C) for a per-thread tb and a
-// compile-time C with disjoint bits: swz(tb | C) = swz(tb) ^ swz(C); the XOR
-// part of swz(C) falls in bits 2..4 and selects one of eight bases, the rest
-// is an immediate offset.
-struct SwzBase {
-  int b[8];
-  __device__ __forceinline__ SwzBase(int row_off, int tb) {
-    const int s = swz(tb);
-#pragma unroll
-    for (int v = 0; v < 8; ++v) b[v] = row_off + (s ^ (v << 2));
-  }
-  template <int C>
-  __device__ __forceinline__ int at() const {
-    constexpr int sc = swz(C);
-    return b[(sc >> 2) & 7] + (sc & ~0x1C);
-  }
-};
-
-// Butterfly over register-index bit B: (e[r], e[r + 2^B]) -> (sum, difference).
-template <int B, int N>
-__device__ __forceinline__ void stage(float (&e)[N]) {
-  if constexpr (B == 0) {
-#pragma unroll
-    for (int r = 0; r < N; r += 2) {
-      float a = e[r], c = e[r + 1];
-      e[r] = a + c;
-      e[r + 1] = a - c;
-    }
-  } else {
-#pragma unroll
-    for (int r = 0; r < N; r += 2)
-      if (!(r & (1 << B))) bfly2(e[r], e[r + 1], e[r | (1 << B)], e[(r | (1 << B)) + 1]);
-  }
-}
-
-template <int N>
-__device__ __forceinline__ void stage_range(float (&e)[N], int lo, int hi) {
-  // register bits lo..hi-1 (lo, hi compile-time after inlining)
-  if (lo <= 0 && 0 < hi) stage<0>(e);
-  if (lo <= 1 && 1 < hi) stage<1>(e);
-  if (lo <= 2 && 2 < hi) stage<2>(e);
-  if (lo <= 3 && 3 < hi) stage<3>(e);
-  if (lo <= 4 && 4 < hi) stage<4>(e);
-  if (lo <= 5 && 5 < hi) stage<5>(e);
-}
-
-// Thread bit j of pass 2 -> index bit: {PB .. 5} then {k-3, k-2, k-1}.
-template <int LOGK>
-__host__ __device__ constexpr int p2_bit(int j) {
-  return j < 6 - Shape<LOGK>::PB ? Shape<LOGK>::PB + j : LOGK - 3 + (j - (6 - Shape<LOGK>::PB));
-}
-
-// 4 floats (or fewer, for vectors narrower than 16 bytes) at a smem address.
-template <int W>
-__device__ __forceinline__ void lds(const float* s, int a, float* o) {
-  if constexpr (W == 4) {
-    float4 v = *reinterpret_cast<const float4*>(s + a);
-    o[0] = v.x; o[1] = v.y; o[2] = v.z; o[3] = v.w;
-  } else if constexpr (W == 2) {
-    float2 v = *reinterpret_cast<const float2*>(s + a);
-    o[0] = v.x; o[1] = v.y;
-  } else {
-    o[0] = s[a];
-  }
-}
-
-template <int W>
-__device__ __forceinline__ void sts(float* s, int a, const float* o) {
-  if constexpr (W == 4) {
-    *reinterpret_cast<float4*>(s + a) = make_float4(o[0], o[1], o[2], o[3]);
-  } else if constexpr (W == 2) {
-    *reinterpret_cast<float2*>(s + a) = make_float2(o[0], o[1]);
-  } else {
-    s[a] = o[0];
-  }
-}
-
-template <int LOGK, int R0, int NREG>
-struct Pass2 {
-  // registers r = p * 2^PB + v  <->  index tb | (p << 6) | v; chunks of W floats
-  static constexpr int PB = Shape<LOGK>::PB;
-  static constexpr int W = PB >= 2 ? 4 : (PB == 1 ? 2 : 1);
-  template <int R>
-  __device__ __forceinline__ static void load(float (&e)[64], const float* smem, const SwzBase& sb) {
-    if constexpr (R < 64) {
-      constexpr int p = R >> PB, v = R & ((1 << PB) - 1);
-      lds<W>(smem, sb.at<(p << 6) | v>(), &e[R]);
-      load<R + W>(e, smem, sb);
-    }
-  }
-  template <int R>
-  __device__ __forceinline__ static void store(const float (&e)[64], float* smem, const SwzBase& sb) {
-    if constexpr (R < 64) {
-      constexpr int p = R >> PB, v = R & ((1 << PB) - 1);
-      sts<W>(smem, sb.at<(p << 6) | v>(), &e[R]);
-      store<R + W>(e, smem, sb);
-    }
-  }
-};
-
-template <int J>
-__device__ __forceinline__ void load_pass3(float (&e)[64], const float* smem, const SwzBase& sb) {
-  if constexpr (J < 16) {
-    lds<4>(smem, sb.at<4 * J>(), &e[4 * J]);
-    load_pass3<J + 1>(e, smem, sb);
-  }
-}
-
-template <int JJ, int T>
-__device__ __forceinline__ void store_pass1(const float (&e)[64], float* smem, const SwzBase& sb) {
-  if constexpr (JJ < 8) {
-    sts<4>(smem, sb.at<JJ * T * 8>(), &e[JJ * 8]);
-    sts<4>(smem, sb.at<JJ * T * 8 + 4>(), &e[JJ * 8 + 4]);
-    store_pass1<JJ + 1, T>(e, smem, sb);
-  }
-}
+using namespace fhtrows;
 
 // One CTA handles one group of R rows.
 // Sum of four floats over the T threads of a row (the RowReduce pattern with a
@@ -242,7 +101,6 @@ ln_fht_quant_kernel(const void* __restrict__ x, int64_t M, float sK, void* __res
   constexpr bool IN_BF16 = MODE == K1_LNBWD ? false : BF16;
   const size_t esz = IN_BF16 ? 2 : 4;
   const void* xrow = reinterpret_cast<const unsigned char*>(x) + (size_t)(active ? row : 0) * K * esz;
-  const int row_off = rl * S::STRIDE;
   // the plain transform and the backward transform have no forward LayerNorm
   constexpr bool kLN = MODE != K1_FHT_F32 && MODE != K1_LNBWD;
   // a programmatic dependent of this kernel may start now (it waits for this
@@ -250,75 +108,8 @@ ln_fht_quant_kernel(const void* __restrict__ x, int64_t M, float sK, void* __res
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   float e[64];
-
-  // ---- pass 1: load, remove a large row offset, stages of bits {0,1,2,k-3,k-2,k-1}
-  float f8[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-  if (active) {
-    load8<IN_BF16>(xrow, 0, f8);
-#pragma unroll
-    for (int jj = 0; jj < 8; ++jj) load8<IN_BF16>(xrow, (jj * T + t) * 8, &e[jj * 8]);
-  } else {
-#pragma unroll
-    for (int r = 0; r < 64; ++r) e[r] = 0.0f;
-  }
-  {
-    // mu~ = mean of the row's first 8 values; subtracted only when it exceeds
-    // their spread, i.e. when the row mean could cost float precision
-    const float mu = (((f8[0] + f8[1]) + (f8[2] + f8[3])) + ((f8[4] + f8[5]) + (f8[6] + f8[7]))) * 0.125f;
-    float lo = f8[0], hi = f8[0];
-#pragma unroll
-    for (int u = 1; u < 8; ++u) {
-      lo = fminf(lo, f8[u]);
-      hi = fmaxf(hi, f8[u]);
-    }
-    if (kLN && fabsf(mu) > hi - lo) {
-#pragma unroll
-      for (int r = 0; r < 64; r += 2) sub2(e[r], e[r + 1], mu);
-    }
-  }
-  stage_range(e, 0, 6);
-  {
-    SwzBase sb(row_off, t * 8);
-    store_pass1<0, T>(e, smem, sb);
-  }
-  __syncthreads();
-
-  // ---- pass 2: stages of bits {6 .. k-4} on vectors of 2^PB floats
-  if constexpr (LOGK >= 10) {
-    int tb = 0;
-#pragma unroll
-    for (int j = 0; j < LOGK - 6; ++j) tb |= ((t >> j) & 1) << p2_bit<LOGK>(j);
-    SwzBase sb(row_off, tb);
-    Pass2<LOGK, 0, 64>::template load<0>(e, smem, sb);
-    stage_range(e, S::PB, 6);
-    Pass2<LOGK, 0, 64>::template store<0>(e, smem, sb);
-    __syncthreads();
-  }
-
-  // ---- pass 3: 64 contiguous elements per thread, stages of bits {3,4,5} left
+  fht_ln_rows<S, IN_BF16, kLN>(xrow, active, rl, t, smem, reinterpret_cast<float*>(red1), sK, e);
   const int base = t * 64;
-  {
-    SwzBase sb(row_off, base);
-    load_pass3<0>(e, smem, sb);
-  }
-  stage_range(e, 3, LOGK - 3 < 6 ? LOGK - 3 : 6);
-
-  // ---- LayerNorm statistics from the transform: K^2 var = sum_{i>=1} Y_i^2
-  float cmul = sK;
-  if constexpr (kLN) {
-    float s0 = 0.0f, s1 = 0.0f;
-    const float e0 = e[0];
-    if (t == 0) e[0] = 0.0f;
-#pragma unroll
-    for (int r = 0; r < 64; r += 2) sq_acc2(s0, s1, e[r], e[r + 1]);
-    if (t == 0) e[0] = e0;
-    const float ss = RowReduce<T, S::WPR>::run(s0 + s1, AddF(), reinterpret_cast<float*>(red1), rl, t);
-    const float var = ss * (1.0f / ((float)K * (float)K));
-    cmul = __fmul_rn(__fdiv_rn(1.0f, sqrtf(__fadd_rn(var, 1e-5f))), sK);
-  }
-#pragma unroll
-  for (int r = 0; r < 64; r += 2) mul2(e[r], e[r + 1], cmul);
-  if (kLN && t == 0) e[0] = 0.0f;
 
   if constexpr (MODE == K1_LNBWD) {
     // e = g_u[base .. base + 63]; the LayerNorm backward at the forward's x of
@@ -386,29 +177,13 @@ ln_fht_quant_kernel(const void* __restrict__ x, int64_t M, float sK, void* __res
       for (int j = 0; j < 16; ++j) dst[j] = make_float4(e[4 * j], e[4 * j + 1], e[4 * j + 2], e[4 * j + 3]);
     }
   } else {
-    q::RowParams p;
-    if constexpr (MODE == K1_Q8_I8) {
-      float gm = 0.0f;
-#pragma unroll
-      for (int r = 0; r < 64; ++r) gm = fmaxf(gm, fabsf(e[r]));
-      gm = RowReduce<T, S::WPR>::run(gm, MaxF(), reinterpret_cast<float*>(red2), rl, t);
-      p = q::params_int8(gm);
-    } else {
-      double a0 = 0.0, a1 = 0.0;
-#pragma unroll
-      for (int r = 0; r < 64; r += 2) {
-        a0 += q::abs_f64(e[r]);
-        a1 += q::abs_f64(e[r + 1]);
-      }
-      const double a = RowReduce<T, S::WPR>::run(a0 + a1, AddD(), reinterpret_cast<double*>(red2), rl, t);
-      p = q::params_int4(a, K);
-    }
+    const q::RowParams p = row_params<S, MODE>(e, red2, rl, t);
     if (active) {
-      if (t == 0) scales[row] = p.scale;
-      uint32_t m[64];
-#pragma unroll
-      for (int r = 0; r < 64; r += 2) magic2(e[r], e[r + 1], p.r, m[r], m[r + 1]);
+      if (t == 0) scales[row] = p.scale();
       if constexpr (MODE == K1_Q4_PACKED) {
+        uint32_t m[64];
+#pragma unroll
+        for (int r = 0; r < 64; r += 2) magic2(e[r], e[r + 1], p.r, m[r], m[r + 1]);
         uint32_t w[8];
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
@@ -421,14 +196,8 @@ ln_fht_quant_kernel(const void* __restrict__ x, int64_t M, float sK, void* __res
         dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
         dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
       } else {
-        if constexpr (MODE == K1_Q4_I8) {
-#pragma unroll
-          for (int r = 0; r < 64; ++r) m[r] = q::clip_magic_int4(m[r]);
-        }
         uint32_t w[16];
-#pragma unroll
-        for (int j = 0; j < 16; ++j)
-          w[j] = q::gather_low_bytes(m[4 * j], m[4 * j + 1], m[4 * j + 2], m[4 * j + 3]);
+        codes64_i8<MODE>(e, p.r, w);
         uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(out) + (size_t)row * K + base);
 #pragma unroll
         for (int j = 0; j < 4; ++j) dst[j] = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
@@ -524,7 +293,7 @@ quant_rows_kernel(const float* __restrict__ t, int64_t K, int bits, int packed, 
     }
     p = q::params_int8(block_max(g, reinterpret_cast<float*>(red)));
   }
-  if (threadIdx.x == 0) scales[row] = p.scale;
+  if (threadIdx.x == 0) scales[row] = p.scale();
   for (int64_t c = threadIdx.x; c < nchunk; c += kQThreads) {
     float4 u = __ldg(reinterpret_cast<const float4*>(trow + c * 8));
     float4 v = __ldg(reinterpret_cast<const float4*>(trow + c * 8 + 4));

@@ -660,12 +660,13 @@ ln_fht_quant_tc_kernel(const __grid_constant__ CUtensorMap tmX, TcParams p) {
           qp = q::params_int8(__fmul_rn(cmul, gmax));
         } else {
           // round 2: beta = (float)(sum |t| / K) from a double sum, as the
-          // quantizer-only kernel computes it
+          // quantizer-only kernel computes it; the sum is scaled by 2^-896,
+          // so one multiply by 2^(896 - log2 K) gives the mean exactly
           const double sa = group_reduce_d<RT>(sum_abs64_scaled(y), redd + rset, wq, lane, bar_row, bar_row_n);
-          qp = q::params_int4(sa * q::kUnscaleAbs, K);
+          qp = q::params_int4_mean(sa * (q::kUnscaleAbs * q::pow2_recip(LOGK)));
         }
         const float cq = qp.r;  // codes are rint(t r)
-        if (row_ok && i_hi == 0 && (!PAIR || h == 0)) p.scales[row] = qp.scale;
+        if (row_ok && i_hi == 0 && (!PAIR || h == 0)) p.scales[row] = qp.scale();
         if (row_ok) {
           uint8_t* crow_out = p.codes + crow * (MODE == K1_Q4_PACKED ? C / 2 : C);
           if constexpr (MODE == K1_Q4_PACKED) {
@@ -980,11 +981,10 @@ ln_fht_quant_tc256_kernel(const __grid_constant__ CUtensorMap tmX, TcParams p) {
         if constexpr (MODE == K1_Q8_I8)
           qp = q::params_int8(__fmul_rn(cmul, gmax));
         else
-          qp = q::params_int4(group_reduce_d<512>(sum_abs64_scaled(y), redd + rset, wq, lane, bar_row, 512) *
-                                  q::kUnscaleAbs,
-                              K);
+          qp = q::params_int4_mean(group_reduce_d<512>(sum_abs64_scaled(y), redd + rset, wq, lane, bar_row, 512) *
+                                   (q::kUnscaleAbs * q::pow2_recip(15)));
         const float cq = qp.r;
-        if (m == 0 && g == 0) p.scales[row] = qp.scale;
+        if (m == 0 && g == 0) p.scales[row] = qp.scale();
         uint8_t* crow_out = p.codes + crow * (MODE == K1_Q4_PACKED ? k256Cols / 2 : k256Cols);
         if constexpr (MODE == K1_Q4_PACKED) {
           // 32 codes (16 bytes) per half, at bytes 16 g and 64 + 16 g

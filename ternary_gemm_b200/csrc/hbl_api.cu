@@ -176,11 +176,19 @@ hbl_status hbl_forward(const void* x, hbl_dtype xt, int64_t M, int64_t K, const 
   int8_t* B = reinterpret_cast<int8_t*>(ws + L.b_off);
   cudaError_t e;
   const K1Mode mode = bits == 4 ? hbl::K1_Q4_I8 : hbl::K1_Q8_I8;
+  if (hbl::decode_forward_supports(M, K)) {
+    // decode-sized batch: one launch quantizes x and takes the product
+    // straight from the packed weights (the workspace is not touched)
+    return cuda_status(hbl::launch_decode_forward(x, xt == HBL_BF16, M, l, bits, packed, alpha_dev, N,
+                                                  yt == HBL_BF16 ? 2 : 1, y, stream));
+  }
   if (hbl::gemv_ternary_supports(M, K)) {
-    // decode-sized batch: the product straight from the packed weights
+    // a few longer rows: the quantizer once, then the product from the packed
+    // weights, whose copies start while the quantizer runs
     e = hbl::launch_ln_fht_quant(x, xt == HBL_BF16, M, l, mode, A, scales, stream);
     if (e == cudaSuccess)
-      e = hbl::launch_gemv_ternary(A, scales, packed, alpha_dev, M, N, K, yt == HBL_BF16 ? 2 : 1, y, stream);
+      e = hbl::launch_gemv_ternary(A, scales, packed, alpha_dev, M, N, K, yt == HBL_BF16 ? 2 : 1, y, stream,
+                                   /*early=*/true);
     return cuda_status(e);
   }
   if (hbl::ln_fht_quant_tc_supports(xt == HBL_BF16, l, mode, x, A)) {

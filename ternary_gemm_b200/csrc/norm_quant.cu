@@ -111,7 +111,7 @@ norm_quant_kernel(const void* __restrict__ x, int64_t M, void* __restrict__ out,
       p = q::params_int4(RowReduce<T, S::WPR>::run(a0 + a1, AddD(), red_d, rl, t), K);
     }
     if (!active) return;
-    if (t == 0) scales[row] = p.scale;
+    if (t == 0) scales[row] = p.scale();
     uint32_t m[64];
 #pragma unroll
     for (int r = 0; r < 64; r += 2) magic2(e[r], e[r + 1], p.r, m[r], m[r + 1]);

@@ -45,24 +45,41 @@ __device__ __forceinline__ double abs_scaled_f64(float t) {
 constexpr double kUnscaleAbs = 0x1p896;
 
 struct RowParams {
-  float r;      // multiplier applied to t before rounding
-  float scale;  // dequantisation factor of the row
+  float r;     // multiplier applied to t before rounding
+  float stat;  // beta (INT4) or gamma (INT8)
+  float c;     // sqrt(7) or 127
+  // dequantisation factor of the row, stat / c (one IEEE division; computed
+  // only by the thread that stores it)
+  __device__ __forceinline__ float scale() const { return __fdiv_rn(stat, c); }
 };
+
+// beta from the mean of |t|, already formed in double and rounded here once.
+__device__ __forceinline__ RowParams params_int4_mean(double abs_mean) {
+  RowParams p;
+  p.stat = (float)abs_mean;
+  p.c = kSqrt7;
+  p.r = __fdiv_rn(kSqrt7, __fadd_rn(p.stat, kEps));
+  return p;
+}
 
 // beta from the double sum of |t| over K elements.
 __device__ __forceinline__ RowParams params_int4(double abs_sum, int64_t K) {
-  float beta = (float)(abs_sum / (double)K);
-  RowParams p;
-  p.r = __fdiv_rn(kSqrt7, __fadd_rn(beta, kEps));
-  p.scale = __fdiv_rn(beta, kSqrt7);
-  return p;
+  return params_int4_mean(abs_sum / (double)K);
+}
+
+// The same for K = 2^log2k: dividing by a power of two and multiplying by its
+// reciprocal give the identical double (both the correctly rounded value of
+// the same real number), without the division sequence.
+__device__ __forceinline__ double pow2_recip(int log2k) {
+  return __longlong_as_double((long long)(1023 - log2k) << 52);
 }
 
 // gamma = max |t| (exact, order free).
 __device__ __forceinline__ RowParams params_int8(float gamma) {
   RowParams p;
+  p.stat = gamma;
+  p.c = 127.0f;
   p.r = __fdiv_rn(127.0f, __fadd_rn(gamma, kEps));
-  p.scale = __fdiv_rn(gamma, 127.0f);
   return p;
 }
 

@@ -1,10 +1,13 @@
 """GPU parity of the decode-sized product straight from the packed ternary
-weights (hbl_gemv_ternary_dequant, and hbl_forward, which uses it for M <= 4
-and M * K <= 65536).
+weights (hbl_gemv_ternary_dequant) and of hbl_forward's one-launch decode
+kernel (M <= 4 and M * K <= 65536), which quantizes x itself with the
+quantizer kernel's arithmetic and keeps the codes in shared memory.
 
 Tolerances: y bit-exact, against both the tensor-core GEMM + dequantisation
 on the same codes and the oracle's int64 GEMM + float dequantisation (the int32
-sums are exact and the rescaling is the same two float products).
+sums are exact and the rescaling is the same two float products).  The fused
+decode forward is bit-exact against the stage path (hbl_fht_quant_i8, whose
+codes and scales the oracle pins, then the tensor-core GEMM).
 """
 import numpy as np
 import pytest
@@ -64,17 +67,58 @@ def test_gemv_rejects_large_batches(H, orc):
         assert ei.value.status == H.HBL_ERR_UNSUPPORTED
 
 
-@pytest.mark.parametrize("bits", [4, 8])
-@pytest.mark.parametrize("M,K,N", [(1, 4096, 4096), (3, 1024, 48), (4, 4096, 272), (2, 32768, 64),
-                                   (5, 4096, 4096)])
-def test_forward_decode_path_matches_tensor_path(H, orc, bits, M, K, N):
-    """hbl_forward at decode size equals the stage-by-stage tensor-core path."""
+def _decode_vs_stages(H, x_host, W, bits, y_dtype=None):
     import torch
-    wl = WORKLOADS["sweep"].with_shape(M, K, N)
-    x = to_device(make_x(wl))
-    packed, alpha = H.hbl_pack_ternary(to_device(make_w(wl)))
-    y = H.hbl_forward(x, packed, alpha, N, bits)
+    M, K = x_host.shape
+    N = W.shape[0]
+    x = to_device(x_host)
+    packed, alpha = H.hbl_pack_ternary(to_device(W))
+    y = H.hbl_forward(x, packed, alpha, N, bits, y_dtype=y_dtype)
     codes, scales = H.hbl_fht_quant_i8(x, bits)
-    y_tc = H.hbl_gemm_dequant(codes, H.hbl_widen_ternary(packed, K), scales, alpha)
+    y_tc = H.hbl_gemm_dequant(codes, H.hbl_widen_ternary(packed, K), scales, alpha, y_dtype=y.dtype)
     torch.cuda.synchronize()
     assert np.array_equal(to_host(y), to_host(y_tc))
+    assert H.hbl_last_device_error() == H.HBL_OK
+    return to_host(codes), to_host(scales), to_host(y)
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+@pytest.mark.parametrize("M,K,N", [(1, 4096, 4096), (3, 1024, 48), (4, 4096, 272), (2, 32768, 64),
+                                   (5, 4096, 4096), (1, 64, 16), (4, 128, 80), (4, 256, 16), (3, 512, 112),
+                                   (4, 2048, 4096), (2, 8192, 528), (4, 16384, 1040), (1, 32768, 4096),
+                                   (1, 4096, 8192), (2, 1024, 10000 // 16 * 16)])
+def test_forward_decode_path_matches_tensor_path(H, orc, bits, M, K, N):
+    """hbl_forward at decode size equals the stage-by-stage tensor-core path:
+    every power-of-two K, ragged N (a partial last block of 32 weight rows),
+    and N above 148 x 32 (CTAs that take several blocks)."""
+    wl = WORKLOADS["sweep"].with_shape(M, K, N)
+    _decode_vs_stages(H, make_x(wl), make_w(wl), bits)
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+def test_forward_decode_float_input_and_output(H, orc, bits):
+    """float x (the small workload's dtype) and float y through the fused
+    decode kernel; y also bit-exact against the oracle's GEMM + dequant of the
+    codes."""
+    import torch
+    wl = WORKLOADS["sweep"].with_shape(4, 1024, 272)
+    # float values that bf16 cannot hold
+    x = np.ascontiguousarray(orc.bf16_bits_to_float(make_x(wl)), dtype=np.float32) * np.float32(1.1)
+    W = make_w(wl)
+    codes, scales, y = _decode_vs_stages(H, x, W, bits, y_dtype=torch.float32)
+    w, a = orc.ternary(W)
+    assert np.array_equal(y, orc.dequant(orc.gemm_i32(codes, w), scales, a))
+
+
+def test_forward_decode_degenerate_rows(H, orc):
+    """A zero row, a constant row (LayerNorm gives zeros: codes 0, scale 0) and
+    a row with a large mean through the fused decode kernel."""
+    wl = WORKLOADS["sweep"].with_shape(4, 4096, 272)
+    x = orc.bf16_bits_to_float(make_x(wl)).astype(np.float32)
+    x[0] = 0.0
+    x[1] = 3.0
+    x[2] = x[2] + 1000.0
+    x = orc.round_to_bf16(x)
+    codes, scales, _ = _decode_vs_stages(H, x, make_w(wl), 4)
+    assert scales[0] == 0.0 and not codes[0].any()
+    assert scales[1] == 0.0 and not codes[1].any()
