@@ -461,6 +461,24 @@ def stage_times(torch, hbl, x, packed, alpha, N, bits, y, stream, n):
     return t_k1, t_wd, t_gm
 
 
+def stage_graph_times(torch, hbl, x, packed, alpha, N, bits, y, n):
+    """Device seconds per launch of the forward's stages (quantizer, widening, GEMM),
+    each captured n times in a CUDA graph: no host launch cost, which small shapes
+    would otherwise measure."""
+    M, K = x.shape
+    dev = x.device
+    sc = torch.empty((M,), dtype=torch.float32, device=dev)
+    q = torch.empty((M, K), dtype=torch.int8, device=dev)
+    Wi = torch.empty((N, K), dtype=torch.int8, device=dev)
+    hbl.hbl_fht_quant_i8(x, bits, codes=q, scales=sc)
+    hbl.hbl_widen_ternary(packed, K, w=Wi)
+    t_k1 = _graph_timed(torch, lambda st: hbl.hbl_fht_quant_i8(x, bits, codes=q, scales=sc, stream=st), n)
+    t_wd = _graph_timed(torch, lambda st: hbl.hbl_widen_ternary(packed, K, w=Wi, stream=st), n)
+    t_gm = _graph_timed(torch, lambda st: hbl.hbl_gemm_dequant(q, Wi, sc, alpha, y=y, stream=st), n)
+    del q, Wi, sc
+    return t_k1, t_wd, t_gm
+
+
 def k1_bytes_of(M, K, x_bytes, bits):
     """Algorithmic bytes of the forward's quantizer launch: x read, codes and scales written
     (packed INT4 nibbles on the packed route, one byte per code otherwise)."""
@@ -481,15 +499,18 @@ def config_numbers(torch, hbl, wl, bits, peaks, int8_peak, stream, x=None, packe
     y = torch.empty((M, N), dtype=x.dtype, device=x.device)
     ws = torch.empty((hbl.hbl_forward_workspace_bytes(M, K, N, bits),), dtype=torch.uint8, device=x.device)
     n = 50 if M * K <= (1 << 25) else 20
-    t = _events_timed(torch, lambda: hbl.hbl_forward(x, packed, alpha, N, bits, y=y, workspace=ws), n, stream)
-    t_k1, t_wd, t_gm = stage_times(torch, hbl, x, packed, alpha, N, bits, y, stream, n)
+    t_eager = _events_timed(torch, lambda: hbl.hbl_forward(x, packed, alpha, N, bits, y=y, workspace=ws), n,
+                            stream)
+    t = _graph_timed(torch, lambda st: hbl.hbl_forward(x, packed, alpha, N, bits, y=y, workspace=ws, stream=st), n)
+    t_k1, t_wd, t_gm = stage_graph_times(torch, hbl, x, packed, alpha, N, bits, y, n)
     ops = 2.0 * M * N * K
     k1_bytes = k1_bytes_of(M, K, x.element_size(), bits)
     out = {"workload": wl.name, "M": M, "K": K, "N": N, "bits": bits, "x_dtype": wl.dtype,
-           "tokens_per_s": M / t, "ms_per_forward": t * 1e3,
+           "tokens_per_s": M / t, "ms_per_forward": t * 1e3, "ms_per_forward_eager": t_eager * 1e3,
            "gemm_tops": ops / t_gm / 1e12, "gemm_frac": ops / t_gm / 1e12 / int8_peak, "gemm_ms": t_gm * 1e3,
            "k1_gbs": k1_bytes / t_k1 / 1e9, "k1_frac": k1_bytes / t_k1 / 1e9 / peaks["hbm_gbs"],
-           "k1_ms": t_k1 * 1e3, "widen_ms": t_wd * 1e3}
+           "k1_ms": t_k1 * 1e3, "widen_ms": t_wd * 1e3,
+           "timing": "device time: n launches captured in one CUDA graph (eager: host launches included)"}
     del y, ws
     return out
 
