@@ -181,7 +181,8 @@ def test_device_error_word(H):
 
 @pytest.mark.parametrize("bits", [4, 8])
 @pytest.mark.parametrize("M,K,N", [(5, 4096, 4096), (33, 1024, 1040), (64, 4096, 256), (65, 4096, 4096),
-                                   (100, 1024, 528), (128, 4096, 4096), (200, 2048, 1040), (255, 4096, 2048)])
+                                   (100, 1024, 528), (128, 4096, 4096), (200, 2048, 1040), (255, 4096, 2048),
+                                   (16, 16384, 1040), (9, 256, 48), (7, 128, 272)])
 def test_forward_short_batch_split_matches_stage_path(H, orc, bits, M, K, N):
     """Short batches split K over a cluster; with INT4 codes and ternary weights
     each rank's partial is bounded by 8 x its k-range and is exchanged as int16
