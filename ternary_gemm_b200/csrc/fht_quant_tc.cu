@@ -58,11 +58,12 @@
 //              statistics, quantizer, codes stored straight to global memory
 //              (each warp writes whole consecutive chunk rows).
 // Row statistics reduce over the threads of a token row: warp shuffles, then
-// per-warp slots behind a named barrier of the row's warpgroup (pair).  Round
-// 1 gives sum Y^2 (and for INT8 max |y| of the transformed but unscaled y),
-// hence cmul; every mode then forms t = fl(cmul y), the value the debug mode
-// writes out.  INT8 is exact from round 1: gamma = fl(cmul max|y|) = max|t|
-// (rounding is monotone).  INT4 needs sum |t| itself: round 2 sums |t| in
+// per-warp slots behind a named barrier of the row's warpgroup (pair).  The
+// first reduction gives sum Y^2 (and for INT8 max |y| of the transformed but
+// unscaled y), hence cmul; every mode then forms t = fl(cmul y), the value the
+// debug mode writes out.  INT8 is exact from the first reduction: gamma =
+// fl(cmul max|y|) = max|t| (rounding is monotone).  INT4 needs sum |t|
+// itself: a second reduction sums |t| in
 // double (each |t| made exactly from its bits, scaled by a power of two) and
 // rounds the mean once to float, as the quantizer-only kernel does.  Both then take r = c / (stat + eps) and
 // the scale stat / c as correctly rounded divisions and the codes as
@@ -612,10 +613,10 @@ ln_fht_quant_tc_kernel(const __grid_constant__ CUtensorMap tmX, TcParams p) {
         y[0] = (m == 0 && h == 0) ? 0.0f : y[0];  // t_0 = 0
       }
 
-      // Row statistics.  Round 1: K^2 var = sum_{i>=1} Y_i^2, and for INT8
-      // max |y| (max |t| = fl(cmul max |y|) exactly, rounding being
+      // Row statistics.  First reduction: K^2 var = sum_{i>=1} Y_i^2, and for
+      // INT8 max |y| (max |t| = fl(cmul max |y|) exactly, rounding being
       // monotone).  INT4 needs sum |t| over t = fl(cmul y) itself, which
-      // exists only once cmul is known: round 2 sums it in double.
+      // exists only once cmul is known: a second reduction sums it in double.
       const int rset = 16 * pr + 8 * ((j >> 1) & 1) + (PAIR ? 0 : 4 * h);
       float ss, gmax = 0.0f;
       if constexpr (MODE == K1_Q8_I8) {
@@ -659,7 +660,7 @@ ln_fht_quant_tc_kernel(const __grid_constant__ CUtensorMap tmX, TcParams p) {
         if constexpr (MODE == K1_Q8_I8) {
           qp = q::params_int8(__fmul_rn(cmul, gmax));
         } else {
-          // round 2: beta = (float)(sum |t| / K) from a double sum, as the
+          // second reduction: beta = (float)(sum |t| / K) from a double sum, as the
           // quantizer-only kernel computes it; the sum is scaled by 2^-896,
           // so one multiply by 2^(896 - log2 K) gives the mean exactly
           const double sa = group_reduce_d<RT>(sum_abs64_scaled(y), redd + rset, wq, lane, bar_row, bar_row_n);
