@@ -140,6 +140,24 @@ def aggregate_value(tokens_per_rank: int, world: int, max_seconds_per_step: floa
 
 # ------------------------------------------------------------------ clocks
 
+# Throttle reasons that make a timed region unusable: the GPU slowed itself
+# down for protection (power-cap throttling, sw_power_cap, is normal for a
+# dense GEMM on a 1 kW part and is kept and reported).
+BAD_REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown")
+
+
+def clocks_rejected(clk) -> bool:
+    """True if a clock record disqualifies its timed region: a hardware or
+    thermal slowdown was active, or the SM clock under load sat well below its
+    maximum (under 70%) with no reason reported (a clock lock left behind by
+    someone else).  Such a region is measured once more."""
+    if not clk or clk.get("sm_mhz") is None:
+        return False
+    if any(r in BAD_REASONS for r in clk.get("reasons", [])):
+        return True
+    mx = clk.get("sm_max_mhz")
+    return bool(mx) and not clk.get("reasons") and clk["sm_mhz"] < 0.7 * mx
+
 class ClockSampler:
     """SM clock, power and clock-event reasons sampled while timing: NVML every
     millisecond (a timed region of a few milliseconds still gets samples),
@@ -597,24 +615,32 @@ def bench_ours(args):
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
-    clocks = ClockSampler(gpu_uuid)
-    clocks.start()
-    clocks.wait_first_sample()
-
     # -------- headline: K whole forwards
-    ranks.barrier()
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.steps):
-        step()
-    e1.record(stream)
-    e1.synchronize()
-    ranks.barrier()
-    torch.cuda.synchronize()
-    clk = clocks.stop()
-    ms = e0.elapsed_time(e1) / args.steps
+    def timed_region():
+        clocks = ClockSampler(gpu_uuid)
+        clocks.start()
+        clocks.wait_first_sample()
+        ranks.barrier()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+        e1.synchronize()
+        ranks.barrier()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / args.steps, clocks.stop()
+
+    ms, clk = timed_region()
     ms_max = ranks.max(ms, dev)
+    # a region that any rank's clock record disqualifies is measured once more
+    # (every rank takes the same decision: the flag is maxed over ranks)
+    rejected = None
+    if ranks.max(1.0 if clocks_rejected(clk) else 0.0, dev) > 0:
+        rejected = {"ms_per_step": ms_max, "clocks": clk}
+        ms, clk = timed_region()
+        ms_max = ranks.max(ms, dev)
     value = aggregate_value(M, ranks.world, ms_max / 1e3)
 
     # -------- per-kernel times through the stage entry points (same kernels as hbl_forward)
@@ -748,6 +774,8 @@ def bench_ours(args):
                           "clocks": stage_clk},
             "cpu_baseline": cpu, "cpu_baseline_all_cores": cpu_all, "e2e": e2e, "gpu_launches": 2 * args.steps,
             "clocks": clk}
+    if rejected is not None:
+        line["remeasured"] = {"why": "the first timed region's clock record showed a slowdown", "first": rejected}
     line.update(extras)
     if ranks.rank == 0:
         print(json.dumps(line), flush=True)

@@ -92,3 +92,20 @@ def test_clock_parser():
     r = c.stop()
     assert r["sm_mhz"] == 1900 and r["sm_max_mhz"] == 1965 and r["reasons"] == ["sw_power_cap"]
     assert r["samples"] == 3
+
+
+def test_clock_record_rejection():
+    """A timed region is measured again when its clock record shows a hardware
+    or thermal slowdown, or a clock far below its maximum with no reason (a
+    leftover clock lock); power-cap throttling alone is kept."""
+    ok = {"sm_mhz": 1590.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"], "samples": 500}
+    assert not bench.clocks_rejected(ok)
+    assert not bench.clocks_rejected({"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": [], "samples": 9})
+    for r in bench.BAD_REASONS:
+        assert bench.clocks_rejected(dict(ok, reasons=["sw_power_cap", r]))
+    assert bench.clocks_rejected({"sm_mhz": 1000.0, "sm_max_mhz": 1965.0, "reasons": [], "samples": 50})
+    # a low clock with the power cap active is the cap, not a lock
+    assert not bench.clocks_rejected(dict(ok, sm_mhz=1000.0))
+    # no clock source: nothing to judge
+    assert not bench.clocks_rejected({"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no clock source"],
+                                      "samples": 0})
