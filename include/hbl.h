@@ -85,8 +85,9 @@ size_t hbl_forward_workspace_bytes(int64_t M, int64_t K, int64_t N, int bits);
 
 /* ---------------------------------------------------------------- compute */
 
-/* Ternary weight quantization ("per-tensor absmean quantizes the weights to
- * {-1, 0, 1}"; weight-quantization formula of section "H-BitLinear").
+/* Ternary weight quantization (the weights are quantized per tensor by
+ * absmean to {-1, 0, 1}: the weight-quantization formula of section
+ * "H-BitLinear").
  *   W         device, [N][K] of dtype wt (HBL_F32 or HBL_BF16)
  *   packed    device, hbl_packed_ternary_bytes(K, N) bytes (output)
  *   alpha_dev device, one float (output): alpha = mean|W| (accumulated in
@@ -99,8 +100,8 @@ hbl_status hbl_pack_ternary(const void* W, hbl_dtype wt, int64_t K, int64_t N, u
                             cudaStream_t stream);
 
 /* LN -> H -> per-token quantization of M rows (the activation path of
- * H-BitLinear: LayerNorm, online Hadamard transformation, then "per-token
- * absmean (4-bit) / absmax (8-bit)" quantization).
+ * H-BitLinear: LayerNorm, online Hadamard transformation, then per-token
+ * absmean quantization for 4 bits or absmax quantization for 8 bits).
  *   x      device, [M][K] of dtype xt
  *   bits   4 or 8
  *   codes  device, hbl_codes_bytes(M, K, bits) bytes (output, layout above)
@@ -123,7 +124,9 @@ hbl_status hbl_fht_quant(const void* x, hbl_dtype xt, int64_t M, int64_t K, int 
  *   workspace  device, >= hbl_forward_workspace_bytes(M, K, N, bits) bytes,
  *              256-byte aligned; its contents are scratch
  * The integer GEMM runs on the tcgen05 tensor cores (kind::i8) with exact
- * int32 accumulation. */
+ * int32 accumulation; decode-sized batches (M <= 4, M * K <= 65536) take exact
+ * dp4a products straight from the packed weights instead, with the same y
+ * (see "forward stages" below). */
 hbl_status hbl_forward(const void* x, hbl_dtype xt, int64_t M, int64_t K, const uint8_t* packed,
                        const float* alpha_dev, int64_t N, int bits, void* y, hbl_dtype yt,
                        void* workspace, size_t workspace_bytes, cudaStream_t stream);
@@ -154,8 +157,8 @@ hbl_status hbl_pack_ternary_rotated(const void* W, hbl_dtype wt, int64_t K, int6
 
 /* ---------------------------------------------------------------- BitLinear without the transform
  * The activation path of the BitLinear layers that have no Hadamard
- * transform ("all linear layers except the input/output embeddings" are
- * fine-tuned to 4-bit activations, H-BitLinear only replaces Wo and Wdown;
+ * transform (every linear layer but the input and output embeddings moves to
+ * 4-bit activations, and H-BitLinear replaces only Wo and Wdown;
  * BitNet b1.58 keeps 8-bit absmax activations): normalisation, then the same
  * per-token quantizer as hbl_fht_quant. */
 typedef enum { HBL_NORM_LAYER = 0, HBL_NORM_RMS = 1 } hbl_norm;

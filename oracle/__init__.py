@@ -120,7 +120,8 @@ def _as_input(x: np.ndarray):
 
 
 def layernorm_row(x: np.ndarray) -> np.ndarray:
-    """LayerNorm of one row in double, no affine, eps 1e-5 ("LN denotes LayerNorm")."""
+    """LayerNorm of one row in double, no affine, eps 1e-5 (the symbol LN of the
+    matrix-operation formula is LayerNorm)."""
     x = np.ascontiguousarray(x, dtype=np.float64)
     u = np.empty_like(x)
     _L().orc_layernorm_row(_ptr(x), x.size, _ptr(u))

@@ -94,8 +94,9 @@ static double orc_rint(double v) { return rint(v); }
 /* -------------------------------------------------------------- LayerNorm */
 
 /* LN of one row in double: mu = mean x, var = mean (x - mu)^2 (two passes),
- * u = (x - mu) / sqrt(var + eps_ln).  "LN(.) denotes LayerNorm" (H-BitLinear
- * matmul formula); no affine parameters are given, the model has no bias. */
+ * u = (x - mu) / sqrt(var + eps_ln).  The symbol LN of the H-BitLinear
+ * matrix-operation formula is LayerNorm; no affine parameters are given, the
+ * model has no bias. */
 void orc_layernorm_row(const double* x, int64_t K, double* u) {
   double s = 0.0;
   for (int64_t i = 0; i < K; ++i) s += x[i];
@@ -110,9 +111,10 @@ void orc_layernorm_row(const double* x, int64_t K, double* u) {
 /* LayerNorm backward of one row in double (no affine, eps 1e-5), the chain
  * rule through u = (x - mu) / sigma with mu and sigma functions of x:
  *   g_x = (g_u - mean(g_u) - u mean(g_u u)) / sigma
- * ("the straight-through estimator approximates the gradient ... the
- * Hadamard matrix's orthogonality transforms the gradient": everything before
- * the transform is ordinary backpropagation). */
+ * (the pages' training strategy: the straight-through estimator stands in
+ * for the quantizers' gradient and the orthogonal Hadamard matrix carries the
+ * gradient through the transform; everything before the transform is
+ * ordinary backpropagation). */
 void orc_ln_backward_row(const double* x, const double* gu, int64_t K, double* gx) {
   double sum = 0.0;
   for (int64_t i = 0; i < K; ++i) sum += x[i];
@@ -136,7 +138,7 @@ void orc_ln_backward_row(const double* x, const double* gu, int64_t K, double* g
 /* In-place unnormalised fast Walsh-Hadamard transform, natural (Sylvester)
  * order: H_1 = [1], H_2n = [[H_n, H_n], [H_n, -H_n]].  The recursion applied
  * bottom up: at span h every pair (j, j+h) in a block of 2h becomes
- * (a + b, a - b).  O(n log n) additions ("fast Hadamard transform"). */
+ * (a + b, a - b).  O(n log n) additions: the fast transform the pages name. */
 void orc_fht_unnormalized(double* v, int64_t n) {
   for (int64_t h = 1; h < n; h *= 2)
     for (int64_t i = 0; i < n; i += 2 * h)
@@ -242,7 +244,8 @@ int orc_fht_rows(const void* x, int dtype, int64_t M, int64_t K, double* t64, fl
 
 /* Per-token activation quantization of M rows of length K (any K >= 1).
  * bits = 4: absmean, codes in [-8, 7]; bits = 8: absmax, codes in [-128, 127].
- * ("for 8-bit and 4-bit activations, per-token absmax and absmean are used").
+ * (the pages: absmax per token for 8-bit activations, absmean per token for
+ * 4-bit ones).
  * codes: int8 [M][K] (unpacked); scales: float [M] (dequant factor per row).
  * Returns 0, or -1 on bad bits. */
 int orc_quant(const float* t, int64_t M, int64_t K, int bits, int8_t* codes, float* scales) {
@@ -285,7 +288,7 @@ int orc_quant(const float* t, int64_t M, int64_t K, int bits, int8_t* codes, flo
  * alpha = mean|W| (double sum, rounded once to float),
  * w = clip(rint(W / (alpha + eps)), -1, 1) computed as rint of the exact
  * product W * r with the float reciprocal r = 1/(alpha+eps).
- * ("per-tensor absmean quantizes the weights to {-1, 0, 1}") */
+ * (the pages: the weights go to {-1, 0, 1} by a per-tensor absmean) */
 void orc_ternary(const void* W, int dtype, int64_t N, int64_t K, int8_t* w, float* alpha) {
   fesetround(FE_TONEAREST);
   double s = 0.0;
@@ -421,7 +424,7 @@ int orc_forward_rows(const void* x, int dtype, int64_t M, int64_t K, const int64
 /* ------------------------------------------------------- low-bit QKV states */
 
 /* Post-RoPE QKV-state quantizer of the low-bit attention experiments (QbitAI
- * report / Xinzhiyuan article, "low-bit attention": the QKV heads are quantized
+ * report / Xinzhiyuan article, section on low-bit attention: the QKV heads are quantized
  * to unsigned integers by the absmax function, with no calibration data; a
  * 3-bit KV cache matches full precision).  Reading of the open steps: one head
  * vector of D values (one token, one head) at a time; gamma = max|x|; the
