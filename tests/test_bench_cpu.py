@@ -109,3 +109,19 @@ def test_clock_record_rejection():
     # no clock source: nothing to judge
     assert not bench.clocks_rejected({"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no clock source"],
                                       "samples": 0})
+
+
+def test_traffic_record_follows_its_sources(tmp_path, monkeypatch):
+    """DRAM traffic from the committed ncu record is reported only while the
+    kernel's sources hash to the digest recorded with it; a changed source (or
+    a missing entry) reports nothing."""
+    src = tmp_path / "k.cu"
+    src.write_text("// kernel v1\n")
+    (tmp_path / "profiles").mkdir()
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    rec = {"sources": ["k.cu"], "dram_bytes_per_launch": 12345, "source_sha256": bench.source_digest(["k.cu"])}
+    (tmp_path / "profiles" / "traffic.json").write_text(json.dumps({"k": rec}))
+    assert bench.measured_traffic("k") == 12345
+    assert bench.measured_traffic("other") is None
+    src.write_text("// kernel v2\n")
+    assert bench.measured_traffic("k") is None
