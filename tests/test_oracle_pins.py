@@ -143,6 +143,34 @@ def test_quant_int4_hand(orc):
     assert s[0] == f32(g["scale"])
 
 
+def _nearest_f32(fr):
+    """The float32 nearest to a rational number, ties to even (exact comparisons)."""
+    from fractions import Fraction
+    b = f32(float(fr))
+    cands = [np.nextafter(b, f32(-np.inf)), b, np.nextafter(b, f32(np.inf))]
+    dist = [abs(Fraction(float(c)) - fr) for c in cands]
+    best = min(dist)
+    ties = [c for c, d in zip(cands, dist) if d == best]
+    return next((c for c in ties if int(np.array(c, np.float32).view(np.uint32)) % 2 == 0), ties[0])
+
+
+def test_int4_scale_is_the_exactly_rounded_mean(orc):
+    """The absmean's reduction (a double sum of |t|, rounded once to float)
+    against the plain definition computed exactly: the mean of |t| as a
+    rational number rounded to the nearest float, then scale = beta / sqrt(7)
+    as one float division.  Rows with a wide spread of magnitudes, powers of
+    two K of the path up to 4096."""
+    from fractions import Fraction
+    rng = np.random.default_rng(11)
+    c = f32(math.sqrt(7.0))
+    for K in (64, 128, 256, 1024, 4096):
+        t = (rng.standard_normal((40, K)) * 10.0 ** rng.integers(-6, 4, (40, K))).astype(np.float32)
+        _, s = orc.quant(t, 4)
+        for i in range(t.shape[0]):
+            exact = sum(Fraction(float(v)) for v in np.abs(t[i])) / K
+            assert s[i] == _nearest_f32(exact) / c
+
+
 def test_quant_int4_saturation(orc):
     g = GOLD["int4_saturation"]
     q, _ = orc.quant(np.array(g["rows"], np.float32), 4)
