@@ -32,6 +32,12 @@ MUTANTS = [
     ("INT4 clip to 8", "const double hi = (bits == 4) ? 7.0 : 127.0;", "const double hi = (bits == 4) ? 8.0 : 127.0;"),
     ("missing quantizer eps", "volatile float den = stat + ORC_EPS_Q;", "volatile float den = stat;"),
     ("absmean over K-1", "stat = (float)(s / (double)K);", "stat = (float)(s / (double)(K - 1));"),
+    ("absmean summed in float", "double s = 0.0;                       /* beta = mean |t| */",
+     "float s = 0.0f;                       /* beta = mean |t| */"),
+    ("absmax over signed values", "for (int64_t i = 0; i < K; ++i) if (fabsf(r[i]) > g) g = fabsf(r[i]);",
+     "for (int64_t i = 0; i < K; ++i) if (r[i] > g) g = r[i];"),
+    ("codes from the float-rounded product t * r", "double q = orc_rint((double)r[i] * (double)rcp);",
+     "volatile float pr = r[i] * rcp; double q = orc_rint((double)pr);"),
     ("scale inverted", "volatile float sc = stat / c;", "volatile float sc = c / stat;"),
     ("alpha without abs", "for (int64_t i = 0; i < n; ++i) s += fabs(orc_load(W, dtype, i));",
      "for (int64_t i = 0; i < n; ++i) s += orc_load(W, dtype, i);"),

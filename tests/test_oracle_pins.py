@@ -217,6 +217,115 @@ def test_quant_round_half_to_even(orc, bits, target, want):
     assert q[0, 1] == want
 
 
+def _row_reciprocal(row, bits):
+    """r = fl(c / fl(stat + eps)) of one row, the statistic from its definition
+    (exact mean of |t| rounded to float, or max |t|)."""
+    from fractions import Fraction
+    c = f32(math.sqrt(7.0)) if bits == 4 else f32(127.0)
+    if bits == 4:
+        stat = _nearest_f32(sum(Fraction(float(v)) for v in np.abs(row)) / len(row))
+    else:
+        stat = f32(np.abs(row).max())
+    return f32(c / f32(stat + f32(1e-5)))
+
+
+def _near_ties(r, n, limit):
+    """Floats t just off (k + 1/2) / r whose product with r is not a half-integer
+    but rounds in float to one: rint of the exact product and rint of the
+    float-rounded product differ for them."""
+    from fractions import Fraction
+    out = []
+    for k in range(limit):
+        for sgn in (1.0, -1.0):
+            t0 = f32(sgn * (k + 0.5) / float(r))
+            for t in (np.nextafter(t0, f32(-np.inf)), t0, np.nextafter(t0, f32(np.inf))):
+                exact = Fraction(float(t)) * Fraction(float(r))
+                if abs(exact.denominator) != 2 and f32(t * r) == f32(sgn * (k + 0.5)):
+                    out.append(t)
+        if len(out) >= n:
+            break
+    return np.array(out[:n], np.float32)
+
+
+def _steer_int4_row(rest, R):
+    """Prepend to `rest` an element a (walked one ulp at a time) such that the
+    row's INT4 reciprocal fl(sqrt7 / fl(beta + eps)) is exactly R."""
+    c = f32(math.sqrt(7.0))
+    d0 = f32(c / R)
+    dens = [d for d in (np.nextafter(np.nextafter(d0, f32(-np.inf)), f32(-np.inf)), np.nextafter(d0, f32(-np.inf)),
+                        d0, np.nextafter(d0, f32(np.inf)), np.nextafter(np.nextafter(d0, f32(np.inf)), f32(np.inf)))
+            if f32(c / d) == R]
+    assert dens, "no denominator gives R"
+    den = dens[len(dens) // 2]
+    K = len(rest) + 1
+    a = f32(K * (float(den) - 1e-5) - float(np.abs(rest.astype(np.float64)).sum()))
+    for _ in range(2000):
+        row = np.concatenate([[a], rest]).astype(np.float32)
+        s = f32(_row_stat_int4(row) + f32(1e-5))
+        if s == den:
+            return row
+        a = np.nextafter(a, f32(-np.inf) if s > den else f32(np.inf))
+    raise RuntimeError("statistic not reached")
+
+
+def _row_stat_int4(row):
+    from fractions import Fraction
+    return _nearest_f32(sum(Fraction(float(v)) for v in np.abs(row)) / len(row))
+
+
+def _row_reciprocal(row, bits):
+    """r = fl(c / fl(stat + eps)) of one row, the statistic from its definition
+    (exact mean of |t| rounded to float, or max |t|)."""
+    c = f32(math.sqrt(7.0)) if bits == 4 else f32(127.0)
+    stat = _row_stat_int4(row) if bits == 4 else f32(np.abs(row).max())
+    return f32(c / f32(stat + f32(1e-5)))
+
+
+def _near_ties(r, limit):
+    """Floats t just off (k + 1/2) / r, k < limit, whose product with r is not a
+    half-integer but rounds in float to one: rint of the exact product and rint
+    of the float-rounded product differ for them."""
+    from fractions import Fraction
+    out = []
+    for k in range(limit):
+        for sgn in (1.0, -1.0):
+            t0 = f32(sgn * (k + 0.5) / float(r))
+            for t in (np.nextafter(t0, f32(-np.inf)), t0, np.nextafter(t0, f32(np.inf))):
+                exact = Fraction(float(t)) * Fraction(float(r))
+                if exact.denominator != 2 and f32(t * r) == f32(sgn * (k + 0.5)):
+                    out.append(t)
+    return np.array(out, np.float32)
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+def test_quant_rounds_the_exact_product(orc, bits):
+    """Codes are the nearest integer to the exact product t * r (ties to even),
+    not to its float rounding: rows planted with values whose product with the
+    row's r lies within half a float ulp of a half-integer."""
+    from fractions import Fraction
+    rng = np.random.default_rng(21 + bits)
+    base = (rng.standard_normal(255) * 0.5).astype(np.float32)
+    if bits == 8:
+        R = _row_reciprocal(np.concatenate([[10.0], base]).astype(np.float32), 8)
+        ties = _near_ties(R, 120)
+        row = np.concatenate([[10.0], ties, base[len(ties):]]).astype(np.float32)   # max |t| stays 10
+    else:
+        R = f32(3.25)
+        ties = _near_ties(R, 8)
+        row = _steer_int4_row(np.concatenate([ties, base[len(ties):]]).astype(np.float32), R)
+    r = _row_reciprocal(row, bits)
+    assert r == R and len(ties) >= 8
+    q, _ = orc.quant(row[None, :], bits)
+    lo, hi = (-8, 7) if bits == 4 else (-128, 127)
+    differ = 0
+    for i, t in enumerate(row):
+        exact = Fraction(float(t)) * Fraction(float(r))
+        want = min(hi, max(lo, round(exact)))     # Fraction rounds half to even
+        assert q[0, i] == want, (i, float(t))
+        differ += want != min(hi, max(lo, int(np.rint(f32(t * r)))))
+    assert differ >= 4
+
+
 @pytest.mark.parametrize("bits", [4, 8])
 def test_quant_code_ranges(orc, bits):
     rng = np.random.default_rng(bits)
