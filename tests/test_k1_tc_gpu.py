@@ -14,7 +14,7 @@ import numpy as np
 import pytest
 
 from helpers import check_codes_exact, check_t, to_device, to_host, unpack_nibbles
-from ternary_gemm_b200.inputs import WORKLOADS, f32_to_bf16_bits, make_x, make_x_rows, sample_rows
+from ternary_gemm_b200.inputs import WORKLOADS, f32_to_bf16_bits, make_w, make_x, make_x_rows, sample_rows
 
 pytestmark = pytest.mark.gpu
 
@@ -110,3 +110,62 @@ def test_tc_single_row_and_partial_tile(H, orc):
         codes, scales = H.hbl_fht_quant(xd, 4)
         qo, so = orc.quant(t, 4)
         check_codes_exact(unpack_nibbles(to_host(codes), K), to_host(scales), qo, so)
+
+
+# Rows whose transform is one dominant element: x = a * (Walsh row j) + noise,
+# so t is a spike at j plus noise.  With the spike holding most of the row's L1
+# mass, |t r| reaches about sqrt(7) K / (1 + eps sqrt(K)): at K >= 16384 codes
+# far beyond the int16 range, where the widened INT4 mode clips on 32-bit values
+# instead of packed 16-bit halves; the noise levels take ||t|| r across the
+# bound (3e4) that selects between the two.
+SPIKE_NOISE = [0.0, 0.0022, 0.003, 0.008, 0.012, 0.014, 0.02, 0.05]
+
+
+def spiky_rows(K, M, seed):
+    rng = np.random.default_rng(seed)
+    i = np.arange(K, dtype=np.int64)
+    x = np.empty((M, K), np.float32)
+    for m in range(M):
+        j = int(rng.integers(1, K))
+        walsh = np.where(np.bitwise_count(i & j) % 2 == 0, 1.0, -1.0)
+        a = (1.0, -3.5, 0.25, 2.0)[m % 4]
+        x[m] = a * walsh + a * SPIKE_NOISE[m % len(SPIKE_NOISE)] * rng.standard_normal(K)
+    x[0] = 0.0
+    x[0, ::2] = 1.0            # alternating row: a spike at K / 2 with no rounding noise
+    x[3] += 7.0                # a mean for LayerNorm to remove
+    return f32_to_bf16_bits(x)
+
+
+@pytest.mark.parametrize("K", [1024, 16384, 32768])
+def test_tc_spiky_rows_codes_and_forward(H, orc, K):
+    """Packed and int8-widened codes, INT4 and INT8, bit-exact on the kernel's
+    own t for rows with codes far outside the int16 range; the forward through
+    the int8-widened GEMM is then the oracle's GEMM + dequant of those codes."""
+    import torch
+    M = 8 * 37
+    x = spiky_rows(K, M, K + 5)
+    xd = to_device(x)
+    t = to_host(H.hbl_debug_ln_fht(xd))
+    if K >= 16384:
+        bound = np.abs(t).max(axis=1) * np.sqrt(7.0) / np.abs(t.astype(np.float64)).mean(axis=1)
+        assert bound.max() > 40000 and bound.min() < 30000     # both clip forms are reached
+    ref = {}
+    for bits in (4, 8):
+        qo, so = orc.quant(t, bits)
+        ref[bits] = (qo, so)
+        codes, scales = H.hbl_fht_quant(xd, bits)
+        q = unpack_nibbles(to_host(codes), K) if bits == 4 else to_host(codes)
+        check_codes_exact(q, to_host(scales), qo, so)
+        codes_i8, scales_i8 = H.hbl_fht_quant_i8(xd, bits)
+        check_codes_exact(to_host(codes_i8), to_host(scales_i8), qo, so)
+    wl = WORKLOADS["sweep"].with_shape(M, K, 256)
+    W = make_w(wl)
+    packed, alpha = H.hbl_pack_ternary(to_device(W))
+    w, a = orc.ternary(W)
+    rows = np.arange(16)
+    for bits in (4, 8):
+        y = H.hbl_forward(xd, packed, alpha, 256, bits)
+        torch.cuda.synchronize()
+        qo, so = ref[bits]
+        y_exact = orc.dequant(orc.gemm_i32(qo[rows], w), so[rows], a)
+        assert np.array_equal(to_host(y)[rows], orc.round_to_bf16(y_exact))
