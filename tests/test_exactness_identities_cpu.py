@@ -14,7 +14,11 @@ with plain integer and double arithmetic (no GPU, no oracle):
   acc_0 + acc_1 / 4 + acc_2 / 16 + acc_3 / 64 is the plain dot product;
 * the 4 x 4 byte transpose built from byte permutes (selector semantics of
   prmt / __byte_perm: result byte i = input byte (selector nibble i & 7) of the
-  pair (a, b) seen as bytes 0..7).
+  pair (a, b) seen as bytes 0..7);
+* the codes: one fused multiply-add fl(t r + 1.5 * 2^23) holds rint of the exact
+  product t r in its low bits; clipping those bits clips the code; the packed
+  16-bit clip is exact only below 2^15, and the row guard that selects it
+  (ss * cr * cr < 9e8) keeps every code there.
 """
 import struct
 
@@ -108,3 +112,103 @@ def test_byte_transpose_from_permutes():
         for f in range(4):
             for j in range(4):
                 assert (out[f] >> (8 * j)) & 0xFF == (w[j] >> (8 * f)) & 0xFF
+
+
+# ------------------------------------------------ codes from one fused multiply-add
+
+MAGIC = 12582912.0          # 1.5 * 2^23
+MAGIC_BITS = 0x4B400000
+
+
+def _nearest_f32_bits(v) -> int:
+    """Bits of the float32 nearest to the rational v (ties to even): the result
+    of one fused multiply-add whose exact value is v (v > 0 here)."""
+    from fractions import Fraction
+    v = Fraction(v)
+    e = v.numerator.bit_length() - v.denominator.bit_length()
+    if Fraction(2) ** e > v:
+        e -= 1
+    ulp = Fraction(2) ** (e - 23)
+    q = round(v / ulp)                       # Fraction rounds half to even
+    return int(np.array(float(q * ulp), np.float32).view(np.uint32))
+
+
+def _products():
+    """(t, r) float pairs: random ones with |t r| up to 2^22, exact half-integer
+    products and products within half a float ulp of a half-integer."""
+    from fractions import Fraction
+    rng = np.random.default_rng(5)
+    out = []
+    for _ in range(3000):
+        r = np.float32(2.0 ** rng.uniform(-10, 10))
+        t = np.float32(rng.uniform(-1, 1) * 2.0 ** rng.uniform(-20, 22) / float(r))
+        if abs(Fraction(float(t)) * Fraction(float(r))) < 2 ** 22:
+            out.append((t, r))
+    for k in range(-300, 300):
+        out.append((np.float32((k + 0.5) / 4.0), np.float32(4.0)))        # exact ties
+        r = np.float32(3.25)
+        t0 = np.float32((k + 0.5) / float(r))
+        for t in (np.nextafter(t0, np.float32(-np.inf)), t0, np.nextafter(t0, np.float32(np.inf))):
+            out.append((t, r))
+    return out
+
+
+def test_magic_fma_rounds_the_exact_product():
+    """fl(t r + 1.5 * 2^23), one rounding, has the bits MAGIC_BITS + rint(t r)
+    (rint of the exact product, half to even) whenever |t r| < 2^22."""
+    from fractions import Fraction
+    assert int(np.array(MAGIC, np.float32).view(np.uint32)) == MAGIC_BITS
+    for t, r in _products():
+        p = Fraction(float(t)) * Fraction(float(r))
+        assert _nearest_f32_bits(p + Fraction(MAGIC)) - MAGIC_BITS == round(p), (float(t), float(r))
+
+
+def _clip(n, lo, hi):
+    return max(lo, min(hi, n))
+
+
+def test_clip_on_the_magic_bits():
+    """Clipping the magic sum's bits to [MAGIC_BITS - 8, MAGIC_BITS + 7] clips the
+    code to the INT4 range, and the low byte is then the code as an int8."""
+    for code in range(-(1 << 22) + 1, 1 << 22, 997):
+        m = _clip(MAGIC_BITS + code, MAGIC_BITS - 8, MAGIC_BITS + 7)
+        assert np.array([m & 0xFF], np.uint8).view(np.int8)[0] == _clip(code, -8, 7)
+
+
+def test_packed_16_bit_clip_needs_codes_below_2_15():
+    """The low 16 bits of the magic sum's bits, read as int16 and clamped to
+    [-8, 7], are the clipped code exactly when |code| < 2^15 (MAGIC_BITS has a
+    zero low half); above that they can wrap into the range, so the kernel
+    takes this form only for rows it has bounded below 2^15."""
+    def s16_clip(code):
+        low = np.array([(MAGIC_BITS + code) & 0xFFFF], np.uint16).view(np.int16)[0]
+        return _clip(int(low), -8, 7)
+    assert MAGIC_BITS & 0xFFFF == 0
+    for code in range(-(1 << 15) + 1, 1 << 15):
+        assert s16_clip(code) == _clip(code, -8, 7)
+    assert s16_clip(65536 + 3) == 3 and _clip(65536 + 3, -8, 7) == 7     # a wrapped code
+
+
+def test_row_guard_of_the_packed_clip():
+    """The row test ss * cr * cr < 9e8 (float, left to right), with ss the float
+    sum of y^2 and cr = fl(cmul r), bounds every |t r| (t = fl(cmul y)) below
+    3.01e4 < 2^15 even when ss is summed in sequence (relative error below
+    K 2^-24 = 2e-3 at K = 32768): rows whose energy sits in one element, where
+    max |t r| comes closest to ||t|| r, scanned across the guard's threshold."""
+    rng = np.random.default_rng(6)
+    f32 = np.float32
+    hit = 0
+    for K in (1024, 16384, 32768):
+        for _ in range(60):
+            y = (rng.standard_normal(K) * 10.0 ** rng.uniform(-4, -1)).astype(np.float32)
+            y[rng.integers(K)] = f32(rng.choice([-1.0, 1.0]) * 10.0 ** rng.uniform(-1, 2))
+            cmul = f32(10.0 ** rng.uniform(-3, 0))
+            t = (cmul * y).astype(np.float32)
+            # r chosen so that ss * cr^2 lands near the threshold
+            ss = np.add.accumulate((y * y).astype(np.float32), dtype=np.float32)[-1]
+            r = f32(np.sqrt(9e8 / float(ss)) / float(cmul) * rng.uniform(0.98, 1.02))
+            cr = f32(cmul * r)
+            if f32(f32(ss * cr) * cr) < f32(9.0e8):
+                hit += 1
+                assert np.max(np.abs(t.astype(np.float64) * float(r))) < 3.01e4
+    assert hit > 50
