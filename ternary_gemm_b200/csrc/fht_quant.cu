@@ -23,8 +23,12 @@
 //           stores.
 // Shared memory uses an XOR swizzle of index bits 5..8 into bits 2..4; it is
 // linear over GF(2), so an address splits into a per-thread part (eight
-// precomputed bases) and a compile-time offset, and it keeps the accesses of
-// all three passes free of bank conflicts.  Butterflies, scaling and the
+// precomputed bases) and a compile-time offset.  The accesses of all three
+// passes are free of bank conflicts for K = 512, 1024 and K >= 4096; pass 2
+// at K = 2048 is 2-way (its threads differ in index bits 4, 5 and 8, and bit
+// 8 folds onto bit 4), and at K = 64 .. 256 rows of a quarter-warp share
+// banks through the row padding (4-way at 64, 2-way at 128 and 256).
+// Butterflies, scaling and the
 // quantizer's products run as paired f32x2 instructions (one issue slot for
 // two IEEE float operations).
 //
