@@ -23,7 +23,9 @@
 // The other 15 warps consume the stages: lane l owns row l of the group and
 // keeps its int32 sums in registers across K; the warps split the stage's
 // 16-byte pieces (64 codes each).  For a piece, every lane reads its row's 16
-// bytes (the swizzle spreads the 32 rows over all banks), splits each word of
+// bytes (for K >= 512 the swizzle spreads the rows of a quarter-warp over all
+// banks; the narrower unswizzled boxes of K = 128 and 256 read 2- and 4-way
+// conflicted), splits each word of
 // 16 codes into four signed-byte planes (tern_planes: 10 integer operations,
 // no widening to one byte per code) and takes dp4a products with the M code
 // rows, which sit in shared memory in 16-byte units ordered (row, 16-code
