@@ -179,10 +179,11 @@ hbl_status hbl_debug_norm(const void* x, hbl_dtype xt, int64_t M, int64_t K, hbl
 /* ---------------------------------------------------------------- forward stages
  * hbl_forward is made of these calls on slices of its workspace:
  * hbl_fht_quant_i8, hbl_widen_ternary and hbl_gemm_dequant.  For
- * decode-sized batches (M <= 4 and M * K <= 65536) it runs instead one kernel
- * that does what hbl_fht_quant_i8 then hbl_gemv_ternary_dequant do, with the
- * same arithmetic (y bit-identical), keeping the codes in shared memory and
- * leaving the workspace untouched.  hbl_fht_quant then hbl_gemm_tern_dequant is another
+ * decode-sized batches (M <= 4 and M * K <= 65536) it runs hbl_fht_quant_i8
+ * then hbl_gemv_ternary_dequant instead, and when M * K <= 16384 one kernel
+ * that does what those two do, with the same arithmetic (y bit-identical),
+ * keeping the codes in shared memory and leaving the workspace untouched.
+ * hbl_fht_quant then hbl_gemm_tern_dequant is another
  * route to the identical y that needs no int8 buffers (it measured slower, so
  * hbl_forward does not take it).  They are public so that callers can overlap
  * stages or time each kernel on their own stream. */
