@@ -42,6 +42,9 @@ MUTANTS = [
     ("alpha without abs", "for (int64_t i = 0; i < n; ++i) s += fabs(orc_load(W, dtype, i));",
      "for (int64_t i = 0; i < n; ++i) s += orc_load(W, dtype, i);"),
     ("ternary clip to 2", "if (q > 1.0) q = 1.0;", "if (q > 2.0) q = 2.0;"),
+    ("ternary codes from the float-rounded product W * r",
+     "double q = orc_rint(orc_load(W, dtype, i) * (double)rcp);   /* exact product, one rounding */",
+     "volatile float pr = (float)orc_load(W, dtype, i) * rcp; double q = orc_rint((double)pr);"),
     ("transposed GEMM operand", "s += (int64_t)A[m * K + k] * (int64_t)B[n * K + k];",
      "s += (int64_t)A[m * K + k] * (int64_t)B[k * N + n];"),
     ("RMSNorm without the square", "for (int64_t i = 0; i < K; ++i) s += x[i] * x[i];",

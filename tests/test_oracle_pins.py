@@ -217,40 +217,10 @@ def test_quant_round_half_to_even(orc, bits, target, want):
     assert q[0, 1] == want
 
 
-def _row_reciprocal(row, bits):
-    """r = fl(c / fl(stat + eps)) of one row, the statistic from its definition
-    (exact mean of |t| rounded to float, or max |t|)."""
-    from fractions import Fraction
-    c = f32(math.sqrt(7.0)) if bits == 4 else f32(127.0)
-    if bits == 4:
-        stat = _nearest_f32(sum(Fraction(float(v)) for v in np.abs(row)) / len(row))
-    else:
-        stat = f32(np.abs(row).max())
-    return f32(c / f32(stat + f32(1e-5)))
-
-
-def _near_ties(r, n, limit):
-    """Floats t just off (k + 1/2) / r whose product with r is not a half-integer
-    but rounds in float to one: rint of the exact product and rint of the
-    float-rounded product differ for them."""
-    from fractions import Fraction
-    out = []
-    for k in range(limit):
-        for sgn in (1.0, -1.0):
-            t0 = f32(sgn * (k + 0.5) / float(r))
-            for t in (np.nextafter(t0, f32(-np.inf)), t0, np.nextafter(t0, f32(np.inf))):
-                exact = Fraction(float(t)) * Fraction(float(r))
-                if abs(exact.denominator) != 2 and f32(t * r) == f32(sgn * (k + 0.5)):
-                    out.append(t)
-        if len(out) >= n:
-            break
-    return np.array(out[:n], np.float32)
-
-
-def _steer_int4_row(rest, R):
+def _steer_mean_row(rest, R, c):
     """Prepend to `rest` an element a (walked one ulp at a time) such that the
-    row's INT4 reciprocal fl(sqrt7 / fl(beta + eps)) is exactly R."""
-    c = f32(math.sqrt(7.0))
+    reciprocal fl(c / fl(mean|.| + eps)) of the whole array, its mean of
+    absolute values rounded once to float, is exactly R."""
     d0 = f32(c / R)
     dens = [d for d in (np.nextafter(np.nextafter(d0, f32(-np.inf)), f32(-np.inf)), np.nextafter(d0, f32(-np.inf)),
                         d0, np.nextafter(d0, f32(np.inf)), np.nextafter(np.nextafter(d0, f32(np.inf)), f32(np.inf)))
@@ -312,7 +282,7 @@ def test_quant_rounds_the_exact_product(orc, bits):
     else:
         R = f32(3.25)
         ties = _near_ties(R, 8)
-        row = _steer_int4_row(np.concatenate([ties, base[len(ties):]]).astype(np.float32), R)
+        row = _steer_mean_row(np.concatenate([ties, base[len(ties):]]).astype(np.float32), R, f32(math.sqrt(7.0)))
     r = _row_reciprocal(row, bits)
     assert r == R and len(ties) >= 8
     q, _ = orc.quant(row[None, :], bits)
@@ -379,6 +349,38 @@ def test_ternary_zero_fraction_gaussian(orc):
     assert set(np.unique(w)) == {-1, 0, 1}
     assert abs(a - 0.02 * math.sqrt(2 / math.pi)) < 2e-4
     assert abs(np.mean(w == 0) - 0.3101) < 0.005
+
+
+def test_ternary_rounds_the_exact_product(orc):
+    """Ternary codes are clip(rint(W r), -1, 1) of the exact product W r, r =
+    fl(1 / fl(alpha + eps)) with alpha the mean of |W| rounded once to float:
+    tensors steered to a chosen r and planted with weights whose product with it
+    lies within half a float ulp of +-1/2."""
+    from fractions import Fraction
+    rng = np.random.default_rng(31)
+    differ = used = 0
+    for i in range(400):
+        R = f32(20.0 + 0.37 * i)
+        d0 = f32(f32(1.0) / R)
+        reachable = any(f32(f32(1.0) / d) == R
+                        for d in (np.nextafter(d0, f32(-np.inf)), d0, np.nextafter(d0, f32(np.inf))))
+        ties = _near_ties(R, 1)
+        if not reachable or len(ties) == 0:
+            continue
+        used += 1
+        if used > 6:
+            break
+        base = (rng.standard_normal(255) * 0.02).astype(np.float32)
+        W = _steer_mean_row(np.concatenate([ties, base[len(ties):]]).astype(np.float32), R, f32(1.0)).reshape(4, 64)
+        alpha = _row_stat_int4(W.ravel())
+        assert f32(f32(1.0) / f32(alpha + f32(1e-5))) == R
+        w, a = orc.ternary(W)
+        assert a == alpha
+        for v, q in zip(W.ravel(), w.ravel()):
+            want = min(1, max(-1, round(Fraction(float(v)) * Fraction(float(R)))))
+            assert q == want, float(v)
+            differ += want != min(1, max(-1, int(np.rint(f32(v * R)))))
+    assert differ >= 3
 
 
 def test_ternary_zero_weight(orc):
