@@ -50,10 +50,30 @@ MUTANTS = [
     ("RMSNorm without the square", "for (int64_t i = 0; i < K; ++i) s += x[i] * x[i];",
      "for (int64_t i = 0; i < K; ++i) s += x[i];"),
     ("dequant without alpha", "volatile float sa = scales[m] * alpha;", "volatile float sa = scales[m];"),
+    ("dequant product order (acc * scale) * alpha", "      volatile float v = (float)acc[m * N + n] * sa;",
+     "      volatile float v0 = (float)acc[m * N + n] * scales[m]; volatile float v = v0 * alpha;"),
     ("nibbles swapped", "out[m * (K / 2) + j] = (uint8_t)(lo | (hi << 4));",
      "out[m * (K / 2) + j] = (uint8_t)(hi | (lo << 4));"),
     ("ternary -1 encoded as 10", "unsigned f = (v == 0) ? 0u : (v == 1 ? 1u : 3u);",
      "unsigned f = (v == 0) ? 0u : (v == 1 ? 1u : 2u);"),
+    ("Hadamard entry from popcount(i | j)",
+     "return (__builtin_popcountll((unsigned long long)(i & j)) & 1) ? -1 : 1;",
+     "return (__builtin_popcountll((unsigned long long)(i | j)) & 1) ? -1 : 1;"),
+    ("RMSNorm without eps", "double inv = 1.0 / sqrt(s / (double)K + ORC_EPS_LN);",
+     "double inv = 1.0 / sqrt(s / (double)K);"),
+    ("LayerNorm eps 1e-6", "#define ORC_EPS_LN 1e-5", "#define ORC_EPS_LN 1e-6"),
+    ("LayerNorm divides by the variance", "double inv = 1.0 / sqrt(v + ORC_EPS_LN);",
+     "double inv = 1.0 / (v + ORC_EPS_LN);"),
+    ("quantizer eps 1e-6", "#define ORC_EPS_Q 1e-5f", "#define ORC_EPS_Q 1e-6f"),
+    ("absmean of signed t", "for (int64_t i = 0; i < K; ++i) s += (double)fabsf(r[i]);",
+     "for (int64_t i = 0; i < K; ++i) s += (double)r[i];"),
+    ("INT4 rate without sqrt(7)", "volatile float rcp = c / den;           /* one float division per row */",
+     "volatile float rcp = 1.0f / den;"),
+    ("scale by a reciprocal multiply", "volatile float sc = stat / c;", "volatile float sc = stat * (1.0f / c);"),
+    ("INT4 low clip at -7", "const double lo = (bits == 4) ? -8.0 : -128.0;",
+     "const double lo = (bits == 4) ? -7.0 : -128.0;"),
+    ("INT8 clip at 126", "const double hi = (bits == 4) ? 7.0 : 127.0;", "const double hi = (bits == 4) ? 7.0 : 126.0;"),
+    ("ternary without eps", "volatile float den = a + ORC_EPS_Q;", "volatile float den = a;"),
     # the backward pass (tests/test_oracle_backward_pins.py)
     ("LayerNorm backward without the mean term", "gx[i] = (gu[i] - mg - (x[i] - mu) * inv * mgu) * inv;",
      "gx[i] = (gu[i] - (x[i] - mu) * inv * mgu) * inv;"),

@@ -420,6 +420,33 @@ def test_dequant_exact(orc):
     assert y.tolist() == [[0.375, -0.5], [3.5, 0.0]]
 
 
+def test_dequant_rounding_points(orc):
+    """y = fl(fl(acc) * fl(scale * alpha)): the int32 sum rounded to float
+    (nearest even, above 2^24 too), the row's factor scale * alpha rounded once,
+    then one rounded product; written out in exact rationals.  The rows mix
+    sums beyond 2^24 with factors where the other product order rounds
+    differently."""
+    from fractions import Fraction
+    rng = np.random.default_rng(51)
+    M, N = 64, 64
+    acc = rng.integers(-(1 << 31), (1 << 31) - 1, (M, N), dtype=np.int64)
+    acc[:, :16] = rng.integers(-(1 << 20), 1 << 20, (M, 16))
+    acc = acc.astype(np.int32)
+    scales = (rng.random(M) * 10.0 ** rng.integers(-6, 0, M)).astype(np.float32)
+    alpha = f32(0.0137)
+    y = orc.dequant(acc, scales, alpha)
+    other = 0
+    for m in range(M):
+        fa = _nearest_f32(Fraction(float(scales[m])) * Fraction(float(alpha)))
+        for n in range(N):
+            a = _nearest_f32(Fraction(int(acc[m, n])))
+            want = _nearest_f32(Fraction(float(a)) * Fraction(float(fa)))
+            assert y[m, n] == want, (m, n)
+            other += want != _nearest_f32(Fraction(float(_nearest_f32(Fraction(float(a)) * Fraction(float(scales[m])))))
+                                          * Fraction(float(alpha)))
+    assert other >= 50
+
+
 # ----------------------------------------------------------------- packing
 
 def test_pack_int4_golden_and_roundtrip(orc):
