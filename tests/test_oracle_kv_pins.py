@@ -2,8 +2,10 @@
 by absmax; the reading of the open steps is in the oracle's docstring): the
 hand-worked examples in tests/golden/hand_examples.json, nearest-level
 optimality against brute force over all 2^b levels, the code range, the
-absmax elements landing on the end levels, and the mirror symmetry of the
-map.  CPU only."""
+absmax elements landing on the end levels, the mirror symmetry of the
+map, and its rounding points (x r and + L/2 each rounded to float, then ties to
+even) on planted values where any other order or rounding gives another code.
+CPU only."""
 import json
 import os
 
@@ -80,3 +82,62 @@ def test_kv_dequant_error_bound_and_end_levels(orc, bits):
     for m in range(x.shape[0]):
         i = int(np.argmax(np.abs(x[m])))
         assert xr[m, i] == np.float64(x[m, i])
+
+
+def _kv_planted(bits, g=1.0, spread=64):
+    """Values x whose code under the reading's float steps, rint(fl(fl(x r) + L/2))
+    with ties to even, differs from a rounding of the exact x r + L/2, from the
+    fused fl(x r + L/2), or from rounding half away from zero, for a head whose
+    max |x| is g.  Returns (x values, r, the three counts of differences)."""
+    from fractions import Fraction
+    f32 = np.float32
+    L = f32((1 << bits) - 1)
+    half = f32(0.5) * L
+    r = f32(L / f32(f32(2.0) * f32(f32(g) + f32(1e-5))))
+    picked, n_exact, n_fused, n_away = [], 0, 0, 0
+    for k in range(int(L)):
+        x0 = f32((k + 0.5 - float(half)) / float(r))
+        for d in range(-spread, spread + 1):
+            x = f32(x0 + d * np.spacing(max(abs(x0), f32(1e-30))))
+            if abs(x) >= g:
+                continue
+            u = f32(f32(x * r) + half)
+            q = int(np.rint(u))
+            ex = Fraction(float(x)) * Fraction(float(r)) + Fraction(float(half))
+            fu = float(np.float32(float(ex)))                  # double first: checked below against exact
+            if abs(Fraction(fu) - ex) > abs(Fraction(float(np.nextafter(f32(fu), f32(np.inf)))) - ex) or \
+               abs(Fraction(fu) - ex) > abs(Fraction(float(np.nextafter(f32(fu), f32(-np.inf)))) - ex):
+                continue                                       # skip the rare double-rounding case
+            e_q, f_q = round(ex), int(np.rint(f32(fu)))
+            a_q = int(np.floor(float(u) + 0.5))
+            if e_q != q or f_q != q or a_q != q:
+                picked.append(x)
+                n_exact += e_q != q
+                n_fused += f_q != q
+                n_away += a_q != q
+    return np.array(picked, np.float32), r, (n_exact, n_fused, n_away)
+
+
+@pytest.mark.parametrize("bits", [3, 8])
+def test_kv_rounding_points(orc, bits):
+    """Codes follow the reading's rounding points exactly: x r rounded to float,
+    plus L/2 rounded to float, then rint with ties to even, clipped to [0, L];
+    heads planted with values where rounding the exact x r + L/2, the fused
+    x r + L/2, or rounding half away from zero would give another code."""
+    f32 = np.float32
+    xs, r, counts = _kv_planted(bits)
+    assert min(counts) >= 1, counts
+    L = (1 << bits) - 1
+    D = 128
+    rows = []
+    for i in range(0, len(xs), D - 1):
+        row = np.zeros(D, np.float32)
+        row[0] = 1.0                                           # max |x| of every head
+        chunk = xs[i:i + D - 1]
+        row[1:1 + len(chunk)] = chunk
+        rows.append(row)
+    x = np.stack(rows)
+    codes, scales = orc.kv_quant(x, bits)
+    assert np.all(scales == f32(1.0))
+    want = np.clip(np.rint(((x * r).astype(np.float32) + f32(0.5) * f32(L)).astype(np.float32)), 0, L)
+    assert np.array_equal(codes.astype(np.int64), want.astype(np.int64))

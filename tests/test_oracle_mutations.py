@@ -88,6 +88,14 @@ MUTANTS = [
     ("KV absmax without abs", "float a = fabsf((float)orc_load(x, dtype, m * D + i));",
      "float a = (float)orc_load(x, dtype, m * D + i);"),
     ("KV 2^b levels off by one", "const float L = (float)((1 << bits) - 1);", "const float L = (float)(1 << bits);"),
+    ("KV rounding half away from zero", "      double q = orc_rint((double)u);", "      double q = round((double)u);"),
+    ("KV code from the exact x r + L/2",
+     "      volatile float t = (float)orc_load(x, dtype, m * D + i) * r;\n      volatile float u = t + half;\n"
+     "      double q = orc_rint((double)u);",
+     "      double q = orc_rint((double)(float)orc_load(x, dtype, m * D + i) * (double)r + (double)half);"),
+    ("KV fused x r + L/2",
+     "      volatile float t = (float)orc_load(x, dtype, m * D + i) * r;\n      volatile float u = t + half;",
+     "      volatile float u = fmaf((float)orc_load(x, dtype, m * D + i), r, half);"),
 ]
 
 
