@@ -1,5 +1,6 @@
 """Near ties on the GPU: the quantizer (hbl_quant_from_f32, the arithmetic every
-fused quantizer shares) and the ternary packing (hbl_pack_ternary) on inputs
+fused quantizer shares), the ternary packing (hbl_pack_ternary) and the
+QKV-state quantizer (hbl_kv_quant) on inputs
 planted with values whose product with the row's (or tensor's) reciprocal r
 lies within half a float ulp of a rounding boundary, so that rint of the exact
 product and rint of its float rounding differ.  Codes, scales and alpha must be
@@ -11,6 +12,7 @@ import numpy as np
 import pytest
 
 from helpers import check_codes_exact, to_device, to_host, unpack_nibbles
+from test_oracle_kv_pins import _kv_planted
 from test_oracle_pins import _near_ties, _row_reciprocal, _steer_mean_row
 
 pytestmark = pytest.mark.gpu
@@ -78,3 +80,24 @@ def test_ternary_pack_near_ties(H, orc):
         assert to_host(alpha)[0] == a
         assert np.array_equal(to_host(packed), orc.pack_ternary(w))
     assert used == 4
+
+
+@pytest.mark.parametrize("bits", [3, 8])
+def test_kv_quant_rounding_points(H, orc, bits):
+    """Heads planted with values where rounding the exact x r + L/2, fusing the
+    two steps, or rounding half away from zero would change the code."""
+    xs, _, counts = _kv_planted(bits)
+    assert min(counts) >= 1
+    D = 128
+    rows = []
+    for i in range(0, len(xs), D - 1):
+        row = np.zeros(D, np.float32)
+        row[0] = 1.0
+        chunk = xs[i:i + D - 1]
+        row[1:1 + len(chunk)] = chunk
+        rows.append(row)
+    x = np.stack(rows)
+    codes, scales = H.hbl_kv_quant(to_device(x), bits)
+    c_o, s_o = orc.kv_quant(x, bits)
+    assert np.array_equal(to_host(codes), c_o)
+    assert np.array_equal(to_host(scales), s_o)
