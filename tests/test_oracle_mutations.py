@@ -83,6 +83,11 @@ MUTANTS = [
      "gx[i] = (gu[i] - mg - (x[i] - mu) * inv * mgu);"),
     ("LayerNorm backward unbiased variance", "const double var = ss / (double)K;",
      "const double var = ss / (double)(K - 1);"),
+    ("LayerNorm backward mean term over K - 1", "  mg /= (double)K;", "  mg /= (double)(K - 1);"),
+    ("LayerNorm backward projection on x - mu", "    mgu += gu[i] * (x[i] - mu) * inv;",
+     "    mgu += gu[i] * (x[i] - mu);"),
+    ("LayerNorm backward without eps", "const double inv = 1.0 / sqrt(var + ORC_EPS_LN); /* 1 / sigma */",
+     "const double inv = 1.0 / sqrt(var); /* 1 / sigma */"),
     # the QKV-state quantizer (tests/test_oracle_kv_pins.py)
     ("KV levels without the offset", "volatile float u = t + half;", "volatile float u = t;"),
     ("KV absmax without abs", "float a = fabsf((float)orc_load(x, dtype, m * D + i));",
@@ -107,6 +112,9 @@ PY_MUTANTS = [
      "g_u = np.stack([fht_unnormalized(r) for r in g_t])"),
     ("backward weight columns reversed", "g_t = float(alpha) * (gy @ np.asarray(w, dtype=np.float64))",
      "g_t = float(alpha) * (gy @ np.asarray(w, dtype=np.float64)[:, ::-1])"),
+    ("backward rows paired with the wrong x",
+     "g_x = np.stack([ln_backward_row(xv[m], g_u[i]) for i, m in enumerate(rows)])",
+     "g_x = np.stack([ln_backward_row(xv[m], g_u[::-1][i]) for i, m in enumerate(rows)])"),
     ("weight gradient without the scales",
      "a = np.asarray(codes, dtype=np.float64) * np.asarray(scales, dtype=np.float64)[:, None]",
      "a = np.asarray(codes, dtype=np.float64)"),
