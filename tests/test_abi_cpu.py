@@ -1,5 +1,6 @@
 """The C ABI without a GPU: the library builds, loads, exports every symbol the
-header declares, answers size queries, and rejects bad arguments on the host
+header declares with the argument and return types the binding uses, answers
+size queries, and rejects bad arguments on the host
 before any launch (every call here fails validation, so nothing reaches CUDA).
 """
 import ctypes
@@ -29,6 +30,39 @@ def test_exports_every_declared_symbol(L):
     out = os.popen("nm -D --defined-only %s" % hbl.LIB_PATH).read()
     exported = set(re.findall(r"\bT (hbl_[a-z0-9_]+)\b", out))
     assert exported == set(names)
+
+
+def _ctype_of(decl: str):
+    """ctypes class for one C declaration (a parameter with its name, or a
+    return type): pointers and cudaStream_t are void pointers, char pointers
+    C strings, the enums int."""
+    d = " ".join(decl.replace("*", " * ").split())
+    if d in ("const char *",):
+        return ctypes.c_char_p
+    if "*" in d or d.split()[0] == "cudaStream_t":
+        return ctypes.c_void_p
+    base = [w for w in d.split() if w != "const"][0]
+    return {"int64_t": ctypes.c_int64, "int": ctypes.c_int, "hbl_dtype": ctypes.c_int, "hbl_norm": ctypes.c_int,
+            "hbl_status": ctypes.c_int, "size_t": ctypes.c_size_t, "uint64_t": ctypes.c_uint64}[base]
+
+
+def test_binding_signatures_match_the_header(L):
+    """Every prototype of include/hbl.h against the binding's ctypes argtypes and
+    restype, parameter by parameter (a drift would pass wrong arguments only at
+    run time on a GPU)."""
+    text = re.sub(r"/\*.*?\*/", "", open(os.path.join(ROOT, "include", "hbl.h")).read(), flags=re.S)
+    protos = re.findall(r"([A-Za-z_][\w \t\*]*?)\b(hbl_[a-z0-9_]+)\s*\(([^;{)]*)\)\s*;", text)
+    seen = set()
+    for ret, name, params in protos:
+        params = " ".join(params.split())
+        args = [] if params in ("", "void") else [a.strip() for a in params.split(",")]
+        want = [_ctype_of(re.sub(r"\b\w+$", "", a).strip()) for a in args]
+        fn = getattr(L, name)
+        assert fn.argtypes is not None, name
+        assert list(fn.argtypes) == want, (name, fn.argtypes, want)
+        assert fn.restype == _ctype_of(ret.strip()), (name, fn.restype, ret)
+        seen.add(name)
+    assert seen == set(hbl.declared_symbols())
 
 
 def test_size_queries(L):
