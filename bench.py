@@ -437,40 +437,26 @@ def measure_int8_peak(torch, dev, reps=10):
                    % (M, K, N, reps)}
 
 
-def packed_route(M, bits):
-    """hbl_forward's route through packed codes and the packed-operand GEMM: not taken
-    (measured slower than the int8-operand GEMM at every size)."""
-    return False
-
-
 def stage_times(torch, hbl, x, packed, alpha, N, bits, y, stream, n):
     """Mean seconds per launch of the forward's stages, through the stage entry points
-    (the same kernels hbl_forward runs): the quantizer, the weight widening (zero on the
-    packed route, which has none) and the GEMM."""
+    (the same kernels hbl_forward runs): the quantizer, the weight widening and the GEMM."""
     M, K = x.shape
     dev = x.device
     sc = torch.empty((M,), dtype=torch.float32, device=dev)
-    if packed_route(M, bits):
-        q = torch.empty((M, K // 2), dtype=torch.uint8, device=dev)
-        stages = [lambda: hbl.hbl_fht_quant(x, 4, codes=q, scales=sc), None,
-                  lambda: hbl.hbl_gemm_tern_dequant(q, packed, sc, alpha, y=y)]
-    else:
-        q = torch.empty((M, K), dtype=torch.int8, device=dev)
-        Wi = torch.empty((N, K), dtype=torch.int8, device=dev)
-        stages = [lambda: hbl.hbl_fht_quant_i8(x, bits, codes=q, scales=sc),
-                  lambda: hbl.hbl_widen_ternary(packed, K, w=Wi),
-                  lambda: hbl.hbl_gemm_dequant(q, Wi, sc, alpha, y=y)]
+    q = torch.empty((M, K), dtype=torch.int8, device=dev)
+    Wi = torch.empty((N, K), dtype=torch.int8, device=dev)
+    stages = [lambda: hbl.hbl_fht_quant_i8(x, bits, codes=q, scales=sc),
+              lambda: hbl.hbl_widen_ternary(packed, K, w=Wi),
+              lambda: hbl.hbl_gemm_dequant(q, Wi, sc, alpha, y=y)]
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(n)]
     for _ in range(3):
         for f in stages:
-            if f is not None:
-                f()
+            f()
     torch.cuda.synchronize()
     for i in range(n):
         for j, f in enumerate(stages):
             evs[i][j].record(stream)
-            if f is not None:
-                f()
+            f()
         evs[i][3].record(stream)
     torch.cuda.synchronize()
     t_k1 = statistics.mean(e[0].elapsed_time(e[1]) for e in evs) / 1e3
@@ -498,10 +484,9 @@ def stage_graph_times(torch, hbl, x, packed, alpha, N, bits, y, n):
 
 
 def k1_bytes_of(M, K, x_bytes, bits):
-    """Algorithmic bytes of the forward's quantizer launch: x read, codes and scales written
-    (packed INT4 nibbles on the packed route, one byte per code otherwise)."""
-    codes = M * K // 2 if packed_route(M, bits) else M * K
-    return M * K * x_bytes + codes + 4 * M
+    """Algorithmic bytes of the forward's quantizer launch: x read, codes (one int8 per
+    element, the GEMM's operand) and scales written."""
+    return M * K * x_bytes + M * K + 4 * M
 
 
 def config_numbers(torch, hbl, wl, bits, peaks, int8_peak, stream, x=None, packed=None, alpha=None):
@@ -660,9 +645,7 @@ def bench_ours(args):
     achieved_tops = ops / t_gm / 1e12
     k1_bytes = k1_bytes_of(M, K, 2 if wl.dtype == "bf16" else 4, bits)
     k1_gbs = k1_bytes / t_k1 / 1e9
-    gemm_kernel = ("gemm_tern_pair_kernel (packed INT4 codes and 2-bit weights widened in shared memory; tcgen05 "
-                   "kind::i8, cta_group::2, dequant epilogue)" if packed_route(M, bits) else
-                   "gemm_i8_2sm_kernel (tcgen05 kind::i8, cta_group::2, dequant epilogue)")
+    gemm_kernel = "gemm_i8_2sm_kernel (tcgen05 kind::i8, cta_group::2, dequant epilogue)"
     roofline = {"bound": "tensor", "kernel": gemm_kernel,
                 "achieved": achieved_tops, "peak": int8_peak, "unit": "TFLOP/s", "frac": achieved_tops / int8_peak,
                 "traffic": measured_traffic("gemm_7b_wdown"),
@@ -676,7 +659,7 @@ def bench_ours(args):
     if roofline["frac"] > 1.0:
         roofline["peak_suspect"] = "achieved above the peak: the denominator does not bound this kernel"
     k1 = {"bound": "hbm", "kernel": "ln_fht_quant_tc_kernel (tcgen05 high Hadamard factor; INT%d, %s out)"
-          % (bits, "packed nibbles" if packed_route(M, bits) else "int8 codes"), "achieved": k1_gbs,
+          % (bits, "int8 codes"), "achieved": k1_gbs,
           "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": k1_gbs / peaks["hbm_gbs"],
           "traffic": measured_traffic("k1_7b_wdown"),
           "algorithmic_bytes_per_launch": k1_bytes, "launch_ms": t_k1 * 1e3}
