@@ -32,7 +32,11 @@ def test_check_t_rejects_a_relative_error_above_1e_5():
 def test_check_t_rejects_one_wrong_element():
     t64 = _t_rows()
     bad = t64.astype(np.float32)
-    bad[1, 5] += np.float32(1e-3)               # above 1e-5 rms(t) + 4 ulp of the element
+    # 1e-4 keeps the row within 1e-5 of its norm (16) but is far above the
+    # element's bound, 1e-5 rms(t) + 4 ulp: only the elementwise rule fails
+    bad[1, 5] += np.float32(1e-4)
+    d = bad.astype(np.float64) - t64
+    assert np.linalg.norm(d[1]) <= 1e-5 * np.linalg.norm(t64[1])
     with pytest.raises(AssertionError):
         check_t(bad, t64)
 
