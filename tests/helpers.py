@@ -52,7 +52,7 @@ def check_t(t_gpu, t64, rel=1e-5):
     nz = nrm > 0
     assert np.all(np.linalg.norm(d, axis=1)[nz] <= rel * nrm[nz]), np.max(np.linalg.norm(d, axis=1)[nz] / nrm[nz])
     bound = rel * rms[:, None] + T_ELEM_ULP * np.abs(t64)
-    assert np.all((np.abs(d) <= bound)[nz]), np.max((np.abs(d) / bound)[nz])
+    assert np.all((np.abs(d) <= bound)[nz]), np.max(np.abs(d)[nz] / bound[nz])
     assert np.all(np.abs(t_gpu[~nz]) == 0)
 
 
