@@ -296,6 +296,49 @@ def test_quant_rounds_the_exact_product(orc, bits):
     assert differ >= 4
 
 
+_WORKLOAD_T = {}
+
+
+def _workload_t(orc, name, rows):
+    """The oracle's float t of some rows of a workload (cached across tests)."""
+    from ternary_gemm_b200.inputs import WORKLOADS, make_x_rows
+    if name not in _WORKLOAD_T:
+        _WORKLOAD_T[name] = orc.ln_fht(make_x_rows(WORKLOADS[name], rows))[1]
+    return _WORKLOAD_T[name]
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+def test_reciprocal_reading_against_the_literal_division(orc, bits):
+    """The reading (one float reciprocal r = c / (stat + eps) per row, then rint
+    of the exact product t r) against the literal per-element form
+    rint(c t / (stat + eps)), evaluated in double, on the 7B workload's rows and
+    the sweep's: at least 99.99% of the codes agree, and every difference is one
+    step at a value within the reciprocal's rounding (2^-22 relative) of a
+    half-integer."""
+    c = float(f32(math.sqrt(7.0))) if bits == 4 else 127.0
+    lo, hi = (-8, 7) if bits == 4 else (-128, 127)
+    total = differ = 0
+    for name, rows in (("wdown_7b", np.arange(0, 1024, 64)), ("sweep", np.arange(64))):
+        t = _workload_t(orc, name, rows)
+        q, _ = orc.quant(t, bits)
+        t64 = t.astype(np.float64)
+        if bits == 4:
+            stat = np.abs(t64).sum(axis=1) / t.shape[1]
+            stat = stat.astype(np.float32).astype(np.float64)
+        else:
+            stat = np.abs(t64).max(axis=1)
+        v = c * t64 / (stat + float(f32(1e-5)))[:, None]
+        lit = np.clip(np.rint(v), lo, hi)
+        bad = lit != q
+        total += q.size
+        differ += int(bad.sum())
+        if bad.any():
+            assert np.all(np.abs(lit[bad] - q[bad]) == 1)
+            frac = np.abs(v[bad] - np.floor(v[bad]) - 0.5)
+            assert np.all(frac <= np.abs(v[bad]) * 2.0 ** -22)
+    assert differ <= 1e-4 * total, (differ, total)
+
+
 @pytest.mark.parametrize("bits", [4, 8])
 def test_quant_code_ranges(orc, bits):
     rng = np.random.default_rng(bits)
