@@ -1,0 +1,40 @@
+"""The fused LN -> Hadamard -> quantize path on every row of every workload (the
+full-size tests elsewhere sample rows): the transform output of each row within
+the path's 1e-5 tolerance of the oracle's double result, and the codes and scales
+of each row, packed and int8-widened, bit for bit against the oracle's quantizer
+applied to the kernel's own t."""
+import numpy as np
+import pytest
+
+from helpers import check_codes_exact, check_t, to_device, to_host, unpack_nibbles
+from ternary_gemm_b200.inputs import WORKLOADS, make_x
+
+pytestmark = [pytest.mark.gpu, pytest.mark.slow]
+
+
+@pytest.fixture(scope="module")
+def H():
+    import torch
+    from ternary_gemm_b200 import build
+    assert torch.cuda.is_available()
+    build.build()
+    import ternary_gemm_b200 as hbl
+    return hbl
+
+
+@pytest.mark.parametrize("name", ["tiny", "wo_1p3b", "wdown_3b", "wdown_7b"])
+def test_k1_every_row(H, orc, name):
+    wl = WORKLOADS[name]
+    x = make_x(wl)
+    xd = to_device(x)
+    t = to_host(H.hbl_debug_ln_fht(xd))
+    t64, _ = orc.ln_fht(x)
+    check_t(t, t64)
+    del t64
+    for bits in wl.bits:
+        qt, st = orc.quant(t, bits)
+        codes, scales = H.hbl_fht_quant(xd, bits)
+        q = to_host(codes)
+        check_codes_exact(unpack_nibbles(q, wl.K) if bits == 4 else q, to_host(scales), qt, st)
+        codes_i8, scales_i8 = H.hbl_fht_quant_i8(xd, bits)
+        check_codes_exact(to_host(codes_i8), to_host(scales_i8), qt, st)
