@@ -299,11 +299,11 @@ def test_quant_rounds_the_exact_product(orc, bits):
 _WORKLOAD_T = {}
 
 
-def _workload_t(orc, name, rows):
-    """The oracle's float t of some rows of a workload (cached across tests)."""
-    from ternary_gemm_b200.inputs import WORKLOADS, make_x_rows
+def _workload_t(orc, name):
+    """The oracle's float t of 64 rows drawn by a workload's recipe (cached)."""
+    from ternary_gemm_b200.inputs import WORKLOADS, make_x
     if name not in _WORKLOAD_T:
-        _WORKLOAD_T[name] = orc.ln_fht(make_x_rows(WORKLOADS[name], rows))[1]
+        _WORKLOAD_T[name] = orc.ln_fht(make_x(WORKLOADS[name].with_rows(64)))[1]
     return _WORKLOAD_T[name]
 
 
@@ -311,15 +311,16 @@ def _workload_t(orc, name, rows):
 def test_reciprocal_reading_against_the_literal_division(orc, bits):
     """The reading (one float reciprocal r = c / (stat + eps) per row, then rint
     of the exact product t r) against the literal per-element form
-    rint(c t / (stat + eps)), evaluated in double, on the 7B workload's rows and
-    the sweep's: at least 99.99% of the codes agree, and every difference is one
+    rint(c t / (stat + eps)), evaluated in double, on 64 rows of the 7B
+    workload's recipe and 64 of the sweep's: at least 99.99% of the codes agree,
+    and every difference is one
     step at a value within the reciprocal's rounding (2^-22 relative) of a
     half-integer."""
     c = float(f32(math.sqrt(7.0))) if bits == 4 else 127.0
     lo, hi = (-8, 7) if bits == 4 else (-128, 127)
     total = differ = 0
-    for name, rows in (("wdown_7b", np.arange(0, 1024, 64)), ("sweep", np.arange(64))):
-        t = _workload_t(orc, name, rows)
+    for name in ("wdown_7b", "sweep"):
+        t = _workload_t(orc, name)
         q, _ = orc.quant(t, bits)
         t64 = t.astype(np.float64)
         if bits == 4:
