@@ -125,3 +125,32 @@ def test_traffic_record_follows_its_sources(tmp_path, monkeypatch):
     assert bench.measured_traffic("other") is None
     src.write_text("// kernel v2\n")
     assert bench.measured_traffic("k") is None
+
+
+def test_profile_commands_use_current_options():
+    """Every bench.py command quoted in profiles/*.md (indented command lines,
+    with their backslash continuations) parses with bench.py's present options,
+    and names only workloads that exist."""
+    import glob
+    import re
+    import shlex
+    from ternary_gemm_b200.inputs import WORKLOADS
+    found = 0
+    for path in glob.glob(os.path.join(ROOT, "profiles", "*.md")):
+        lines = open(path).read().split("\n")
+        i = 0
+        while i < len(lines):
+            line = lines[i]
+            if line.startswith("    ") and "bench.py" in line:
+                cmd = re.split(r"\s{2,}\(", line.strip())[0]          # a trailing "(aside)" is prose
+                while cmd.endswith("\\") and i + 1 < len(lines):
+                    i += 1
+                    cmd = cmd[:-1] + " " + lines[i].strip()
+                words = shlex.split(cmd)
+                k = max(j for j, w in enumerate(words) if w.endswith("bench.py"))
+                args = [w for w in words[k + 1:] if not re.match(r"^[>|&]|^\d?>", w)]
+                a = bench.parse_args(args)
+                assert a.workload in WORKLOADS, (path, cmd)
+                found += 1
+            i += 1
+    assert found >= 5
