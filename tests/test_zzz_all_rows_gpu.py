@@ -14,6 +14,16 @@ from ternary_gemm_b200.inputs import WORKLOADS, make_x
 pytestmark = [pytest.mark.gpu, pytest.mark.slow]
 
 
+_X = {}
+
+
+def _x(name):
+    """A workload's activations, generated once for both tests of this module."""
+    if name not in _X:
+        _X[name] = make_x(WORKLOADS[name])
+    return _X[name]
+
+
 @pytest.fixture(scope="module")
 def H():
     import torch
@@ -27,7 +37,7 @@ def H():
 @pytest.mark.parametrize("name", ["tiny", "wo_1p3b", "wdown_3b", "wdown_7b"])
 def test_k1_every_row(H, orc, name):
     wl = WORKLOADS[name]
-    x = make_x(wl)
+    x = _x(name)
     xd = to_device(x)
     t = to_host(H.hbl_debug_ln_fht(xd))
     t64, _ = orc.ln_fht(x)
@@ -50,7 +60,7 @@ def test_forward_258_rows_full_n(H, orc, name):
     import torch
     from ternary_gemm_b200.inputs import make_w, sample_rows
     wl = WORKLOADS[name]
-    x, W = make_x(wl), make_w(wl)
+    x, W = _x(name), make_w(wl)
     xd = to_device(x)
     packed, alpha = H.hbl_pack_ternary(to_device(W))
     w, a = orc.ternary(W)
