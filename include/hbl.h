@@ -348,7 +348,11 @@ hbl_status hbl_gemm_i8_i32(const int8_t* A, const int8_t* B, int64_t M, int64_t 
 
 /* Synchronises `stream`, then reports and clears the device error word that
  * kernels set when a bounded wait runs out: HBL_ERR_TIMEOUT if one did,
- * HBL_ERR_CUDA if the synchronisation failed, else HBL_OK. */
+ * HBL_ERR_CUDA if the synchronisation failed, else HBL_OK.  The word is one
+ * per device, shared by every stream and host thread that uses the library
+ * there: a timeout is reported to the first caller that reads it after the
+ * kernel that set it has run (work still running on other streams is not
+ * waited for). */
 hbl_status hbl_last_device_error(cudaStream_t stream);
 
 /* Sets the device error word as a kernel would on a bounded-wait timeout
