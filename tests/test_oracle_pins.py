@@ -590,3 +590,28 @@ def test_fht_rows_matches_scipy(orc):
     t64, t32 = orc.fht_rows(x)
     np.testing.assert_allclose(t64, x.astype(np.float64) @ scipy.linalg.hadamard(64).T / 8.0, atol=1e-12)
     assert np.array_equal(t32, t64.astype(np.float32))
+
+
+def test_ternary_rotated_is_the_rotation_then_ternary(orc):
+    """Weights rotated along K by scipy's Hadamard matrix over sqrt(K), then the
+    pinned ternarization: integer-valued weights over a power of two keep every
+    rotated value exact, so codes and alpha must be identical."""
+    rng = np.random.default_rng(13)
+    K = 256
+    W = (rng.integers(-50, 51, (16, K)) * 2.0 ** -6).astype(np.float32)
+    Wr = (W.astype(np.float64) @ scipy.linalg.hadamard(K).astype(np.float64).T / math.sqrt(K)).astype(np.float32)
+    w, a = orc.ternary_rotated(W)
+    w2, a2 = orc.ternary(Wr)
+    assert a == a2 and np.array_equal(w, w2)
+
+
+def test_bf16_inputs_read_as_torch_reads_them(orc):
+    import torch
+    rng = np.random.default_rng(14)
+    bits = rng.integers(0, 1 << 16, 4096, dtype=np.uint32).astype(np.uint16)
+    bits = bits[(bits & 0x7F80) != 0x7F80]                         # finite values only
+    want = torch.from_numpy(bits.view(np.int16).copy()).view(torch.bfloat16).float().numpy()
+    assert np.array_equal(orc.bf16_bits_to_float(bits).view(np.uint32), want.view(np.uint32))
+    assert np.array_equal(orc.input_as_float64(bits), want.astype(np.float64))
+    f = rng.standard_normal(100).astype(np.float32)
+    assert np.array_equal(orc.input_as_float64(f), f.astype(np.float64))
