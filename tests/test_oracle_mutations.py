@@ -118,6 +118,8 @@ PY_MUTANTS = [
     ("weight gradient without the scales",
      "a = np.asarray(codes, dtype=np.float64) * np.asarray(scales, dtype=np.float64)[:, None]",
      "a = np.asarray(codes, dtype=np.float64)"),
+    ("rotated ternarization without the rotation", "    _, w32 = fht_rows(W)\n    return ternary(w32)",
+     "    w32 = np.asarray(W, dtype=np.float32)\n    return ternary(w32)"),
     ("KV dequant without the doubling", "return (2.0 * np.asarray(codes, np.float64) - L)",
      "return (np.asarray(codes, np.float64) - L)"),
     ("KV dequant over 2^b", "L = float((1 << bits) - 1)\n    return", "L = float(1 << bits)\n    return"),
