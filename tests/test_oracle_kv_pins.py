@@ -12,6 +12,8 @@ import os
 import numpy as np
 import pytest
 
+from near_ties import _kv_planted
+
 GOLD = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "hand_examples.json")))
 
 
@@ -82,40 +84,6 @@ def test_kv_dequant_error_bound_and_end_levels(orc, bits):
     for m in range(x.shape[0]):
         i = int(np.argmax(np.abs(x[m])))
         assert xr[m, i] == np.float64(x[m, i])
-
-
-def _kv_planted(bits, g=1.0, spread=64):
-    """Values x whose code under the reading's float steps, rint(fl(fl(x r) + L/2))
-    with ties to even, differs from a rounding of the exact x r + L/2, from the
-    fused fl(x r + L/2), or from rounding half away from zero, for a head whose
-    max |x| is g.  Returns (x values, r, the three counts of differences)."""
-    from fractions import Fraction
-    f32 = np.float32
-    L = f32((1 << bits) - 1)
-    half = f32(0.5) * L
-    r = f32(L / f32(f32(2.0) * f32(f32(g) + f32(1e-5))))
-    picked, n_exact, n_fused, n_away = [], 0, 0, 0
-    for k in range(int(L)):
-        x0 = f32((k + 0.5 - float(half)) / float(r))
-        for d in range(-spread, spread + 1):
-            x = f32(x0 + d * np.spacing(max(abs(x0), f32(1e-30))))
-            if abs(x) >= g:
-                continue
-            u = f32(f32(x * r) + half)
-            q = int(np.rint(u))
-            ex = Fraction(float(x)) * Fraction(float(r)) + Fraction(float(half))
-            fu = float(np.float32(float(ex)))                  # double first: checked below against exact
-            if abs(Fraction(fu) - ex) > abs(Fraction(float(np.nextafter(f32(fu), f32(np.inf)))) - ex) or \
-               abs(Fraction(fu) - ex) > abs(Fraction(float(np.nextafter(f32(fu), f32(-np.inf)))) - ex):
-                continue                                       # skip the rare double-rounding case
-            e_q, f_q = round(ex), int(np.rint(f32(fu)))
-            a_q = int(np.floor(float(u) + 0.5))
-            if e_q != q or f_q != q or a_q != q:
-                picked.append(x)
-                n_exact += e_q != q
-                n_fused += f_q != q
-                n_away += a_q != q
-    return np.array(picked, np.float32), r, (n_exact, n_fused, n_away)
 
 
 @pytest.mark.parametrize("bits", [3, 8])

@@ -16,6 +16,8 @@ import numpy as np
 import pytest
 import scipy.linalg
 
+from near_ties import _near_ties, _nearest_f32, _row_reciprocal, _row_stat_int4, _steer_mean_row
+
 GOLD = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "hand_examples.json")))
 f32 = np.float32
 
@@ -143,17 +145,6 @@ def test_quant_int4_hand(orc):
     assert s[0] == f32(g["scale"])
 
 
-def _nearest_f32(fr):
-    """The float32 nearest to a rational number, ties to even (exact comparisons)."""
-    from fractions import Fraction
-    b = f32(float(fr))
-    cands = [np.nextafter(b, f32(-np.inf)), b, np.nextafter(b, f32(np.inf))]
-    dist = [abs(Fraction(float(c)) - fr) for c in cands]
-    best = min(dist)
-    ties = [c for c, d in zip(cands, dist) if d == best]
-    return next((c for c in ties if int(np.array(c, np.float32).view(np.uint32)) % 2 == 0), ties[0])
-
-
 def test_int4_scale_is_the_exactly_rounded_mean(orc):
     """The absmean's reduction (a double sum of |t|, rounded once to float)
     against the plain definition computed exactly: the mean of |t| as a
@@ -215,56 +206,6 @@ def test_quant_round_half_to_even(orc, bits, target, want):
     row = _tie_input(bits, target)
     q, _ = orc.quant(row[None, :], bits)
     assert q[0, 1] == want
-
-
-def _steer_mean_row(rest, R, c):
-    """Prepend to `rest` an element a (walked one ulp at a time) such that the
-    reciprocal fl(c / fl(mean|.| + eps)) of the whole array, its mean of
-    absolute values rounded once to float, is exactly R."""
-    d0 = f32(c / R)
-    dens = [d for d in (np.nextafter(np.nextafter(d0, f32(-np.inf)), f32(-np.inf)), np.nextafter(d0, f32(-np.inf)),
-                        d0, np.nextafter(d0, f32(np.inf)), np.nextafter(np.nextafter(d0, f32(np.inf)), f32(np.inf)))
-            if f32(c / d) == R]
-    assert dens, "no denominator gives R"
-    den = dens[len(dens) // 2]
-    K = len(rest) + 1
-    a = f32(K * (float(den) - 1e-5) - float(np.abs(rest.astype(np.float64)).sum()))
-    for _ in range(2000):
-        row = np.concatenate([[a], rest]).astype(np.float32)
-        s = f32(_row_stat_int4(row) + f32(1e-5))
-        if s == den:
-            return row
-        a = np.nextafter(a, f32(-np.inf) if s > den else f32(np.inf))
-    raise RuntimeError("statistic not reached")
-
-
-def _row_stat_int4(row):
-    from fractions import Fraction
-    return _nearest_f32(sum(Fraction(float(v)) for v in np.abs(row)) / len(row))
-
-
-def _row_reciprocal(row, bits):
-    """r = fl(c / fl(stat + eps)) of one row, the statistic from its definition
-    (exact mean of |t| rounded to float, or max |t|)."""
-    c = f32(math.sqrt(7.0)) if bits == 4 else f32(127.0)
-    stat = _row_stat_int4(row) if bits == 4 else f32(np.abs(row).max())
-    return f32(c / f32(stat + f32(1e-5)))
-
-
-def _near_ties(r, limit):
-    """Floats t just off (k + 1/2) / r, k < limit, whose product with r is not a
-    half-integer but rounds in float to one: rint of the exact product and rint
-    of the float-rounded product differ for them."""
-    from fractions import Fraction
-    out = []
-    for k in range(limit):
-        for sgn in (1.0, -1.0):
-            t0 = f32(sgn * (k + 0.5) / float(r))
-            for t in (np.nextafter(t0, f32(-np.inf)), t0, np.nextafter(t0, f32(np.inf))):
-                exact = Fraction(float(t)) * Fraction(float(r))
-                if exact.denominator != 2 and f32(t * r) == f32(sgn * (k + 0.5)):
-                    out.append(t)
-    return np.array(out, np.float32)
 
 
 @pytest.mark.parametrize("bits", [4, 8])

@@ -12,8 +12,7 @@ import numpy as np
 import pytest
 
 from helpers import check_codes_exact, to_device, to_host, unpack_nibbles
-from test_oracle_kv_pins import _kv_planted
-from test_oracle_pins import _near_ties, _row_reciprocal, _steer_mean_row
+from near_ties import _kv_planted, _near_ties, _row_reciprocal, _steer_mean_row
 
 pytestmark = pytest.mark.gpu
 
