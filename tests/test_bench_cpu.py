@@ -154,3 +154,25 @@ def test_profile_commands_use_current_options():
                 found += 1
             i += 1
     assert found >= 5
+
+
+def test_traffic_record_sources_cover_the_kernels_includes():
+    """Each DRAM-traffic record digests its kernel file and every library
+    header that file includes, directly or not, so any change to the compiled
+    kernel withdraws the record."""
+    import re
+    csrc = os.path.join(ROOT, "ternary_gemm_b200", "csrc")
+
+    def closure(f, seen):
+        p = os.path.join(csrc, f)
+        if f in seen or not os.path.exists(p):
+            return seen
+        seen.add(f)
+        for inc in re.findall(r'#include\s+"([^"]+)"', open(p).read()):
+            closure(inc, seen)
+        return seen
+
+    rec = json.load(open(os.path.join(ROOT, "profiles", "traffic.json")))
+    for key, kernel_file in (("gemm_7b_wdown", "gemm_i8.cu"), ("k1_7b_wdown", "fht_quant_tc.cu")):
+        have = {os.path.basename(p) for p in rec[key]["sources"]}
+        assert closure(kernel_file, set()) <= have, key
