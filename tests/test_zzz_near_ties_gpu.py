@@ -1,11 +1,11 @@
 """Near ties on the GPU: the quantizer (hbl_quant_from_f32, the arithmetic every
 fused quantizer shares), the ternary packing (hbl_pack_ternary) and the
-QKV-state quantizer (hbl_kv_quant) on inputs
-planted with values whose product with the row's (or tensor's) reciprocal r
-lies within half a float ulp of a rounding boundary, so that rint of the exact
-product and rint of its float rounding differ.  Codes, scales and alpha must be
-the oracle's bit for bit; the oracle's own rounding of the exact product is
-pinned on the CPU (tests/test_oracle_pins.py) with the same constructions."""
+QKV-state quantizer (hbl_kv_quant) on inputs planted with values whose product
+with the row's (or tensor's) reciprocal r lies within half a float ulp of a
+rounding boundary, so that rint of the exact product and rint of its float
+rounding differ.  Codes, scales and alpha must be the oracle's bit for bit; the
+oracle's own rounding is pinned on the CPU (tests/test_oracle_pins.py,
+tests/test_oracle_kv_pins.py) with the same constructions (tests/near_ties.py)."""
 import math
 
 import numpy as np
